@@ -1,0 +1,445 @@
+"""Pins of the CPU oracle against what the SAS paper and the mathematics fix.
+
+None of these tests uses a GPU. Each pin is something other than the oracle
+itself: hand-derived worked examples, closed forms, invariants, special cases
+that reduce to torch's scaled_dot_product_attention / log_softmax / autograd,
+brute force on tiny inputs, and central finite differences.
+"""
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import sas_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def _val(expr: str) -> float:
+    expr = expr.strip()
+    if expr.startswith("ln"):
+        inner = expr[2:].strip().strip("()")
+        return math.log(float(Fraction(inner)))
+    return float(Fraction(expr))
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _selection_inputs(B=1, Hq=2, Hkv=1, T=256, d=16, block=64, K=3, seed=0, s_scale=1.0):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((B, Hq, T, d))
+    Kt = rng.standard_normal((B, Hkv, T, d))
+    V = rng.standard_normal((B, Hkv, T, d))
+    dO = rng.standard_normal((B, Hq, T, d))
+    NB = T // block
+    s = s_scale * rng.standard_normal((B, Hkv, T, NB))
+    logG = orc.gate_normalize(s, block)
+    tau, tidx, sel = orc.select_threshold(logG, K, block)
+    return Q, Kt, V, dO, s, logG, tau, tidx, sel
+
+
+# ---------------------------------------------------------------- worked examples
+@pytest.mark.parametrize("case_idx", [0, 1, 2])
+def test_worked_example(case_idx):
+    gold = json.load(open(GOLDEN))
+    case = gold["cases"][case_idx]
+    block, T = gold["block"], gold["T"]
+    NB = T // block
+    s = np.zeros((1, 1, T, NB))
+    for r, vals in case["s_rows"].items():
+        s[0, 0, int(r)] = vals
+    logG = orc.gate_normalize(s, block)
+    tau, tidx, _ = orc.select_threshold(logG, case["K"], block)
+    Q = np.zeros((1, 1, T, 1))
+    Kt = np.ones((1, 1, T, 1))
+    V = np.asarray(gold["v"], float).reshape(1, 1, T, 1)
+    dO = np.asarray(case["dO"], float).reshape(1, 1, T, 1)
+    out = orc.forward_backward(Q, Kt, V, dO, logG, tau, tidx, block, 1.0)
+    np.testing.assert_allclose(out["O"][0, 0, :, 0], [_val(x) for x in case["O"]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["LSE"][0, 0], [_val(x) for x in case["LSE"]], rtol=0, atol=1e-12)
+    if "dLogG_row4" in case:
+        np.testing.assert_allclose(out["dLogG"][0, 0, 4], [_val(x) for x in case["dLogG_row4"]], atol=1e-12)
+        np.testing.assert_allclose(out["dV"][0, 0, :, 0], [_val(x) for x in case["dV"]], atol=1e-12)
+        np.testing.assert_allclose(out["dQ"][0, 0, 4, 0], _val(case["dQ_row4"]), atol=1e-12)
+        others = np.delete(out["dLogG"][0, 0], 4, axis=0)
+        assert np.all(others == 0.0)
+
+
+# ---------------------------------------------------------------- gate normalisation
+def test_normalize_matches_log_softmax_prefix():
+    block, T = 16, 160
+    s = _rand((2, 3, T, T // block), 1)
+    logG = orc.gate_normalize(s, block)
+    st = torch.from_numpy(s)
+    for t in range(T):
+        c = t // block
+        assert np.all(np.isneginf(logG[:, :, t, c:]))
+        if c:
+            ref = F.log_softmax(st[:, :, t, :c], dim=-1).numpy()
+            np.testing.assert_allclose(logG[:, :, t, :c], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_normalize_shift_invariance_and_unit_mass():
+    block, T = 8, 96
+    s = _rand((1, 2, T, T // block), 2) * 3
+    a = orc.gate_normalize(s, block)
+    b = orc.gate_normalize(s + 123.25, block)
+    fin = np.isfinite(a)
+    np.testing.assert_allclose(a[fin], b[fin], atol=1e-11)
+    for t in range(block, T):
+        c = t // block
+        np.testing.assert_allclose(np.exp(a[:, :, t, :c]).sum(-1), 1.0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- top-k threshold
+def _brute_force_topk(vals, c, H):
+    """The unique H-subset whose every member beats every non-member under
+    (value descending, index ascending); found by enumerating all subsets."""
+    if min(c, H) == 0:
+        return []
+    if c <= H:
+        return list(range(c))
+
+    def beats(a, b):
+        return vals[a] > vals[b] or (vals[a] == vals[b] and a < b)
+
+    found = [sub for sub in itertools.combinations(range(c), H)
+             if all(beats(a, b) for a in sub for b in range(c) if b not in sub)]
+    assert len(found) == 1
+    return list(found[0])
+
+
+@pytest.mark.parametrize("H", [0, 1, 2, 3, 5])
+def test_select_brute_force_with_ties(H):
+    rng = np.random.default_rng(H)
+    for trial in range(150):
+        c = int(rng.integers(0, 9))
+        vals = rng.integers(-2, 3, size=9).astype(np.float64)   # many ties
+        if trial % 3 == 0:
+            vals[rng.integers(0, 9)] = -0.0
+            vals[rng.integers(0, 9)] = 0.0
+        tau, tidx, chosen = orc.topk_threshold_row(vals, c, H)
+        assert chosen == _brute_force_topk(vals, c, H)
+        # The threshold pair reproduces the chosen set through the predicate.
+        pred = [m for m in range(c) if vals[m] > tau or (vals[m] == tau and m <= tidx)]
+        assert pred == chosen
+
+
+def test_select_matches_lexsort_and_mask():
+    block, T, K = 16, 256, 5
+    s = _rand((2, 2, T, T // block), 3)
+    logG = orc.gate_normalize(s, block).astype(np.float32).astype(np.float64)
+    tau, tidx, sel = orc.select_threshold(logG, K, block)
+    mask = orc.selection_mask(logG, tau, tidx, block)
+    for b in range(2):
+        for g in range(2):
+            for t in range(T):
+                c = t // block
+                vals = logG[b, g, t, :c]
+                ref = sorted(np.lexsort((np.arange(c), -vals))[: K - 1].tolist()) if c else []
+                got = [m for m in sel[b, g, t] if m >= 0]
+                assert got == ref
+                assert np.flatnonzero(mask[b, g, t]).tolist() == ref
+
+
+def test_select_signed_zero_ties():
+    vals = np.array([0.0, -0.0, 0.0, -1.0, -0.0])
+    tau, tidx, chosen = orc.topk_threshold_row(vals, 5, 2)
+    assert chosen == [0, 1] and tau == 0.0 and tidx == 1
+
+
+# ---------------------------------------------------------------- forward special cases
+def _sdpa(Q, K, V, mask, sm_scale, G):
+    q = torch.from_numpy(Q)
+    k = torch.from_numpy(K).repeat_interleave(G, dim=1)
+    v = torch.from_numpy(V).repeat_interleave(G, dim=1)
+    return F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=sm_scale).numpy()
+
+
+def test_unit_gates_full_budget_is_dense_causal():
+    B, Hq, Hkv, T, d, block = 1, 4, 2, 192, 16, 32
+    rng = np.random.default_rng(4)
+    Q, K, V = rng.standard_normal((B, Hq, T, d)), rng.standard_normal((B, Hkv, T, d)), rng.standard_normal((B, Hkv, T, d))
+    logG = np.zeros((B, Hkv, T, T // block))        # unit gates
+    tau, tidx, _ = orc.select_threshold(logG, T // block, block)
+    O, LSE = orc.forward(Q, K, V, logG, tau, tidx, block, 0.25)
+    causal = torch.ones(T, T, dtype=torch.bool).tril()
+    np.testing.assert_allclose(O, _sdpa(Q, K, V, causal, 0.25, Hq // Hkv), atol=1e-12)
+    z = 0.25 * np.einsum("bhtd,bhsd->bhts", Q, np.repeat(K, 2, axis=1))
+    z = np.where(causal.numpy(), z, -np.inf)
+    np.testing.assert_allclose(LSE, torch.logsumexp(torch.from_numpy(z), -1).numpy(), atol=1e-12)
+
+
+def test_budget_one_is_current_block_only():
+    B, Hq, Hkv, T, d, block = 2, 2, 1, 128, 8, 16
+    Q, K, V, _, s, logG, _, _, _ = _selection_inputs(B, Hq, Hkv, T, d, block, 1, seed=5)
+    tau, tidx, _ = orc.select_threshold(logG, 1, block)
+    O, _ = orc.forward(Q, K, V, logG, tau, tidx, block, 0.3)
+    i = torch.arange(T)
+    mask = (i[:, None] >= i[None, :]) & (i[:, None] // block == i[None, :] // block)
+    np.testing.assert_allclose(O, _sdpa(Q, K, V, mask, 0.3, Hq), atol=1e-12)
+
+
+def test_uniform_scores_full_budget_is_causal_with_log_count_bias():
+    B, Hq, Hkv, T, d, block = 1, 2, 1, 160, 8, 32
+    rng = np.random.default_rng(6)
+    Q, K, V = rng.standard_normal((B, Hq, T, d)), rng.standard_normal((B, Hkv, T, d)), rng.standard_normal((B, Hkv, T, d))
+    s = np.full((B, Hkv, T, T // block), 0.7)
+    logG = orc.gate_normalize(s, block)
+    tau, tidx, _ = orc.select_threshold(logG, T // block, block)
+    O, _ = orc.forward(Q, K, V, logG, tau, tidx, block, 0.5)
+    i = np.arange(T)
+    c = i // block
+    # Uniform softmax gates: each of the c_t historical blocks has g = 1/c_t.
+    bias = np.where(i[None, :] // block < c[:, None], -np.log(np.maximum(c[:, None], 1)), 0.0)
+    bias = np.where(i[None, :] <= i[:, None], bias, -np.inf)
+    np.testing.assert_allclose(O, _sdpa(Q, K, V, torch.from_numpy(bias), 0.5, Hq), atol=1e-12)
+
+
+def test_materialised_equals_gathered_rows():
+    Q, K, V, dO, s, logG, tau, tidx, sel = _selection_inputs(1, 4, 2, 256, 16, 32, 3, seed=7)
+    full = orc.forward_backward(Q, K, V, dO, logG, tau, tidx, 32, 0.25)
+    for g in range(2):
+        rows = np.arange(0, 256, 7)
+        gat = orc.rows_gathered(Q, K, V, dO, logG, sel, 0, g, rows, 32, 0.25)
+        for hh in range(2):
+            h = g * 2 + hh
+            np.testing.assert_allclose(gat["O"][hh], full["O"][0, h, rows], atol=1e-12)
+            np.testing.assert_allclose(gat["LSE"][hh], full["LSE"][0, h, rows], atol=1e-12)
+            np.testing.assert_allclose(gat["dQ"][hh], full["dQ"][0, h, rows], atol=1e-12)
+        np.testing.assert_allclose(gat["dLogG"], full["dLogG"][0, g, rows], atol=1e-12)
+        for j in range(256 // 32):
+            dK, dV = orc.kv_block_gathered(Q, K, V, dO, logG, sel, 0, g, j, 32, 0.25)
+            np.testing.assert_allclose(dK, full["dK"][0, g, j * 32:(j + 1) * 32], atol=1e-11)
+            np.testing.assert_allclose(dV, full["dV"][0, g, j * 32:(j + 1) * 32], atol=1e-11)
+
+
+def test_row_subset_matches_full():
+    Q, K, V, dO, s, logG, tau, tidx, sel = _selection_inputs(1, 2, 1, 128, 8, 16, 3, seed=8)
+    full = orc.forward_backward(Q, K, V, dO, logG, tau, tidx, 16, 0.4)
+    rows = np.array([0, 15, 16, 17, 63, 100, 127])
+    sub = orc.forward_backward(Q, K, V, dO, logG, tau, tidx, 16, 0.4, rows=rows)
+    for k in ("O", "LSE", "dQ"):
+        np.testing.assert_allclose(sub[k], full[k][:, :, rows], atol=1e-13)
+    np.testing.assert_allclose(sub["dLogG"], full["dLogG"][:, :, rows], atol=1e-13)
+
+
+def test_attention_weights_bounded_and_lse_finite():
+    Q, K, V, dO, s, logG, tau, tidx, sel = _selection_inputs(1, 2, 1, 128, 8, 16, 2, seed=9, s_scale=4.0)
+    _, LSE = orc.forward(Q, K, V, logG, tau, tidx, 16, 3.0)
+    assert np.all(np.isfinite(LSE))
+    # p_i = exp(z_i - LSE) <= 1 (eq. 7): every logit is at most the row LSE.
+    mask = orc.selection_mask(logG, tau, tidx, 16)
+    for h in range(2):
+        z = 3.0 * Q[0, h] @ K[0, 0].T + orc.bias_rows(logG[0, 0], mask[0, 0], np.arange(128), 128, 16)
+        assert np.all(z <= LSE[0, h][:, None] + 1e-12)
+
+
+# ---------------------------------------------------------------- backward
+def _loss(Q, K, V, dO, logG, tau, tidx, block, sm):
+    O, _ = orc.forward(Q, K, V, logG, tau, tidx, block, sm)
+    return float((O * dO).sum())
+
+
+@pytest.mark.parametrize("Kbud", [2, 3])
+def test_backward_central_finite_differences(Kbud):
+    B, Hq, Hkv, T, d, block, sm = 1, 2, 1, 256, 16, 64, 0.25
+    Q, K, V, dO, s, logG, tau, tidx, sel = _selection_inputs(B, Hq, Hkv, T, d, block, Kbud, seed=10 + Kbud)
+    out = orc.forward_backward(Q, K, V, dO, logG, tau, tidx, block, sm)
+    rng = np.random.default_rng(Kbud)
+    eps = 1e-6
+
+    def fd(arr, idx):
+        old = arr[idx]
+        arr[idx] = old + eps
+        lp = _loss(Q, K, V, dO, logG, tau, tidx, block, sm)
+        arr[idx] = old - eps
+        lm = _loss(Q, K, V, dO, logG, tau, tidx, block, sm)
+        arr[idx] = old
+        return (lp - lm) / (2 * eps)
+
+    for name, arr, grad in (("Q", Q, out["dQ"]), ("K", K, out["dK"]), ("V", V, out["dV"])):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            assert abs(fd(arr, idx) - grad[idx]) < 1e-6 * max(1.0, abs(grad[idx])), name
+    # Selected log-gate entries, with the selected set held fixed: an entry that
+    # is the threshold itself carries tau along with it.
+    mask = orc.selection_mask(logG, tau, tidx, block)
+    picks = np.argwhere(mask)
+    assert len(picks) > 0
+
+    def fd_gate(idx):
+        row = idx[:3]
+        at_tau = logG[idx] == tau[row]
+        vals = []
+        for sgn in (1.0, -1.0):
+            old_g, old_t = logG[idx], tau[row]
+            logG[idx] = old_g + sgn * eps
+            if at_tau:
+                tau[row] = logG[idx]
+            assert np.array_equal(orc.selection_mask(logG, tau, tidx, block), mask)
+            vals.append(_loss(Q, K, V, dO, logG, tau, tidx, block, sm))
+            logG[idx], tau[row] = old_g, old_t
+        return (vals[0] - vals[1]) / (2 * eps)
+
+    for k in rng.choice(len(picks), size=min(10, len(picks)), replace=False):
+        idx = tuple(int(x) for x in picks[k])
+        assert abs(fd_gate(idx) - out["dLogG"][idx]) < 1e-6 * max(1.0, abs(out["dLogG"][idx]))
+    assert np.all(out["dLogG"][~mask] == 0.0)
+
+
+def test_backward_unit_gates_matches_autograd_causal_sdpa():
+    B, Hq, Hkv, T, d, block, sm = 1, 4, 2, 128, 8, 32, 0.35
+    rng = np.random.default_rng(11)
+    Q, K, V, dO = (rng.standard_normal(s) for s in ((B, Hq, T, d), (B, Hkv, T, d), (B, Hkv, T, d), (B, Hq, T, d)))
+    logG = np.zeros((B, Hkv, T, T // block))
+    tau, tidx, _ = orc.select_threshold(logG, T // block, block)
+    out = orc.forward_backward(Q, K, V, dO, logG, tau, tidx, block, sm)
+    q, k, v = (torch.from_numpy(a).requires_grad_() for a in (Q, K, V))
+    o = F.scaled_dot_product_attention(q, k.repeat_interleave(2, 1), v.repeat_interleave(2, 1), is_causal=True, scale=sm)
+    (o * torch.from_numpy(dO)).sum().backward()
+    np.testing.assert_allclose(out["dQ"], q.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(out["dK"], k.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(out["dV"], v.grad.numpy(), atol=1e-12)
+
+
+def test_gate_gradient_eq5_closed_form_and_zero_sum():
+    B, Hq, Hkv, T, d, block, sm = 1, 2, 1, 128, 8, 16, 0.5
+    Q, K, V, dO, s, logG, tau, tidx, sel = _selection_inputs(B, Hq, Hkv, T, d, block, 3, seed=12)
+    out = orc.forward_backward(Q, K, V, dO, logG, tau, tidx, block, sm)
+    mask = orc.selection_mask(logG, tau, tidx, block)
+    own_total = np.zeros(T)
+    for h in range(Hq):
+        z = sm * Q[0, h] @ K[0, 0].T + orc.bias_rows(logG[0, 0], mask[0, 0], np.arange(T), T, block)
+        p = np.exp(z - out["LSE"][0, h][:, None])
+        o = out["O"][0, h]
+        # eq. 5 (inner gate) times g_m: d log g_m = sum_{i in B_m} p_i do.(v_i - o)
+        w = p * (dO[0, h] @ V[0, 0].T - (dO[0, h] * o).sum(1, keepdims=True))
+        for t in range(T):
+            c = t // block
+            own_total[t] += w[t, c * block:t + 1].sum()
+    eq5 = np.zeros((T, T // block))
+    for h in range(Hq):
+        z = sm * Q[0, h] @ K[0, 0].T + orc.bias_rows(logG[0, 0], mask[0, 0], np.arange(T), T, block)
+        p = np.exp(z - out["LSE"][0, h][:, None])
+        o = out["O"][0, h]
+        for t in range(T):
+            for m in range(t // block):
+                if mask[0, 0, t, m]:
+                    sl = slice(m * block, (m + 1) * block)
+                    eq5[t, m] += (p[t, sl] * ((V[0, 0, sl] - o[t]) @ dO[0, h, t])).sum()
+    np.testing.assert_allclose(out["dLogG"][0, 0], eq5, atol=1e-12)
+    # sum_i dS_i = 0 per row: the selected blocks' gradients cancel the current block's.
+    np.testing.assert_allclose(out["dLogG"][0, 0].sum(1), -own_total, atol=1e-12)
+
+
+# ---------------------------------------------------------------- decode
+def test_decode_full_budget_is_dense_attention_and_topk_bruteforce():
+    B, Hq, Hkv, L, d, block = 3, 4, 2, 200, 16, 16
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal((B, Hq, d))
+    Kc, Vc = rng.standard_normal((B, Hkv, L, d)), rng.standard_normal((B, Hkv, L, d))
+    s = np.round(rng.standard_normal((B, Hkv, (L + block - 1) // block)), 1)   # rounded: ties happen
+    seqlen = np.array([200, 129, 17])
+    o, sel = orc.decode(q, Kc, Vc, seqlen, s, 100, block, 0.25)
+    for b in range(B):
+        Lb = int(seqlen[b])
+        ref = F.scaled_dot_product_attention(
+            torch.from_numpy(q[b][:, None]), torch.from_numpy(Kc[b, :, :Lb]).repeat_interleave(2, 0),
+            torch.from_numpy(Vc[b, :, :Lb]).repeat_interleave(2, 0), scale=0.25)[:, 0].numpy()
+        np.testing.assert_allclose(o[b], ref, atol=1e-12)
+    o, sel = orc.decode(q, Kc, Vc, seqlen, s, 4, block, 0.25)
+    for b in range(B):
+        c = (int(seqlen[b]) - 1) // block
+        for g in range(Hkv):
+            got = [m for m in sel[b, g] if m >= 0]
+            assert got == _brute_force_topk(s[b, g], c, 3)
+            keys = np.zeros(L, bool)
+            for m in got:
+                keys[m * block:(m + 1) * block] = True
+            keys[c * block:int(seqlen[b])] = True
+            ref = F.scaled_dot_product_attention(
+                torch.from_numpy(q[b, 2 * g:2 * g + 2][:, None]), torch.from_numpy(Kc[b, g][None].repeat(2, 0)),
+                torch.from_numpy(Vc[b, g][None].repeat(2, 0)), attn_mask=torch.from_numpy(keys)[None], scale=0.25)[:, 0].numpy()
+            np.testing.assert_allclose(o[b, 2 * g:2 * g + 2], ref, atol=1e-12)
+
+
+def test_decode_with_log_gate_equals_training_last_row():
+    B, Hq, Hkv, T, d, block, Kb = 1, 2, 1, 192, 8, 32, 3
+    rng = np.random.default_rng(14)
+    Q, K, V = rng.standard_normal((B, Hq, T, d)), rng.standard_normal((B, Hkv, T, d)), rng.standard_normal((B, Hkv, T, d))
+    s = rng.standard_normal((B, Hkv, T, T // block))
+    logG = orc.gate_normalize(s, block)
+    tau, tidx, _ = orc.select_threshold(logG, Kb, block)
+    O, _ = orc.forward(Q, K, V, logG, tau, tidx, block, 0.3)
+    o, _ = orc.decode(Q[:, :, T - 1], K, V, np.array([T]), s[:, :, T - 1], Kb, block, 0.3, apply_log_gate=True)
+    np.testing.assert_allclose(o, O[:, :, T - 1], atol=1e-12)
+
+
+# ---------------------------------------------------------------- the pins catch planted mistakes
+def _bad_normalize(s, block):
+    """Mistake: raw scores used as log-gates (the LSE is not subtracted)."""
+    out = np.full(np.shape(s), -np.inf)
+    for t in range(np.shape(s)[2]):
+        c = t // block
+        out[:, :, t, :c] = np.asarray(s, float)[:, :, t, :c]
+    return out
+
+
+def _bad_topk(vals, c, H):
+    """Mistake: ties broken toward the higher block index."""
+    if min(c, H) == 0:
+        return math.inf, -1, []
+    if c <= H:
+        return -math.inf, c - 1, list(range(c))
+    order = sorted(range(c), key=lambda m: (-float(vals[m]), -m))
+    taken = order[:H]
+    tau = float(vals[taken[-1]])
+    return tau, max(m for m in taken if float(vals[m]) == tau), sorted(taken)
+
+
+_good_bias = orc.bias_rows
+
+
+def _bad_bias_causal(logG_g, mask_g, rows, T, block):
+    """Mistake: the current block lets each query see one key past itself."""
+    b = _good_bias(logG_g, mask_g, rows, T, block)
+    rows = np.asarray(rows)
+    nxt = np.minimum(rows + 1, T - 1)
+    same = (nxt // block) == (rows // block)
+    b[np.arange(len(rows))[same], nxt[same]] = 0.0
+    return b
+
+
+def _bad_bias_sign(logG_g, mask_g, rows, T, block):
+    """Mistake: the log-gate enters the logits with the wrong sign."""
+    b = _good_bias(logG_g, mask_g, rows, T, block)
+    fin = np.isfinite(b) & (b != 0.0)
+    b[fin] = -b[fin]
+    return b
+
+
+@pytest.mark.parametrize("mistake,target", [
+    ("gate_normalize", lambda: test_worked_example(0)),
+    ("topk_threshold_row", lambda: test_worked_example(2)),
+    ("bias_causal", test_unit_gates_full_budget_is_dense_causal),
+    ("bias_sign", test_uniform_scores_full_budget_is_causal_with_log_count_bias),
+    ("bias_sign", lambda: test_worked_example(0)),
+])
+def test_pins_catch_planted_mistakes(monkeypatch, mistake, target):
+    bad = {"gate_normalize": ("gate_normalize", _bad_normalize),
+           "topk_threshold_row": ("topk_threshold_row", _bad_topk),
+           "bias_causal": ("bias_rows", _bad_bias_causal),
+           "bias_sign": ("bias_rows", _bad_bias_sign)}[mistake]
+    monkeypatch.setattr(orc, bad[0], bad[1])
+    with pytest.raises(AssertionError):
+        target()
