@@ -1,0 +1,226 @@
+"""ctypes binding of the SAS C ABI (``include/sas.h``).
+
+Argument marshalling only: every function takes torch tensors (device memory
+owned by the caller), checks that they are contiguous, and passes their
+pointers and sizes to the function of the same name in ``libsas_b200.so``.
+All arithmetic runs in the library's CUDA kernels; there is no fallback. If the
+library is missing, the first call raises ``RuntimeError``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
+_lib = None
+
+SAS_OK = 0
+SAS_DT_F32 = 0
+SAS_DT_BF16 = 1
+BLOCK = 64
+
+_c_int, _c_f, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+# name -> (restype, argtypes), mirroring include/sas.h
+_SIGNATURES = {
+    "sas_status_string": (ctypes.c_char_p, [_c_int]),
+    "sas_version": (_c_int, []),
+    "sas_launch_count": (ctypes.c_uint64, []),
+    "sas_gate_normalize": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "sas_fwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
+    "sas_bwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
+    "sas_decode_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
+    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_f, _vp, _sz, _vp]),
+    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 6
+                + [_c_f, _vp, _sz, _vp]),
+    "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
+                       + [_c_f, _vp, _sz, _vp]),
+    "sas_device_status": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
+    "sas_device_status_clear": (_c_int, [_vp, _vp]),
+}
+
+
+class SasError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {lib().sas_status_string(status).decode()} (status {status})")
+
+
+def lib():
+    """Load ``libsas_b200.so`` (once) and declare its signatures."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"SAS CUDA library not found at {_LIB_PATH}; build it with "
+                "`python -m gated_block_sparse_flashattention_b200.build`")
+        handle = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _check(fn: str, status: int):
+    if status != SAS_OK:
+        raise SasError(fn, status)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("SAS tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SAS_DT_F32
+    if t.dtype == torch.bfloat16:
+        return SAS_DT_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def launch_count() -> int:
+    return int(lib().sas_launch_count())
+
+
+def status_string(status: int) -> str:
+    return lib().sas_status_string(status).decode()
+
+
+def sas_gate_normalize(s, logG, block=BLOCK, stream=None):
+    B, Hkv, T, NB = s.shape
+    _check("sas_gate_normalize", lib().sas_gate_normalize(_ptr(s), _ptr(logG), B, Hkv, T, NB, block, _stream(stream)))
+
+
+def sas_select_threshold(logG, tau, tau_idx, sel, K, block=BLOCK, stream=None):
+    B, Hkv, T, NB = logG.shape
+    _check("sas_select_threshold", lib().sas_select_threshold(
+        _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
+
+
+def _ws_size(name, *args) -> int:
+    out = _sz(0)
+    _check(name, getattr(lib(), name)(*args, ctypes.byref(out)))
+    return out.value
+
+
+def sas_fwd_workspace_size(B, Hq, Hkv, T, d, dtype_code, block=BLOCK) -> int:
+    return _ws_size("sas_fwd_workspace_size", B, Hq, Hkv, T, d, block, dtype_code)
+
+
+def sas_bwd_workspace_size(B, Hq, Hkv, T, d, dtype_code, block=BLOCK) -> int:
+    return _ws_size("sas_bwd_workspace_size", B, Hq, Hkv, T, d, block, dtype_code)
+
+
+def sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, K, block=BLOCK) -> int:
+    return _ws_size("sas_decode_workspace_size", B, Hq, Hkv, Lmax, d, block, K)
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zeroed byte buffer of at least ``nbytes`` (torch allocations are 256-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, sm_scale, ws, block=BLOCK, stream=None):
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    _check("sas_fwd", lib().sas_fwd(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(O), _ptr(LSE),
+        B, Hq, Hkv, T, d, block, float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, sm_scale, ws, block=BLOCK, stream=None):
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    _check("sas_bwd", lib().sas_bwd(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), _ptr(logG), _ptr(tau), _ptr(tau_idx),
+        _ptr(LSE), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dLogG), B, Hq, Hkv, T, d, block, float(sm_scale),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sas_decode_fwd(q, Kc, Vc, seqlen, s, K, o, ws, sm_scale, sel_out=None, apply_log_gate=False, block=BLOCK,
+                   stream=None):
+    B, Hq, d = q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    NBmax = s.shape[-1]
+    _check("sas_decode_fwd", lib().sas_decode_fwd(
+        _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(seqlen), _ptr(s), K, 1 if apply_log_gate else 0,
+        _ptr(o), _ptr(sel_out), B, Hq, Hkv, Lmax, NBmax, d, block, float(sm_scale), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sas_device_status(ws, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    lib().sas_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
+    return out.value
+
+
+def sas_device_status_clear(ws, stream=None):
+    _check("sas_device_status_clear", lib().sas_device_status_clear(_ptr(ws), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------------------------
+# Convenience wrappers that allocate outputs (torch device memory) and chain the calls.
+# ---------------------------------------------------------------------------------------------
+def gate_and_select(s, K, block=BLOCK, want_sel=False, stream=None):
+    """logG, tau, tau_idx (and sel) from selector scores s [B,Hkv,T,NB] on the device."""
+    B, Hkv, T, NB = s.shape
+    logG = torch.empty_like(s)
+    tau = torch.empty(B, Hkv, T, dtype=torch.float32, device=s.device)
+    tidx = torch.empty(B, Hkv, T, dtype=torch.int32, device=s.device)
+    sel = torch.empty(B, Hkv, T, max(K - 1, 1), dtype=torch.int32, device=s.device) if want_sel else None
+    sas_gate_normalize(s, logG, block, stream)
+    sas_select_threshold(logG, tau, tidx, sel, K, block, stream)
+    return logG, tau, tidx, sel
+
+
+def _check_device_status(fn, ws, stream):
+    st = sas_device_status(ws, stream)
+    if st != 0:
+        raise SasError(fn, -4)
+
+
+def forward(Q, K, V, logG, tau, tau_idx, sm_scale, block=BLOCK, stream=None, ws=None, check=True):
+    """O, LSE of ``sas_fwd``. With ``check`` the stream is synchronised and the
+    kernel status word is read (raises ``SasError`` on a kernel-side timeout)."""
+    B, Hq, T, d = Q.shape
+    O = torch.empty_like(Q)
+    LSE = torch.empty(B, Hq, T, dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = workspace(sas_fwd_workspace_size(B, Hq, K.shape[1], T, d, _dtype_code(Q), block), Q.device)
+    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, sm_scale, ws, block, stream)
+    if check:
+        _check_device_status("sas_fwd", ws, stream)
+    return O, LSE
+
+
+def backward(Q, K, V, O, dO, logG, tau, tau_idx, LSE, sm_scale, block=BLOCK, stream=None, ws=None, check=True):
+    """dQ, dK, dV, dLogG of ``sas_bwd`` (``check`` as in ``forward``)."""
+    B, Hq, T, d = Q.shape
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    dLogG = torch.empty_like(logG)
+    if ws is None:
+        ws = workspace(sas_bwd_workspace_size(B, Hq, K.shape[1], T, d, _dtype_code(Q), block), Q.device)
+    sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, sm_scale, ws, block, stream)
+    if check:
+        _check_device_status("sas_bwd", ws, stream)
+    return dQ, dK, dV, dLogG

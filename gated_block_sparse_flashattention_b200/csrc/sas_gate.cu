@@ -1,0 +1,177 @@
+// Gate normalisation, per-query Top-K threshold selection, and the per-q-tile
+// union of selected blocks used by the tensor-core kernels.
+//
+// SAS paper (arXiv 2609.13141): §4.1 eq. 4 and §4.2 eq. 6 (softmax gates in log
+// form over the historical blocks), §4.3 "Kernel Design" and Appendix E (Top-K
+// realised as a per-query threshold on the log gate, no sort).
+#include "sas_common.cuh"
+#include "sas_kernels.h"
+
+namespace sas {
+
+// ---------------------------------------------------------------------------
+// logG[row, m] = s[row, m] - LSE(s[row, :c]) for m < c, -inf otherwise.
+// One warp per (b, g, t) row; two passes over the row (max, then sum of exp).
+// HBM-bound: reads the causal part of s once, writes the full logG row once.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gate_normalize_kernel(const float* __restrict__ s, float* __restrict__ logG,
+                                                             long long rows, int T, int NB) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  const float* src = s + row * (long long)NB;
+  float* dst = logG + row * (long long)NB;
+  float mx = -INFINITY;
+  for (int m = lane; m < c; m += 32) mx = fmaxf(mx, __ldg(src + m));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+  for (int m = lane; m < c; m += 32) sum += expf(__ldg(src + m) - mx);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float lse = mx + logf(sum);
+  for (int m = lane; m < NB; m += 32) dst[m] = (m < c) ? (__ldg(src + m) - lse) : -INFINITY;
+}
+
+__global__ void __launch_bounds__(256) select_threshold_kernel(const float* __restrict__ logG, float* __restrict__ tau,
+                                                               int32_t* __restrict__ tau_idx,
+                                                               int32_t* __restrict__ sel, long long rows, int T,
+                                                               int NB, int H) {
+  __shared__ uint32_t hist_all[8][256];
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * 8 + wid;
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  const float* v = logG + row * (long long)NB;
+  int32_t* out = sel ? sel + row * (long long)H : nullptr;
+  if (min(c, H) == 0) {
+    if (lane == 0) {
+      tau[row] = INFINITY;
+      tau_idx[row] = -1;
+    }
+    if (out)
+      for (int k = lane; k < H; k += 32) out[k] = -1;
+    return;
+  }
+  if (c <= H) {
+    if (lane == 0) {
+      tau[row] = -INFINITY;
+      tau_idx[row] = c - 1;
+    }
+    if (out)
+      for (int k = lane; k < H; k += 32) out[k] = (k < c) ? k : -1;
+    return;
+  }
+  int take_eq = 0;
+  const uint32_t tkey = warp_radix_select(v, c, H, hist_all[wid], &take_eq);
+  // tau_idx: the take_eq-th (1-based) index, ascending, among values whose key equals tkey.
+  int tidx = -1;
+  int run = 0;
+  for (int base = 0; base < c; base += 32) {
+    const int m = base + lane;
+    const bool eq = (m < c) && (float_key(v[m]) == tkey);
+    const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+    const int cnt = __popc(bal);
+    if (run + cnt >= take_eq) {
+      uint32_t b = bal;
+      for (int k = 1; k < take_eq - run; ++k) b &= b - 1u;   // drop the lower set bits
+      tidx = base + __ffs(b) - 1;
+      break;
+    }
+    run += cnt;
+  }
+  if (lane == 0) {
+    tau[row] = key_float(tkey);
+    tau_idx[row] = tidx;
+  }
+  if (out) {
+    int pos = 0;
+    for (int base = 0; base < c; base += 32) {
+      const int m = base + lane;
+      bool take = false;
+      if (m < c) {
+        const uint32_t k = float_key(v[m]);
+        take = (k > tkey) || (k == tkey && m <= tidx);
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(bal & ((1u << lane) - 1u))] = m;
+      pos += __popc(bal);
+    }
+    for (int k = pos + lane; k < H; k += 32) out[k] = -1;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Union of the selected historical blocks over the rows of one q-tile (P
+// consecutive positions of one (b, g); all G heads share the selection).
+// masks[(bg * n_ptiles + pt) * NBW + w] bit i = block 32w + i is selected by
+// at least one position of the tile (current blocks not included).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) tile_union_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
+                                                         const int32_t* __restrict__ tau_idx,
+                                                         uint32_t* __restrict__ masks, int T, int NB, int P,
+                                                         int n_ptiles, int NBW) {
+  extern __shared__ uint32_t words[];
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  const long long bg = blockIdx.x / n_ptiles;
+  const int pt = blockIdx.x % n_ptiles;
+  for (int w = threadIdx.x; w < NBW; w += blockDim.x) words[w] = 0u;
+  __syncthreads();
+  const int t0 = pt * P;
+  for (int p = wid; p < P; p += nw) {
+    const int t = t0 + p;
+    if (t >= T) break;
+    const long long row = bg * T + t;
+    const int c = min(t / kBlock, NB);
+    const float tv = tau[row];
+    const int ti = tau_idx[row];
+    const float* v = logG + row * (long long)NB;
+    for (int base = 0; base < c; base += 32) {
+      const int m = base + lane;
+      bool sel = false;
+      if (m < c) {
+        const float x = v[m];
+        sel = (x > tv) || (x == tv && m <= ti);
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0 && bal) atomicOr(&words[base >> 5], bal);
+    }
+  }
+  __syncthreads();
+  uint32_t* dst = masks + ((long long)bg * n_ptiles + pt) * NBW;
+  for (int w = threadIdx.x; w < NBW; w += blockDim.x) dst[w] = words[w];
+}
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_gate_normalize(const float* s, float* logG, long long rows, int T, int NB, cudaStream_t st) {
+  const int warps = 8;
+  const long long blocks = (rows + warps - 1) / warps;
+  gate_normalize_kernel<<<(unsigned)blocks, warps * 32, 0, st>>>(s, logG, rows, T, NB);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_threshold(const float* logG, float* tau, int32_t* tau_idx, int32_t* sel, long long rows,
+                                    int T, int NB, int H, cudaStream_t st) {
+  const long long blocks = (rows + 7) / 8;
+  select_threshold_kernel<<<(unsigned)blocks, 256, 0, st>>>(logG, tau, tau_idx, sel, rows, T, NB, H);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_union(const float* logG, const float* tau, const int32_t* tau_idx, uint32_t* masks,
+                              long long n_bg, int T, int NB, int P, int n_ptiles, int NBW, cudaStream_t st) {
+  const long long blocks = n_bg * n_ptiles;
+  tile_union_kernel<<<(unsigned)blocks, 256, NBW * sizeof(uint32_t), st>>>(logG, tau, tau_idx, masks, T, NB, P,
+                                                                           n_ptiles, NBW);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace sas

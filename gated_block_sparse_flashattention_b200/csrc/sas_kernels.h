@@ -1,0 +1,70 @@
+// Host-side declarations of the kernel launchers (internal to the library).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace sas {
+
+// Counts one kernel launch (reported by sas_launch_count()).
+void count_launch();
+
+cudaError_t launch_gate_normalize(const float* s, float* logG, long long rows, int T, int NB, cudaStream_t st);
+cudaError_t launch_select_threshold(const float* logG, float* tau, int32_t* tau_idx, int32_t* sel, long long rows,
+                                    int T, int NB, int H, cudaStream_t st);
+cudaError_t launch_tile_union(const float* logG, const float* tau, const int32_t* tau_idx, uint32_t* masks,
+                              long long n_bg, int T, int NB, int P, int n_ptiles, int NBW, cudaStream_t st);
+
+// Shape of the query tiles of the tensor-core kernels: P consecutive positions
+// of one (b, g) times the G heads of the group, P a multiple of 8 with G*P <= 128.
+struct QTileShape {
+  int P;         // positions per tile
+  int n_ptiles;  // tiles per (b, g)
+  int NBW;       // 32-bit words of a per-tile block bitmask
+};
+QTileShape qtile_shape(int G, int T, int NB);
+
+struct TcProblem {
+  int B, Hq, Hkv, T, d, NB, G;
+  float sm_scale;
+  const void* Q;
+  const void* K;
+  const void* V;
+  const void* O;    // bwd only
+  const void* dO;   // bwd only
+  const float* logG;
+  const float* tau;
+  const int32_t* tau_idx;
+  const float* LSE;  // bwd only
+};
+
+// bf16 tensor-core forward; ws holds the status word and the tile masks.
+cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* status, uint32_t* masks,
+                          cudaStream_t st);
+// bf16 tensor-core backward.
+cudaError_t launch_bwd_tc(const TcProblem& pb, void* dQ, void* dK, void* dV, float* dLogG, int32_t* status,
+                          uint32_t* masks, float* delta, cudaStream_t st);
+
+// fp32 CUDA-core forward / backward.
+cudaError_t launch_fwd_simt(const TcProblem& pb, float* O, float* LSE, cudaStream_t st);
+cudaError_t launch_bwd_simt(const TcProblem& pb, float* dQ, float* dK, float* dV, float* dLogG, float* delta,
+                            cudaStream_t st);
+
+// Decode (bf16 or fp32 storage).
+struct DecodeProblem {
+  int B, Hq, Hkv, Lmax, NBmax, d, K, apply_log_gate, dtype;
+  float sm_scale;
+  const void* q;
+  const void* Kc;
+  const void* Vc;
+  const int32_t* seqlen;
+  const float* s;
+  void* o;
+  int32_t* sel_out;
+};
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int K);
+cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st);
+
+}  // namespace sas

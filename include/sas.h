@@ -1,0 +1,184 @@
+/*
+ * sas.h - C ABI of the SAS gated block-sparse attention library for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one defined in "SAS: Simple Attention Sparsification via
+ * End-to-End Optimization of Context Ranking" (arXiv 2609.13141), cited below as
+ * "SAS paper":
+ *
+ *   * a selector score s[m] per historical context block becomes a gate
+ *     g = softmax(s) over the historical blocks, used in log form
+ *     (§4.1 eq. 4, §4.2 "Activation function" eq. 6);
+ *   * each query keeps its current block B_0 (unit gate, causal) and the
+ *     Top-(K-1) historical blocks, realised as a per-query threshold on the log
+ *     gate (§4.3 "Kernel Design", Appendix E);
+ *   * attention is softmax(q K_S^T + log g_S) V_S over the kept tokens
+ *     (§4.3 eq. 9), with dQ/dK/dV and the block-level gate gradient in the
+ *     backward pass (Appendix E "Backward pass"; Appendix D.1 eq. 5);
+ *   * decoding selects Top-(K-1) historical blocks by score and runs ungated
+ *     attention over them and the current block (§4.3 Algorithm 2; §5.1
+ *     "Inference implementation").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Blocks are `block` = 64 consecutive tokens. Query position t is in block
+ *    c_t = t / 64; its historical blocks are m < c_t.
+ *  - K (the budget) counts blocks and INCLUDES the current block: H = K - 1
+ *    historical blocks are kept per query.
+ *  - Grouped-query attention: Hq query heads, Hkv KV heads, G = Hq / Hkv. Query
+ *    head h uses KV head g = h / G. Gates, thresholds and selections are per
+ *    (batch, KV head, position) and shared by the G query heads of the group.
+ *  - Layouts are dense row-major, innermost dimension last:
+ *      Q, O, dO, dQ : [B, Hq, T, d]          K, V, dK, dV : [B, Hkv, T, d]
+ *      s, logG, dLogG : [B, Hkv, T, NB] fp32  tau : [B, Hkv, T] fp32
+ *      tau_idx : [B, Hkv, T] int32            LSE : [B, Hq, T] fp32 (natural log)
+ *  - Pointers are DEVICE pointers unless stated otherwise. The caller owns every
+ *    buffer, including the workspace; the library never allocates or frees
+ *    device memory. All device pointers must be 16-byte aligned.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream). Arguments are validated on the host
+ *    before anything is launched; an invalid call returns an error and
+ *    launches nothing.
+ *  - Kernel-side failures (a bounded wait that expired) are recorded in a status
+ *    word at the start of the workspace; read it with sas_device_status().
+ *  - sm_scale multiplies q.k only; the log gate is added unscaled.
+ *  - The fp32 data type runs on a CUDA-core kernel; bf16 runs on tcgen05
+ *    tensor-core kernels (fwd/bwd: d = 128).
+ */
+#ifndef SAS_B200_H
+#define SAS_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAS_API __attribute__((visibility("default")))
+#else
+#define SAS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call. */
+typedef enum {
+  SAS_OK = 0,
+  SAS_ERR_INVALID_ARG = -1, /* bad pointer, size, alignment or combination of sizes */
+  SAS_ERR_UNSUPPORTED = -2, /* valid, but not a shape/dtype this build implements */
+  SAS_ERR_CUDA = -3,        /* a CUDA runtime call failed (e.g. a launch error) */
+  SAS_ERR_TIMEOUT = -4,     /* a kernel's bounded wait expired (reported by sas_device_status) */
+  SAS_ERR_WORKSPACE = -5    /* workspace missing or smaller than the *_workspace_size answer */
+} sas_status;
+
+/* Element types of Q/K/V/O/dO/dQ/dK/dV. */
+typedef enum { SAS_DT_F32 = 0, SAS_DT_BF16 = 1 } sas_dtype;
+
+/* Human-readable name of a status code. Never NULL. */
+SAS_API const char* sas_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+SAS_API int sas_version(void);
+
+/* Number of kernels this library has launched since it was loaded (all threads). */
+SAS_API uint64_t sas_launch_count(void);
+
+/*
+ * sas_gate_normalize - softmax gate activation in log form.
+ * SAS paper §4.1 eq. 4 (g = phi(s), g_0 = 1) with phi = softmax, §4.2 eq. 6:
+ *   logG[b,g,t,m] = s[b,g,t,m] - log sum_{m' < c_t} exp(s[b,g,t,m'])   for m < c_t,
+ *   logG[b,g,t,m] = -inf                                               for m >= c_t.
+ * s, logG: [B, Hkv, T, NB] fp32 (may not alias). NB >= ceil(T / block).
+ * block must be 64. Rows with c_t = 0 are all -inf.
+ */
+SAS_API int sas_gate_normalize(const float* s, float* logG, int B, int Hkv, int T, int NB, int block, void* stream);
+
+/*
+ * sas_select_threshold - Top-(K-1) historical blocks per query as a threshold.
+ * SAS paper §4.3 "Kernel Design" and Appendix E: block m < c_t is selected iff
+ *   logG[m] > tau  or  (logG[m] == tau and m <= tau_idx),
+ * which keeps exactly min(K-1, c_t) blocks: the K-1 largest values, equal values
+ * going to the lower block index (-0.0 equals +0.0). Rows with c_t <= K-1 keep
+ * every historical block (tau = -inf, tau_idx = c_t - 1); rows that keep none
+ * (c_t = 0 or K = 1) get tau = +inf, tau_idx = -1.
+ * logG: [B,Hkv,T,NB] fp32, finite for m < c_t. tau: [B,Hkv,T] fp32.
+ * tau_idx: [B,Hkv,T] int32. sel (nullable): [B,Hkv,T,K-1] int32, the selected
+ * block indices in ascending order, padded with -1. K >= 1, block == 64.
+ */
+SAS_API int sas_select_threshold(const float* logG, float* tau, int32_t* tau_idx, int32_t* sel, int B, int Hkv, int T,
+                         int NB, int block, int K, void* stream);
+
+/*
+ * Workspace sizes (bytes) for sas_fwd, sas_bwd and sas_decode_fwd with the given
+ * sizes. The workspace is caller-owned device memory, at least 256-byte aligned,
+ * and may be reused across calls on the same stream. Its first word is the
+ * device status word.
+ */
+SAS_API int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes);
+SAS_API int sas_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes);
+SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int block, int K, size_t* bytes);
+
+/*
+ * sas_fwd - gated block-sparse attention forward (SAS paper §4.3 eq. 9, Appendix E
+ * Algorithm 3 "Forward Pass"):
+ *   O[b,h,t]   = sum_i softmax_i(z) V[b,g,i],   z_i = sm_scale q.k_i + bias(t, i),
+ *   LSE[b,h,t] = log sum_i exp(z_i),
+ * with bias = 0 for keys of the current block with i <= t, logG[b,g,t,m] for keys
+ * of a selected historical block m (selection as in sas_select_threshold), and
+ * -inf for every other key.
+ * Q [B,Hq,T,d], K/V [B,Hkv,T,d] of `dtype`; logG [B,Hkv,T,NB], tau, tau_idx as
+ * produced by the two calls above (any values obeying their contract work).
+ * O [B,Hq,T,d] of `dtype`; LSE [B,Hq,T] fp32. T % 64 == 0, NB == T / 64,
+ * Hq % Hkv == 0, d in {64, 128} (fp32) or d == 128 (bf16).
+ * ws: workspace of sas_fwd_workspace_size bytes.
+ */
+SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* tau,
+            const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d, int block,
+            float sm_scale, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * sas_bwd - gradients of a scalar loss through sas_fwd (SAS paper Appendix E
+ * "Backward pass", Algorithm 4; gate gradient per Appendix D.1 eq. 5 / D.3):
+ *   P = exp(z - LSE), Delta = rowsum(O * dO), dS = P * (dO V^T - Delta),
+ *   dQ = sm_scale dS K,  dK = sm_scale sum_{h in g} dS^T Q,  dV = sum_{h in g} P^T dO,
+ *   dLogG[b,g,t,m] = sum_{h in g} sum_{i in block m} dS[h,t,i] for selected m, 0 otherwise.
+ * Inputs as for sas_fwd plus O (the forward output), dO and LSE (the forward's).
+ * Outputs dQ [B,Hq,T,d], dK/dV [B,Hkv,T,d] of `dtype`; dLogG [B,Hkv,T,NB] fp32
+ * (fully written: zero outside the selection). ws: sas_bwd_workspace_size bytes.
+ */
+SAS_API int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
+            const float* logG, const float* tau, const int32_t* tau_idx, const float* LSE, void* dQ, void* dK,
+            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, float sm_scale, void* ws,
+            size_t ws_bytes, void* stream);
+
+/*
+ * sas_decode_fwd - one sparse decode step per sequence (SAS paper §4.3
+ * Algorithm 2; §5.1 "Inference implementation", §6.3):
+ *   L = seqlen[b] (the new token is position L-1), c = (L-1) / 64;
+ *   I = Top-(K-1) of blocks 0..c-1 by s[b,g,:] (ties to the lower index);
+ *   o[b,h] = softmax(sm_scale q K_S^T + bias) V_S over S = block c (positions
+ *   c*64 .. L-1) and the blocks in I; bias = 0 (ungated, Algorithm 2) or, with
+ *   apply_log_gate != 0, s[b,g,m] - log sum_{m'<c} exp(s[b,g,m']) on block m in I.
+ * q [B,Hq,d], Kc/Vc [B,Hkv,Lmax,d] of `dtype` (the KV cache; the new token's
+ * key/value already at position L-1); seqlen [B] int32 DEVICE, 1 <= L <= Lmax;
+ * s [B,Hkv,NBmax] fp32 with NBmax >= ceil(Lmax/64); o [B,Hq,d] of `dtype`;
+ * sel_out (nullable) [B,Hkv,K-1] int32 receives I in ascending order, -1 padded.
+ * d == 128, 1 <= K <= 64. ws: sas_decode_workspace_size bytes.
+ */
+SAS_API int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen, const float* s,
+                   int K, int apply_log_gate, void* o, int32_t* sel_out, int B, int Hq, int Hkv, int Lmax, int NBmax,
+                   int d, int block, float sm_scale, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * sas_device_status - read the device status word of a workspace used by
+ * sas_fwd/sas_bwd/sas_decode_fwd. Synchronises `stream`, copies the word to
+ * *status_out (0 = no kernel-side error) and returns SAS_ERR_TIMEOUT if a bounded
+ * wait expired, else SAS_OK. sas_device_status_clear() zeroes it (asynchronously).
+ */
+SAS_API int sas_device_status(const void* ws, void* stream, int32_t* status_out);
+SAS_API int sas_device_status_clear(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAS_B200_H */

@@ -1,0 +1,89 @@
+"""The C-ABI library loads and exports every symbol include/sas.h declares;
+host-side validation and workspace sizing work without a GPU (nothing here
+launches a kernel)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_block_sparse_flashattention_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sas.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.library_path()):
+        from gated_block_sparse_flashattention_b200 import build
+        build.build()
+    return binding.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SAS_API\s+[\w\s\*]+?\b(sas_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_operations():
+    names = declared_symbols()
+    for op in ("sas_gate_normalize", "sas_select_threshold", "sas_fwd", "sas_bwd", "sas_decode_fwd"):
+        assert op in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(binding._SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings_and_version(lib):
+    assert binding.status_string(0) == "SAS_OK"
+    for code in (-1, -2, -3, -4, -5):
+        assert binding.status_string(code).startswith("SAS_ERR")
+    assert lib.sas_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    # bf16 Qwen3-4B-like layer: status word + Delta + per-tile block masks
+    fwd = binding.sas_fwd_workspace_size(1, 32, 8, 8192, 128, binding.SAS_DT_BF16)
+    bwd = binding.sas_bwd_workspace_size(1, 32, 8, 8192, 128, binding.SAS_DT_BF16)
+    assert fwd >= 256 + 8 * 256 * 4 * 4          # 256 q-tiles x 4 mask words per (b, g)
+    assert bwd >= 256 + 32 * 8192 * 4 + 8 * 256 * 4 * 4
+    assert binding.sas_fwd_workspace_size(1, 4, 1, 1024, 64, binding.SAS_DT_F32) == 256
+    assert binding.sas_decode_workspace_size(16, 32, 8, 32768, 128, 16) > 0
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((1, 32, 8, 8192, 96, binding.SAS_DT_BF16), -2),   # d = 96 not implemented
+    ((1, 32, 8, 8100, 128, binding.SAS_DT_BF16), -1),  # T not a multiple of 64
+    ((1, 30, 8, 8192, 128, binding.SAS_DT_BF16), -1),  # Hq not a multiple of Hkv
+    ((1, 32, 8, 8192, 128, 7), -1),                    # unknown dtype
+    ((1, 64, 2, 8192, 128, binding.SAS_DT_BF16), -2),  # G = 32 > 16
+])
+def test_workspace_size_rejects(lib, args, expect):
+    out = ctypes.c_size_t(0)
+    B, Hq, Hkv, T, d, dt = args
+    assert lib.sas_fwd_workspace_size(B, Hq, Hkv, T, d, 64, dt, ctypes.byref(out)) == expect
+
+
+def test_invalid_calls_return_errors_without_launching(lib):
+    before = lib.sas_launch_count()
+    fake = 0x1000  # never dereferenced: validation fails first
+    assert lib.sas_gate_normalize(None, fake, 1, 1, 64, 1, 64, None) == -1
+    assert lib.sas_gate_normalize(fake, fake, 1, 1, 64, 1, 64, None) == -1          # aliasing
+    assert lib.sas_gate_normalize(fake, fake + 64, 1, 1, 64, 1, 32, None) == -1     # block != 64
+    assert lib.sas_gate_normalize(fake + 4, fake + 64, 1, 1, 64, 1, 64, None) == -1  # misaligned
+    assert lib.sas_select_threshold(fake, fake, fake, None, 1, 1, 128, 2, 64, 0, None) == -1  # K < 1
+    # sas_fwd: missing workspace / bad sizes
+    args = [fake] * 3 + [binding.SAS_DT_BF16] + [fake] * 5 + [1, 4, 1, 128, 128, 64, ctypes.c_float(0.1), None, 0, None]
+    assert lib.sas_fwd(*args) == -5
+    args[-3] = fake
+    args[-2] = 1 << 30
+    args[12] = 100   # T not a multiple of 64
+    assert lib.sas_fwd(*args) == -1
+    assert lib.sas_launch_count() == before
