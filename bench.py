@@ -1,0 +1,460 @@
+"""Benchmark of the SAS hot path on B200.
+
+One step = one pass of the whole training-side path over one batch of the
+Qwen3-4B-like layer (B=1, Hq=32, Hkv=8, d=128, T=8192, block 64, K=16 blocks):
+gate normalisation, Top-K threshold selection, forward and backward
+(dQ/dK/dV/dLogG). The metric is attended-block TFLOP/s: 4*d*sum_rows(n_t) for
+the forward and 2.5x that for the backward, n_t = (t mod 64) + 1 + 64*min(K-1, c_t)
+attended keys of row t. The memory-bound decode step (16 sequences over a
+32768-token cache) is reported beside it in GB/s.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU: launched by torchrun, one process per GPU; each rank runs its own
+batch of the same shape (no collective on the data path: the work splits into
+independent (batch, KV-group) units), timings are reduced with max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from gated_block_sparse_flashattention_b200 import workloads  # noqa: E402
+
+BENCH_WORKLOAD = "qwen3_4b_t8k"
+DECODE_WORKLOAD = "decode_b16_l32k"
+L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2, written between timed steps
+
+
+# ----------------------------------------------------------------------------- work counts
+def attended_keys_per_row(T: int, K: int, block: int = 64) -> np.ndarray:
+    """n_t for every position t: causal part of the current block plus min(K-1, c_t) full blocks."""
+    t = np.arange(T)
+    return (t % block) + 1 + block * np.minimum(K - 1, t // block)
+
+
+def attended_flops(w) -> tuple[float, float]:
+    """(forward, backward) algorithmic FLOPs of one step of workload w."""
+    n = attended_keys_per_row(w.T, w.K, w.block).sum(dtype=np.float64)
+    fwd = 4.0 * w.d * n * w.B * w.Hq
+    return fwd, 2.5 * fwd
+
+
+def decode_bytes(w) -> float:
+    """Algorithmic bytes of one decode step: selected K/V blocks, q, o and the score rows."""
+    el = 2 if w.dtype == "bf16" else 4
+    kv = 2.0 * w.B * w.Hkv * w.K * w.block * w.d * el
+    qo = 2.0 * w.B * w.Hq * w.d * el
+    s = w.B * w.Hkv * w.NB * 4.0
+    return kv + qo + s
+
+
+# ----------------------------------------------------------------------------- multi-rank helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def shard_units(n_units: int, rank: int, world: int) -> list[int]:
+    """Round-robin assignment of independent (batch, KV-group) units to ranks."""
+    return list(range(rank, n_units, world))
+
+
+def reduce_max(value: float, device=None) -> float:
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self._thr = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._thr = threading.Thread(target=self._read, daemon=True)
+            self._thr.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self._thr:
+                self._thr.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+def oracle_sample(w, seconds: float, seed: int = 0):
+    """Time the CPU oracle, as it stands, on consecutive 128-row chunks of one
+    (b, g) group of workload w (the last positions: the longest rows) until
+    about ``seconds`` of work. Returns (TFLOP/s, threads, description)."""
+    from oracle import sas_oracle as orc
+
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        threads = 1
+    inp = workloads.make_training_inputs(w, seed=seed)
+    f64 = lambda t: t[:1, : w.G].float().numpy().astype(np.float64)  # noqa: E731
+    Q, dO = f64(inp["Q"]), f64(inp["dO"])
+    Kt = inp["K"][:1, :1].float().numpy().astype(np.float64)
+    V = inp["V"][:1, :1].float().numpy().astype(np.float64)
+    s = inp["s"][:1, :1].numpy().astype(np.float64)
+    logG = orc.gate_normalize(s, w.block)
+    tau, tidx, _ = orc.select_threshold(logG, w.K, w.block)
+    n_t = attended_keys_per_row(w.T, w.K, w.block)
+    work, elapsed, rows_done = 0.0, 0.0, 0
+    hi = w.T
+    while elapsed < seconds and hi > 0:
+        rows = np.arange(max(0, hi - 128), hi)
+        t0 = time.perf_counter()
+        orc.forward_backward(Q, Kt, V, dO, logG, tau, tidx, w.block, w.sm_scale, rows=rows)
+        elapsed += time.perf_counter() - t0
+        work += 3.5 * 4.0 * w.d * n_t[rows].sum() * w.G
+        rows_done += len(rows)
+        hi -= 128
+    desc = (f"oracle fwd+bwd (materialised, fp64) on {rows_done} query positions x {w.G} heads of one "
+            f"(batch, KV group) of {w.name}; gates normalised/selected by the oracle outside the timing")
+    return work / elapsed / 1e12, threads, desc
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    from gated_block_sparse_flashattention_b200 import binding
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = workloads.WORKLOADS[BENCH_WORKLOAD]
+    fwd_flops, bwd_flops = attended_flops(w)
+    step_flops = fwd_flops + bwd_flops
+    peaks = measured_peaks()
+
+    # Inputs: this rank's own batch (seeded by rank), resident in HBM before timing.
+    host = workloads.make_training_inputs(w, seed=rank)
+    Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
+    logG = torch.empty_like(s)
+    tau = torch.empty(w.B, w.Hkv, w.T, device=device)
+    tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(w.B, w.Hq, w.T, device=device)
+    dQ, dK, dV, dLogG = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s)
+    ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
+    ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        binding.sas_gate_normalize(s, logG, stream=stream)
+        binding.sas_select_threshold(logG, tau, tidx, None, w.K, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.sm_scale, ws_f, stream=stream)
+        if ev:
+            ev[2].record(stream)
+        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.sm_scale, ws_b, stream=stream)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    if binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b):
+        raise RuntimeError("kernel-side timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    launches0 = binding.launch_count()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()      # L2 flush between timed steps (outside the events)
+            step(evs[i])
+        torch.cuda.synchronize(device)
+    launches = binding.launch_count() - launches0
+    barrier(device)
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    gate_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = reduce_max(sum(step_ms), device)
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # Dominant call (the backward) against the tensor-core roofline.
+    bwd_avg = statistics.mean(bwd_ms)
+    fwd_avg = statistics.mean(fwd_ms)
+    dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
+        ("sas_fwd", fwd_avg, fwd_flops)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
+                "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
+                "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
+                "gate_select_ms": round(statistics.mean(gate_ms), 4)}
+
+    legs = set(args.legs.split(","))
+    # End to end through the C ABI from pinned host buffers, results copied back.
+    e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
+    dec = run_decode(args, device, stream, binding, peaks) if "decode" in legs else None
+
+    result = {
+        "metric": "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd step)",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "qwen3_4b_t8k layer fwd+bwd: B=1 Hq=32 Hkv=8 d=128 T=8192 block=64 K=16 "
+                               "(1024-token budget), s~N(0,2) + 3 planted blocks per query",
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "flushed between timed steps (512 MiB write, outside the timed events)",
+                   "attended_gflop_per_step": round(step_flops / 1e9, 2)},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "decode": dec,
+    }
+    if rank == 0 and world == 1 and "cpu" in legs:
+        tf, threads, desc = oracle_sample(w, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                  "sample": desc}
+    result["clocks"] = clk.summary()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, host, device, stream, binding, step_flops, world):
+    pinned = {k: host[k].pin_memory() for k in ("Q", "K", "V", "dO", "s")}
+    out_host = {"O": torch.empty(host["Q"].shape, dtype=host["Q"].dtype).pin_memory(),
+                "dQ": torch.empty(host["Q"].shape, dtype=host["Q"].dtype).pin_memory(),
+                "dK": torch.empty(host["K"].shape, dtype=host["K"].dtype).pin_memory(),
+                "dV": torch.empty(host["V"].shape, dtype=host["V"].dtype).pin_memory(),
+                "dLogG": torch.empty(host["s"].shape, dtype=torch.float32).pin_memory()}
+    dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in pinned.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        logG, tau, tidx, _ = binding.gate_and_select(dev_in["s"], w.K, stream=stream)
+        O, LSE = binding.forward(dev_in["Q"], dev_in["K"], dev_in["V"], logG, tau, tidx, w.sm_scale, stream=stream,
+                                 check=False)
+        dQ, dK, dV, dLogG = binding.backward(dev_in["Q"], dev_in["K"], dev_in["V"], O, dev_in["dO"], logG, tau,
+                                             tidx, LSE, w.sm_scale, stream=stream, check=False)
+        for k, v in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV), ("dLogG", dLogG)):
+            out_host[k].copy_(v, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    total = reduce_max(sum(times), device)
+    return {"value": round(world * step_flops * args.steps / (total * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(total / args.steps, 4)}
+
+
+def run_decode(args, device, stream, binding, peaks):
+    """Decode step (16 sequences x 1 token over a 32768-token cache) in a CUDA graph, L2 flushed between steps."""
+    w = workloads.WORKLOADS[DECODE_WORKLOAD]
+    n_rot = 4
+    inp = workloads.make_decode_inputs(w, seed=0)
+    q, Kc, Vc = inp["q"].to(device), inp["Kc"].to(device), inp["Vc"].to(device)
+    seqlen = inp["seqlen"].to(device)
+    gen = torch.Generator().manual_seed(1)
+    s_rot = [torch.randn(w.B, w.Hkv, w.NB, generator=gen).to(device) for _ in range(n_rot)]
+    s = s_rot[0].clone()
+    o = torch.empty_like(q)
+    ws = binding.workspace(binding.sas_decode_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K), device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    g_stream = torch.cuda.Stream(device)
+    g_stream.wait_stream(stream)
+    with torch.cuda.stream(g_stream):
+        binding.sas_decode_fwd(q, Kc, Vc, seqlen, s, w.K, o, ws, w.sm_scale, stream=g_stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=g_stream):
+            binding.sas_decode_fwd(q, Kc, Vc, seqlen, s, w.K, o, ws, w.sm_scale, stream=g_stream)
+    stream.wait_stream(g_stream)
+    torch.cuda.synchronize(device)
+    steps = max(args.steps, 20)
+    for i in range(max(args.warmup, 3)):
+        s.copy_(s_rot[i % n_rot])
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize(device)
+    times = []
+    for i in range(steps):
+        s.copy_(s_rot[i % n_rot])   # a different selection each step
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize(device)
+    ms = [a.elapsed_time(b) for a, b in times]
+    med = statistics.median(ms)
+    gbs = decode_bytes(w) / (med * 1e-3) / 1e9
+    st = binding.sas_device_status(ws)
+    del graph
+    return {"workload": "decode_b16_l32k: 16 seqs x 1 token, cache 32768, Hq=32 Hkv=8 d=128 K=16",
+            "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
+            "bytes_per_step": decode_bytes(w), "peak": peaks["hbm_gbs"],
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "graph": True, "steps": steps, "device_status": st}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[BENCH_WORKLOAD]
+    per_step = max(2.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        oracle_sample(w, 0.5)
+    vals, threads, desc = [], 1, ""
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, threads, desc = oracle_sample(w, per_step)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    print(json.dumps({
+        "impl": "reference", "metric": "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd step)",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "qwen3_4b_t8k layer fwd+bwd: B=1 Hq=32 Hkv=8 d=128 T=8192 block=64 K=16"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--legs", default="step,e2e,decode,cpu",
+                    help="comma list of what to measure and report: step (device-resident timed steps), e2e "
+                         "(host buffers through the C ABI), decode, cpu (oracle baseline)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -234,11 +234,14 @@ __global__ void __launch_bounds__(THREADS) decode_kernel(const Params p) {
     for (int h = 0; h < p.G; ++h) {
       float acc = 0.f;
       for (int k = 0; k < BPC; ++k) {
-        if (blk[k] < 0) continue;
+        const int m = blk[k];
+        if (m < 0) continue;
+        // Only keys that exist in the cache were copied; rows past them are stale.
+        const int nk = (m == c) ? (L - m * kBlock) : kBlock;
         const T* vb = kv + (2 * k + 1) * 64 * D;
         const float* ph = sc + h * nkeys + k * 64;
 #pragma unroll 8
-        for (int key = 0; key < 64; ++key) acc = fmaf(ph[key], to_f<T>(vb[key * D + dd]), acc);
+        for (int key = 0; key < nk; ++key) acc = fmaf(ph[key], to_f<T>(vb[key * D + dd]), acc);
       }
       p.part_o[(((long long)bg * p.nsplit + split) * p.G + h) * D + dd] = acc;
     }

@@ -34,7 +34,8 @@ def test_normalize_matches_oracle(B, Hkv, T, NB):
     got = out.cpu().numpy().astype(np.float64)
     fin = np.isfinite(ref)
     assert np.array_equal(np.isneginf(got), np.isneginf(ref))
-    assert np.max(np.abs(got[fin] - ref[fin])) < 2e-5
+    if fin.any():
+        assert np.max(np.abs(got[fin] - ref[fin])) < 2e-5
 
 
 @pytest.mark.parametrize("K", [1, 2, 4, 16, 33])
