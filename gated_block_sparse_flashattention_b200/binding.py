@@ -39,6 +39,8 @@ _SIGNATURES = {
                 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                        + [_c_f, _vp, _sz, _vp]),
+    "sas_decode_fwd_static": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
+                              + [_c_f, _vp]),
     "sas_device_status": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "sas_device_status_clear": (_c_int, [_vp, _vp]),
 }
@@ -166,6 +168,17 @@ def sas_decode_fwd(q, Kc, Vc, seqlen, s, K, o, ws, sm_scale, sel_out=None, apply
         _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(seqlen), _ptr(s), K, 1 if apply_log_gate else 0,
         _ptr(o), _ptr(sel_out), B, Hq, Hkv, Lmax, NBmax, d, block, float(sm_scale), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sas_decode_fwd_static(q, Kc, Vc, seqlen, s, K, o, sm_scale, sel_out=None, apply_log_gate=False, block=BLOCK,
+                          stream=None):
+    """sas_decode_fwd with the library's built-in static scratch (no workspace argument)."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    NBmax = s.shape[-1]
+    _check("sas_decode_fwd_static", lib().sas_decode_fwd_static(
+        _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(seqlen), _ptr(s), K, 1 if apply_log_gate else 0,
+        _ptr(o), _ptr(sel_out), B, Hq, Hkv, Lmax, NBmax, d, block, float(sm_scale), _stream(stream)))
 
 
 def sas_device_status(ws, stream=None) -> int:

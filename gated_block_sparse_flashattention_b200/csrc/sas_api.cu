@@ -235,6 +235,40 @@ int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dtype, con
   return cuda_status(launch_decode(pb, ws, as_stream(stream)));
 }
 
+int sas_decode_fwd_static(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen,
+                          const float* s, int K, int apply_log_gate, void* o, int32_t* sel_out, int B, int Hq,
+                          int Hkv, int Lmax, int NBmax, int d, int block, float sm_scale, void* stream) {
+  const void* ptrs[] = {q, Kc, Vc, seqlen, s, o};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return SAS_ERR_INVALID_ARG;
+  if (dtype != SAS_DT_F32 && dtype != SAS_DT_BF16) return SAS_ERR_INVALID_ARG;
+  if ((long long)NBmax * 64 < Lmax || !(sm_scale > 0.f)) return SAS_ERR_INVALID_ARG;
+  size_t need = 0;
+  int st = sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, block, K, &need);
+  if (st != SAS_OK) return st;
+  if (need > decode_static_scratch_limit()) return SAS_ERR_WORKSPACE;   // beyond the built-in scratch
+  DecodeProblem pb{};
+  pb.B = B;
+  pb.Hq = Hq;
+  pb.Hkv = Hkv;
+  pb.Lmax = Lmax;
+  pb.NBmax = NBmax;
+  pb.d = d;
+  pb.K = K;
+  pb.apply_log_gate = apply_log_gate ? 1 : 0;
+  pb.dtype = dtype;
+  pb.sm_scale = sm_scale;
+  pb.q = q;
+  pb.Kc = Kc;
+  pb.Vc = Vc;
+  pb.seqlen = seqlen;
+  pb.s = s;
+  pb.o = o;
+  pb.sel_out = sel_out;
+  return cuda_status(launch_decode_static(pb, as_stream(stream)));
+}
+
 int sas_device_status(const void* ws, void* stream, int32_t* status_out) {
   if (!ws || !status_out) return SAS_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));

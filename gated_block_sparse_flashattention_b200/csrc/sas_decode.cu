@@ -12,6 +12,8 @@
 // heads of the group against them on CUDA cores, and writes an fp32 partial
 // (row max, row sum, unnormalised output). The last CTA of a (b, g) to finish
 // (atomic ticket) merges the partials into o.
+#include <mutex>
+
 #include "sas_common.cuh"
 #include "sas_kernels.h"
 
@@ -342,6 +344,59 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
   }
   count_launch();
   return cudaGetLastError();
+}
+
+}  // namespace sas
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the decode step.
+//
+// Its scratch (status word, per-(b, g) tickets, split partials) lives in one
+// file-scope device array instead of a caller workspace. Every GPU that loads
+// the library keeps this array until the process exits, and every call on a
+// device shares it, so calls that overlap on the GPU race on it.
+// ---------------------------------------------------------------------------
+namespace sas {
+namespace decode_static {
+
+constexpr size_t kScratchBytes = 8u << 20;   // 8 MiB
+static __device__ __align__(256) uint8_t g_decode_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static void* g_scratch_addr[kMaxDevices] = {};
+static std::mutex g_scratch_mutex;
+
+// Device address of g_decode_scratch on the current device, looked up once per
+// device. The host-side name is only a stand-in: the kernel must be given this
+// address, never &g_decode_scratch.
+static cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace decode_static
+
+size_t decode_static_scratch_limit() { return decode_static::kScratchBytes; }
+
+cudaError_t launch_decode_static(const DecodeProblem& pb, cudaStream_t st) {
+  void* ws = nullptr;
+  cudaError_t e = decode_static::scratch_address(&ws);
+  if (e != cudaSuccess) return e;
+  // The status word starts clear on every call (tickets are cleared by launch_decode).
+  e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  return launch_decode(pb, ws, st);
 }
 
 }  // namespace sas

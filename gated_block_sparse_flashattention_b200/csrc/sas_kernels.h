@@ -66,5 +66,8 @@ struct DecodeProblem {
 };
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int K);
 cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st);
+// Decode with the library's own static device scratch instead of a workspace.
+size_t decode_static_scratch_limit();
+cudaError_t launch_decode_static(const DecodeProblem& pb, cudaStream_t st);
 
 }  // namespace sas

@@ -169,6 +169,35 @@ SAS_API int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dt
                    int d, int block, float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * sas_decode_fwd_static - sas_decode_fwd without a workspace argument. It has no
+ * counterpart in the SAS paper; it exists for callers that cannot allocate device
+ * memory themselves: a plugin whose host framework owns every device buffer and
+ * hands it only inputs and outputs, or a latency-critical decode loop that must
+ * not call cudaMalloc (which can synchronise the device) between steps.
+ *
+ * Arguments, layouts, results and errors are those of sas_decode_fwd, minus
+ * ws/ws_bytes. The scratch memory sas_decode_fwd would take from the workspace
+ * lives instead in one static 8 MiB device array inside the library:
+ *  - every GPU that loads the library holds those 8 MiB until the process exits;
+ *  - a problem whose sas_decode_workspace_size exceeds 8 MiB (8388608 bytes) is
+ *    rejected with SAS_ERR_WORKSPACE before anything is launched;
+ *  - the call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *    routine); it clears the parts of the array that must start at zero on
+ *    every call, with asynchronous memsets on `stream`;
+ *  - all calls on a device share the array, so calls whose kernels overlap on the
+ *    GPU (different streams, or different host threads) race on it and give
+ *    wrong results: serialise them;
+ *  - the first call on each device looks up the array's device address (with that
+ *    device current) and caches it; make that first call before any stream capture;
+ *  - the array's status word is cleared at the start of every call and is not
+ *    readable through this ABI.
+ */
+SAS_API int sas_decode_fwd_static(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen,
+                                  const float* s, int K, int apply_log_gate, void* o, int32_t* sel_out, int B,
+                                  int Hq, int Hkv, int Lmax, int NBmax, int d, int block, float sm_scale,
+                                  void* stream);
+
+/*
  * sas_device_status - read the device status word of a workspace used by
  * sas_fwd/sas_bwd/sas_decode_fwd. Synchronises `stream`, copies the word to
  * *status_out (0 = no kernel-side error) and returns SAS_ERR_TIMEOUT if a bounded
