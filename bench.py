@@ -230,7 +230,7 @@ def run_gpu(args):
     LSE = torch.empty(w.B, w.Hq, w.T, device=device)
     dQ, dK, dV, dLogG = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s)
     ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
-    ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
+    ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
@@ -244,7 +244,8 @@ def run_gpu(args):
         binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.sm_scale, ws_f, stream=stream)
         if ev:
             ev[2].record(stream)
-        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.sm_scale, ws_b, stream=stream)
+        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
+                        stream=stream)
         if ev:
             ev[3].record(stream)
 
@@ -339,7 +340,7 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
         O, LSE = binding.forward(dev_in["Q"], dev_in["K"], dev_in["V"], logG, tau, tidx, w.sm_scale, stream=stream,
                                  check=False)
         dQ, dK, dV, dLogG = binding.backward(dev_in["Q"], dev_in["K"], dev_in["V"], O, dev_in["dO"], logG, tau,
-                                             tidx, LSE, w.sm_scale, stream=stream, check=False)
+                                             tidx, LSE, w.K, w.sm_scale, stream=stream, check=False)
         for k, v in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV), ("dLogG", dLogG)):
             out_host[k].copy_(v, non_blocking=True)
 

@@ -32,10 +32,10 @@ _SIGNATURES = {
     "sas_gate_normalize": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_fwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
-    "sas_bwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
+    "sas_bwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_decode_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
     "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_f, _vp, _sz, _vp]),
-    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 6
+    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7
                 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                        + [_c_f, _vp, _sz, _vp]),
@@ -129,8 +129,8 @@ def sas_fwd_workspace_size(B, Hq, Hkv, T, d, dtype_code, block=BLOCK) -> int:
     return _ws_size("sas_fwd_workspace_size", B, Hq, Hkv, T, d, block, dtype_code)
 
 
-def sas_bwd_workspace_size(B, Hq, Hkv, T, d, dtype_code, block=BLOCK) -> int:
-    return _ws_size("sas_bwd_workspace_size", B, Hq, Hkv, T, d, block, dtype_code)
+def sas_bwd_workspace_size(B, Hq, Hkv, T, d, K, dtype_code, block=BLOCK) -> int:
+    return _ws_size("sas_bwd_workspace_size", B, Hq, Hkv, T, d, block, K, dtype_code)
 
 
 def sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, K, block=BLOCK) -> int:
@@ -150,13 +150,14 @@ def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, sm_scale, ws, block=BLOCK, stre
         B, Hq, Hkv, T, d, block, float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, sm_scale, ws, block=BLOCK, stream=None):
+def sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block=BLOCK,
+            stream=None):
     B, Hq, T, d = Q.shape
     Hkv = K.shape[1]
     _check("sas_bwd", lib().sas_bwd(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), _ptr(logG), _ptr(tau), _ptr(tau_idx),
-        _ptr(LSE), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dLogG), B, Hq, Hkv, T, d, block, float(sm_scale),
-        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+        _ptr(LSE), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dLogG), B, Hq, Hkv, T, d, block, int(Kbudget),
+        float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def sas_decode_fwd(q, Kc, Vc, seqlen, s, K, o, ws, sm_scale, sel_out=None, apply_log_gate=False, block=BLOCK,
@@ -226,14 +227,15 @@ def forward(Q, K, V, logG, tau, tau_idx, sm_scale, block=BLOCK, stream=None, ws=
     return O, LSE
 
 
-def backward(Q, K, V, O, dO, logG, tau, tau_idx, LSE, sm_scale, block=BLOCK, stream=None, ws=None, check=True):
+def backward(Q, K, V, O, dO, logG, tau, tau_idx, LSE, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None,
+             check=True):
     """dQ, dK, dV, dLogG of ``sas_bwd`` (``check`` as in ``forward``)."""
     B, Hq, T, d = Q.shape
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     dLogG = torch.empty_like(logG)
     if ws is None:
-        ws = workspace(sas_bwd_workspace_size(B, Hq, K.shape[1], T, d, _dtype_code(Q), block), Q.device)
-    sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, sm_scale, ws, block, stream)
+        ws = workspace(sas_bwd_workspace_size(B, Hq, K.shape[1], T, d, Kbudget, _dtype_code(Q), block), Q.device)
+    sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block, stream)
     if check:
         _check_device_status("sas_bwd", ws, stream)
     return dQ, dK, dV, dLogG

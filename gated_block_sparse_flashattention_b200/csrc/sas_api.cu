@@ -107,12 +107,12 @@ int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int 
   return SAS_OK;
 }
 
-int sas_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes) {
-  if (!bytes) return SAS_ERR_INVALID_ARG;
+int sas_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int K, int dtype, size_t* bytes) {
+  if (!bytes || K < 1) return SAS_ERR_INVALID_ARG;
   const int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
   size_t n = kStatusBytes + align256((size_t)B * Hq * T * sizeof(float));   // Delta
-  if (dtype == SAS_DT_BF16) n += masks_bytes(B, Hkv, T, Hq / Hkv);
+  if (dtype == SAS_DT_BF16) n += bwd_gather_workspace_bytes(B, Hq, Hkv, T, K);
   *bytes = n;
   return SAS_OK;
 }
@@ -161,8 +161,8 @@ int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float*
 
 int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
             const float* logG, const float* tau, const int32_t* tau_idx, const float* LSE, void* dQ, void* dK,
-            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, float sm_scale, void* ws,
-            size_t ws_bytes, void* stream) {
+            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget, float sm_scale,
+            void* ws, size_t ws_bytes, void* stream) {
   const void* ptrs[] = {Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
@@ -170,7 +170,8 @@ int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   if (st != SAS_OK) return st;
   if (!(sm_scale > 0.f)) return SAS_ERR_INVALID_ARG;
   size_t need = 0;
-  sas_bwd_workspace_size(B, Hq, Hkv, T, d, block, dtype, &need);
+  if (Kbudget < 1) return SAS_ERR_INVALID_ARG;
+  sas_bwd_workspace_size(B, Hq, Hkv, T, d, block, Kbudget, dtype, &need);
   if (!ws || !aligned256(ws) || ws_bytes < need) return SAS_ERR_WORKSPACE;
   TcProblem pb{};
   pb.B = B;
@@ -196,9 +197,9 @@ int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   if (dtype == SAS_DT_F32)
     return cuda_status(launch_bwd_simt(pb, static_cast<float*>(dQ), static_cast<float*>(dK), static_cast<float*>(dV),
                                        dLogG, delta, s));
-  uint32_t* masks =
-      reinterpret_cast<uint32_t*>(w + kStatusBytes + align256((size_t)B * Hq * T * sizeof(float)));
-  return cuda_status(launch_bwd_tc(pb, dQ, dK, dV, dLogG, reinterpret_cast<int32_t*>(w), masks, delta, s));
+  uint8_t* scratch = w + kStatusBytes + align256((size_t)B * Hq * T * sizeof(float));
+  return cuda_status(
+      launch_bwd_gather(pb, Kbudget, dQ, dK, dV, dLogG, reinterpret_cast<int32_t*>(w), delta, scratch, s));
 }
 
 int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen, const float* s,

@@ -1,0 +1,724 @@
+// SAS backward, KV-block outer with gathered query rows (sm_100a tensor cores).
+//
+// SAS paper (arXiv 2609.13141) Appendix E "Backward pass": recompute P from the
+// saved LSE, Delta = rowsum(O * dO), dS = P * (dP - Delta); the block log-gate
+// gradient is the per-block sum of dS over the block's tokens (summed over the
+// G query heads of the group, which share the gate).
+//
+// The selection is per query row and, for i.i.d. selector scores, rows of one
+// q-tile pick nearly disjoint blocks. Instead of running a q-tile over the union
+// of its rows' blocks (most of the tile masked), each CTA owns one KV block j of
+// one (b, g) and visits exactly the rows that attend it: its own 64 positions
+// (causal) and the positions that selected j, gathered P at a time (x G heads
+// = up to 128 rows) with TMA row-gather loads. Per tile, on tcgen05:
+//   S = Q K_j^T, dP = dO V_j^T              (M = 128 rows, N = 64 keys)
+//   dV_j^T += dO^T P, dK_j^T += Q^T dS      (M = 128 features, N = 64 keys, K = rows)
+//   dQ_rows = dS K_j                        (M = 128 rows, N = 128 features, K = 64 keys)
+// dK_j/dV_j stay in TMEM for the whole CTA; dQ partials leave through fp32
+// reductions into a workspace accumulator; dLogG[t, j] is written once, by the
+// CTA of block j. Tensor-core work equals the attended work (no union waste).
+//
+// Pre-pass (three small kernels): per-block counts of selecting rows, their
+// offsets, and the position lists.
+#include <algorithm>
+
+#include "sas_common.cuh"
+#include "sas_kernels.h"
+#include "sas_tmap.h"
+
+namespace sas {
+namespace gbwd {
+
+constexpr int D = 128;
+// Warps 0-3: softmax / dS (one thread per tile row); warp 4: control (row
+// positions and gates of each tile, K/V load); warp 5: MMA issuer; warps 6-9:
+// dQ flush (TMEM -> fp32 reductions); warps 10-15: Q/dO row gathers. The gather
+// bandwidth one SM sustains grows with the number of warps issuing copies, so
+// most warps load; the softmax works on 32 key columns at a time to keep the
+// kernel within 128 registers per thread.
+constexpr int THREADS = 512;
+constexpr int LOADER_WARP0 = 10, N_LOADER_WARPS = 6;
+constexpr int NST = 2;                           // Q/dO gather stages
+constexpr uint32_t HALF128 = 128 * 128;          // one d-half of a 128-row tile
+constexpr uint32_t TILE = 2 * HALF128;           // 128 rows x 128 features, bf16
+constexpr uint32_t KV_HALF = 64 * 128;
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = 2 * KV_HALF;
+constexpr uint32_t OFF_QD = 4 * KV_HALF;                  // stage s: Q at +2s*TILE, dO at +(2s+1)*TILE
+constexpr uint32_t OFF_P = OFF_QD + NST * 2 * TILE;       // P  [128 rows][64 keys] bf16 (16 KiB)
+constexpr uint32_t OFF_DS = OFF_P + 128 * 128;            // dS [128 rows][64 keys] bf16 (16 KiB)
+// Per stage: the tile's positions [128] int, the gate of each position for block j
+// [128] float (log2 units), and the chunk tails (LSE and Delta of the G heads) of
+// each position, `tail` bytes apiece (P positions * tail <= 2 KiB for every G).
+constexpr uint32_t CMETA_STAGE = 2048;
+constexpr uint32_t OFF_META = OFF_DS + 128 * 128;
+constexpr uint32_t META_STAGE = 128 * 4 + 128 * 4;
+constexpr uint32_t OFF_CMETA = OFF_META + NST * META_STAGE;
+constexpr uint32_t OFF_QROW = OFF_CMETA + NST * CMETA_STAGE;   // [2][128] global row of each dQ buffer row (-1: none)
+constexpr uint32_t OFF_RED = OFF_QROW + 2 * 128 * 4;      // [2][128] fp32 row sums for dLogG
+constexpr uint32_t OFF_BAR = OFF_RED + 2 * 128 * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
+// TMEM columns
+constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DV = 128, COL_DK = 192, COL_DQ0 = 256, TMEM_COLS = 512;
+
+struct Params {
+  const float* logG;
+  const float* tau;
+  const int32_t* tau_idx;
+  const float* LSE;
+  const int32_t* cnt;        // [B*Hkv*NB] selecting rows per block
+  const int32_t* off;        // [B*Hkv*NB] start of each block's list
+  const int32_t* list;       // positions
+  const int32_t* list_cap;   // [B*Hkv*NB] entries of each list that fit its region
+  // Packed rows, one chunk of `chunk` bytes per (b, g, position): Q [G][D] bf16,
+  // dO [G][D] bf16, then LSE[G] and Delta[G] fp32 (padded to 16 bytes).
+  const uint8_t* packed;
+  int chunk;
+  float* dQacc;              // [B*Hq*T*D] fp32, zeroed before the launch
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  float* dLogG;
+  int32_t* status;
+  int B, Hq, Hkv, T, NB, G, P;
+  float scale_log2;
+  float sm_scale;
+};
+
+struct Bars {
+  uint64_t kv_full, pos_ready[NST], qd_full[NST], qd_empty[NST], s_full, sp_free, p_full, pd_free, dq_done[2],
+      dq_free[2], qrow_full[2], fin;
+};
+
+// Position of list entry `idx` of block j: the block's own positions first, then the selecting rows.
+__device__ __forceinline__ int tile_position(const int32_t* lst, int own_n, int total, int j, int idx) {
+  if (idx >= total) return -1;
+  return idx < own_n ? j * kBlock + idx : lst[idx - own_n];
+}
+
+__device__ __forceinline__ void flush_dq(const Params& p, uint32_t taddr, int qrow) {
+#pragma unroll 1
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t v[32];
+    tmem_ld32(taddr + 32 * ch, v);
+    tmem_wait_ld();
+    if (qrow >= 0) {
+      float* dst = p.dQacc + (long long)qrow * D + 32 * ch;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        red_add_v4(dst + 4 * k, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), __uint_as_float(v[4 * k + 2]),
+                   __uint_as_float(v[4 * k + 3]));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    sas_bwd_gather_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
+  int* qrow_s = reinterpret_cast<int*>(smem + OFF_QROW);
+  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Group-major order: the CTAs running at the same time mostly belong to one
+  // (b, g), so the Q/dO rows they gather (that group's heads only) stay in L2.
+  // Within a group, small j (longest row lists) first.
+  const int bg = blockIdx.x / p.NB;
+  const int j = blockIdx.x % p.NB;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int PP = p.P, G = p.G;
+  const int rows_used = G * PP;
+  const int own_n = min(kBlock, p.T - j * kBlock);
+  const int sel_n = min(p.cnt[(long long)bg * p.NB + j], p.list_cap[(long long)bg * p.NB + j]);
+  const int total = own_n + sel_n;
+  const int n_tiles = (total + PP - 1) / PP;
+  const int32_t* lst = p.list + p.off[(long long)bg * p.NB + j];
+  int32_t* status = p.status;
+
+  if (warp == 5) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (tid == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&bars->pos_ready[i], 1);
+      mbar_init(&bars->qd_full[i], 1 + N_LOADER_WARPS);   // control (metadata) + loader warps (rows)
+      mbar_init(&bars->qd_empty[i], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->sp_free, 4);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->pd_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->dq_done[i], 1);
+      mbar_init(&bars->dq_free[i], 4);
+      mbar_init(&bars->qrow_full[i], 4);
+    }
+    mbar_init(&bars->fin, 1);
+    fence_barrier_init();
+  }
+  if (rows_used < 128) {   // rows never gathered stay zero
+    const int per = (128 - rows_used) * 8;
+    for (int i = tid; i < per * 2 * 2 * NST; i += THREADS) {
+      const int tile = i / (2 * per), half = (i / per) & 1, rem = i % per;
+      *reinterpret_cast<uint4*>(smem + OFF_QD + tile * TILE + half * HALF128 + (rows_used + rem / 8) * 128 +
+                                (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t s_base = smem_u32(smem);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ control: positions + metadata
+    if (lane == 0) {
+      mbar_expect_tx(&bars->kv_full, 4 * KV_HALF);
+      tma_load_3d(smem + OFF_K, &tmK, &bars->kv_full, 0, j * kBlock, bg);
+      tma_load_3d(smem + OFF_K + KV_HALF, &tmK, &bars->kv_full, 64, j * kBlock, bg);
+      tma_load_3d(smem + OFF_V, &tmV, &bars->kv_full, 0, j * kBlock, bg);
+      tma_load_3d(smem + OFF_V + KV_HALF, &tmV, &bars->kv_full, 64, j * kBlock, bg);
+    }
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i % NST;
+      bool ok = true;
+      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      int* pos = reinterpret_cast<int*>(smem + OFF_META + st * META_STAGE);
+      float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
+      int tl[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) tl[u] = (lane + 32 * u < PP) ? tile_position(lst, own_n, total, j, i * PP + lane + 32 * u) : -1;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (lane + 32 * u < PP) pos[lane + 32 * u] = tl[u];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->pos_ready[st]);
+      // Gate of block j for each selecting position (log2 units); own positions get 0.
+      float gv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = tl[u];
+        gv[u] = (t >= 0 && t / kBlock != j) ? __ldg(p.logG + ((long long)bg * p.T + t) * p.NB + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (lane + 32 * u < PP) gate[lane + 32 * u] = gv[u] * kLog2e;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qd_full[st]);
+    }
+    if (lane == 0) mbar_wait_drain(&bars->kv_full, 0);
+  } else if (warp >= LOADER_WARP0) {
+    // ------------------------------------------------------------------ loaders: Q / dO row gathers
+    const int lt = tid - LOADER_WARP0 * 32;
+    constexpr int NL = N_LOADER_WARPS * 32;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i % NST;
+      bool ok = true;
+      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status);
+      if (ok) ok = mbar_wait(&bars->pos_ready[st], (i / NST) & 1, status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
+      const int first = pos[0];
+      const uint32_t qd = s_base + OFF_QD + st * 2 * TILE;
+      const uint32_t cm = s_base + OFF_CMETA + st * CMETA_STAGE;
+      // Pieces of 16 bytes of each position's chunk: 32*G of Q/dO rows (ordered
+      // tensor, head, piece), then the tail. The loaders walk (position, piece)
+      // with a stride of NL pieces, so consecutive lanes copy consecutive bytes.
+      const int rows_pieces = 32 * G;
+      const int per_pos = p.chunk >> 4;
+      const int tail_bytes = p.chunk - rows_pieces * 16;
+      const uint8_t* base = p.packed + (long long)bg * p.T * p.chunk;
+      int pp = 0, piece = lt;
+      while (piece >= per_pos) {
+        piece -= per_pos;
+        ++pp;
+      }
+      while (pp < PP) {
+        const int t0 = pos[pp];
+        const uint8_t* src = base + (long long)(t0 >= 0 ? t0 : first) * p.chunk + piece * 16;
+        if (piece < rows_pieces) {
+          const int tensor = piece >= 16 * G;
+          const int rem2 = piece - tensor * 16 * G;
+          const int hh = rem2 >> 4, c16 = rem2 & 15;
+          const int half = c16 >> 3, ch = c16 & 7;
+          cp_async16(qd + tensor * TILE + half * HALF128 + sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)ch), src);
+        } else {
+          cp_async16(cm + pp * tail_bytes + (piece - rows_pieces) * 16, src);
+        }
+        piece += NL;
+        while (piece >= per_pos) {
+          piece -= per_pos;
+          ++pp;
+        }
+      }
+      cp_async_commit_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qd_full[st]);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    // A polling state machine: S/dP of the next tile and dV/dK/dQ of the oldest
+    // tile are issued as soon as their inputs are ready, in whichever order.
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc_bf16(128, 64, 0, 0);    // rows x keys, K = features
+      const uint32_t idesc_t = make_idesc_bf16(128, 64, 1, 1);    // features x keys, K = rows
+      const uint32_t idesc_q = make_idesc_bf16(128, D, 0, 1);     // rows x features, K = keys
+      bool ok = mbar_wait(&bars->kv_full, 0, status);
+      int ns = 0, nb = 0;
+      uint64_t t_last = global_ns();
+      uint32_t spins = 0;
+      while (ok && nb < n_tiles) {
+        bool prog = false;
+        if (ns < n_tiles) {
+          const int st = ns % NST;
+          if (mbar_try_wait(&bars->qd_full[st], (ns / NST) & 1) &&
+              (ns == 0 || mbar_try_wait(&bars->sp_free, (ns - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t qb = s_base + OFF_QD + st * 2 * TILE;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
+              umma_ss(tmem + COL_S, make_sdesc(qb + half * HALF128 + koff, 16, 1024),
+                      make_sdesc(s_base + OFF_K + half * KV_HALF + koff, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
+              umma_ss(tmem + COL_DP, make_sdesc(qb + TILE + half * HALF128 + koff, 16, 1024),
+                      make_sdesc(s_base + OFF_V + half * KV_HALF + koff, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars->s_full);
+            ++ns;
+            prog = true;
+          }
+        }
+        if (nb < ns && mbar_try_wait(&bars->p_full, nb & 1) &&
+            (nb < 2 || mbar_try_wait(&bars->dq_free[nb & 1], ((nb - 2) >> 1) & 1))) {
+          tc_fence_after();
+          const int st = nb % NST, qb_ = nb & 1;
+          const uint32_t qb = s_base + OFF_QD + st * 2 * TILE;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per MMA
+            umma_ss(tmem + COL_DV, make_sdesc(qb + TILE + ks * 2048, HALF128, 1024),
+                    make_sdesc(s_base + OFF_P + ks * 2048, HALF128, 1024), idesc_t, (nb > 0 || ks > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            umma_ss(tmem + COL_DK, make_sdesc(qb + ks * 2048, HALF128, 1024),
+                    make_sdesc(s_base + OFF_DS + ks * 2048, HALF128, 1024), idesc_t, (nb > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->qd_empty[st]);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {   // dQ partial = dS K_j, K = 64 keys
+            umma_ss(tmem + COL_DQ0 + 128 * qb_, make_sdesc(s_base + OFF_DS + ks * 32, 16, 1024),
+                    make_sdesc(s_base + OFF_K + ks * 2048, KV_HALF, 1024), idesc_q, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->dq_done[qb_]);
+          umma_commit(&bars->pd_free);
+          ++nb;
+          prog = true;
+        }
+        if (prog) {
+          t_last = global_ns();
+          spins = 0;
+        } else if ((++spins & 255u) == 0u) {
+          if (*reinterpret_cast<volatile int32_t*>(status) != 0) break;
+          if (global_ns() - t_last > kWaitLimitNs) {
+            set_status(status, SAS_DEV_ERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+      umma_commit(&bars->fin);
+      mbar_wait_drain(&bars->fin, 0);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------ dQ flush (warps 6-9)
+    const int quarter = warp & 3;                    // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int qb = i & 1;
+      if (!warp_wait(&bars->qrow_full[qb], (i >> 1) & 1, status)) break;
+      if (!warp_wait(&bars->dq_done[qb], (i >> 1) & 1, status)) break;
+      tc_fence_after();
+      flush_dq(p, tmem + lane_base + COL_DQ0 + 128 * qb, qrow_s[qb * 128 + row]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_free[qb]);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax / dS (warps 0-3)
+    const int r = tid;
+    const int hh = r / PP;
+    const int h = g * G + (hh < G ? hh : 0);
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i % NST, qb = i & 1;
+      bool step_ok = warp_wait(&bars->qd_full[st], (i / NST) & 1, status);
+      int t = -1;
+      float lse2 = 0.f, dlt = 0.f, bias2 = 0.f;
+      if (step_ok && r < rows_used) {
+        const int pp = r % PP;
+        t = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE)[pp];
+        if (t >= 0) {
+          const float* tail =
+              reinterpret_cast<const float*>(smem + OFF_CMETA + st * CMETA_STAGE + pp * (p.chunk - 512 * G));
+          lse2 = tail[hh] * kLog2e;
+          dlt = tail[G + hh];
+          bias2 = reinterpret_cast<const float*>(smem + OFF_META + st * META_STAGE + 128 * 4)[pp];
+        }
+      }
+      const bool valid = step_ok && t >= 0;
+      const bool own = valid && (t / kBlock == j);
+      const int lim = own ? t - j * kBlock : 63;
+      if (step_ok) step_ok = warp_wait(&bars->s_full, i & 1, status);
+      // Two passes of 32 key columns: S, dP -> P, dS (bf16) into shared memory.
+      if (step_ok) tc_fence_after();
+      if (step_ok && i >= 1) {
+        // P / dS shared tiles are free once tile i-1's MMAs completed.
+        step_ok = warp_wait(&bars->pd_free, (i - 1) & 1, status);
+      }
+      float rs = 0.f;
+      if (step_ok) {
+#pragma unroll 1
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tmem + lane_base + COL_S + 32 * hc, sr);
+          tmem_ld32(tmem + lane_base + COL_DP + 32 * hc, dr);
+          tmem_wait_ld();
+          if (hc == 1) {   // S / dP of this tile fully read: the next tile's S may overwrite them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->sp_free);
+          }
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t pw[4], sw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              float pv[2], dv[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int kk = ch * 8 + 2 * k + e;       // column within this half
+                const float sv = __uint_as_float(sr[kk]);
+                const float dp = __uint_as_float(dr[kk]);
+                pv[e] = (valid && 32 * hc + kk <= lim) ? ex2(fmaf(sv, p.scale_log2, bias2) - lse2) : 0.f;
+                dv[e] = pv[e] * (dp - dlt);
+                rs += dv[e];
+              }
+              pw[k] = pack_bf16(pv[0], pv[1]);
+              sw[k] = pack_bf16(dv[0], dv[1]);
+            }
+            const uint32_t o = sw128_offset((uint32_t)r, (uint32_t)(4 * hc + ch));
+            *reinterpret_cast<uint4*>(smem + OFF_P + o) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            *reinterpret_cast<uint4*>(smem + OFF_DS + o) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      // The dQ row map of buffer qb is reusable once tile i-2 was flushed.
+      if (step_ok && i >= 2) step_ok = warp_wait(&bars->dq_free[qb], ((i - 2) >> 1) & 1, status);
+      if (step_ok) {
+        qrow_s[qb * 128 + r] = valid ? (int)(((long long)b * p.Hq + h) * p.T + t) : -1;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars->qrow_full[qb]);
+          mbar_arrive(&bars->p_full);
+        }
+      }
+      // dLogG[t, j] for positions that selected j: sum over the G heads (rows hh*PP + pp).
+      red[qb * 128 + r] = (valid && !own) ? rs : 0.f;
+      ok = named_bar_and(1, 128, step_ok);
+      if (!ok) break;
+      if (r < PP && valid && !own) {
+        float acc = 0.f;
+        for (int q = 0; q < G; ++q) acc += red[qb * 128 + q * PP + r];
+        p.dLogG[((long long)bg * p.T + t) * p.NB + j] = acc;
+      }
+    }
+    if (ok && n_tiles > 0) ok = warp_wait(&bars->pd_free, (n_tiles - 1) & 1, status);
+    if (ok) {
+      tc_fence_after();
+      const int dd = r;   // TMEM lane = feature
+      const long long key0 = (long long)bg * p.T + (long long)j * kBlock;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? COL_DV : COL_DK;
+        __nv_bfloat16* dst = which == 0 ? p.dV : p.dK;
+        const float scl = which == 0 ? 1.f : p.sm_scale;
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + col + 32 * ch, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int key = 32 * ch + k;
+            if (key < own_n)
+              dst[(key0 + key) * D + dd] = __float2bfloat16_rn(n_tiles > 0 ? __uint_as_float(v[k]) * scl : 0.f);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------- pre-pass
+// Count, per (b, g, block), the positions whose selection contains the block.
+__global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
+                                                    const int32_t* __restrict__ tau_idx, int32_t* __restrict__ cnt,
+                                                    long long rows, int T, int NB) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const long long bg = row / T;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  const float tv = tau[row];
+  const int ti = tau_idx[row];
+  const float* v = logG + row * (long long)NB;
+  for (int m = lane; m < c; m += 32) {
+    const float x = v[m];
+    if (x > tv || (x == tv && m <= ti)) atomicAdd(cnt + bg * NB + m, 1);
+  }
+}
+
+// Offsets: each (b, g) owns a region of T * min(H, NB) entries; off = region + prefix of counts.
+__global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ cnt, int32_t* __restrict__ off,
+                                                       int32_t* __restrict__ cursor, int32_t* __restrict__ cap,
+                                                       int32_t* status, int NB, long long region) {
+  __shared__ int32_t warp_sums[32];
+  const long long bg = blockIdx.x;
+  int base = 0;
+  for (int j0 = 0; j0 < NB; j0 += 1024) {
+    const int j = j0 + threadIdx.x;
+    const int v = j < NB ? cnt[bg * NB + j] : 0;
+    int incl = v;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_sums[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int ws = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += u;
+      }
+      warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    const int excl = incl - v + (w > 0 ? warp_sums[w - 1] : 0);
+    if (j < NB) {
+      // Lists beyond the (b, g) region (only possible if the threshold kept more
+      // than K-1 blocks for some row) are cut and flagged.
+      const long long start = base + excl;
+      const long long room = region - start;
+      off[bg * NB + j] = (int32_t)(bg * region + (start < region ? start : region));
+      cap[bg * NB + j] = (int32_t)(room <= 0 ? 0 : (room < v ? room : v));
+      if (room < v) set_status(status, SAS_DEV_ERR_BOUNDS);
+      cursor[bg * NB + j] = 0;
+    }
+    base += warp_sums[31];
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
+                                                   const int32_t* __restrict__ tau_idx,
+                                                   const int32_t* __restrict__ off, const int32_t* __restrict__ cap,
+                                                   int32_t* __restrict__ cursor, int32_t* __restrict__ list,
+                                                   long long rows, int T, int NB) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const long long bg = row / T;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  const float tv = tau[row];
+  const int ti = tau_idx[row];
+  const float* v = logG + row * (long long)NB;
+  for (int m = lane; m < c; m += 32) {
+    const float x = v[m];
+    if (x > tv || (x == tv && m <= ti)) {
+      const int slot = atomicAdd(cursor + bg * NB + m, 1);
+      if (slot < cap[bg * NB + m]) list[off[bg * NB + m] + slot] = t;
+    }
+  }
+}
+
+// Packs the rows of each (b, g, position) into one chunk: Q [G][D], dO [G][D]
+// (bf16), LSE [G] and Delta [G] = rowsum(O * dO) (fp32). One warp per (b, g, t, head).
+__global__ void __launch_bounds__(256) pack_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                   const __nv_bfloat16* __restrict__ dO,
+                                                   const __nv_bfloat16* __restrict__ O, const float* __restrict__ LSE,
+                                                   uint8_t* __restrict__ packed, long long n_rows, int T, int G, int Hq,
+                                                   int Hkv, int chunk) {
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // (bg, t, hh)
+  const int lane = threadIdx.x & 31;
+  if (w >= n_rows) return;
+  const int hh = (int)(w % G);
+  const long long bt = w / G;
+  const int t = (int)(bt % T);
+  const long long bg = bt / T;
+  const long long b = bg / Hkv, g = bg % Hkv;
+  const long long row = (b * Hq + g * G + hh) * T + t;
+  const uint2 q = *reinterpret_cast<const uint2*>(Q + row * D + lane * 4);
+  const uint2 d = *reinterpret_cast<const uint2*>(dO + row * D + lane * 4);
+  const uint2 o = *reinterpret_cast<const uint2*>(O + row * D + lane * 4);
+  uint8_t* c = packed + bt * chunk;
+  *reinterpret_cast<uint2*>(c + hh * D * 2 + lane * 8) = q;
+  *reinterpret_cast<uint2*>(c + (G + hh) * D * 2 + lane * 8) = d;
+  const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
+  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float2 x = __bfloat1622float2(o2[k]);
+    const float2 y = __bfloat1622float2(d2[k]);
+    acc = fmaf(x.x, y.x, acc);
+    acc = fmaf(x.y, y.y, acc);
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    float* tail = reinterpret_cast<float*>(c + 2 * G * D * 2);
+    tail[hh] = LSE[row];
+    tail[G + hh] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                         long long n4, float scale) {
+  const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = reinterpret_cast<const float4*>(acc)[i];
+  uint2 o;
+  o.x = pack_bf16(v.x * scale, v.y * scale);
+  o.y = pack_bf16(v.z * scale, v.w * scale);
+  reinterpret_cast<uint2*>(dq)[i] = o;
+}
+
+}  // namespace gbwd
+
+// Bytes of one packed position: Q and dO rows of the G heads, then LSE and Delta padded to 16 bytes.
+static size_t packed_chunk_bytes(int G) { return (size_t)4 * G * 128 + ((size_t)8 * G + 15) / 16 * 16; }
+
+size_t bwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K) {
+  const int NB = T / kBlock;
+  const long long nbg = (long long)B * Hkv;
+  const long long region = (long long)T * max(1, min(K - 1, NB));
+  auto a256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  size_t n = 0;
+  n += a256((size_t)B * Hq * T * 128 * sizeof(float));     // dQ accumulator
+  n += 4 * a256((size_t)nbg * NB * sizeof(int32_t));       // counts, offsets, caps, cursors
+  n += a256((size_t)nbg * region * sizeof(int32_t));       // position lists
+  n += a256((size_t)B * Hkv * T * packed_chunk_bytes(Hq / Hkv));   // packed rows
+  return n;
+}
+
+cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, void* dV, float* dLogG, int32_t* status,
+                              float* delta, uint8_t* scratch, cudaStream_t st) {
+  using namespace gbwd;
+  const int NB = pb.NB;
+  const long long nbg = (long long)pb.B * pb.Hkv;
+  const long long rows = nbg * pb.T;
+  const long long qrows = (long long)pb.B * pb.Hq * pb.T;
+  const long long region = (long long)pb.T * std::max(1, std::min(K - 1, NB));
+  auto a256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  float* dQacc = reinterpret_cast<float*>(scratch);
+  size_t o = a256((size_t)qrows * D * sizeof(float));
+  int32_t* cnt = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * NB * sizeof(int32_t));
+  int32_t* off = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * NB * sizeof(int32_t));
+  int32_t* cursor = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * NB * sizeof(int32_t));
+  int32_t* cap = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * NB * sizeof(int32_t));
+  int32_t* list = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * region * sizeof(int32_t));
+  uint8_t* packed = scratch + o;
+  const int chunk = (int)packed_chunk_bytes(pb.G);
+
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(dLogG, 0, (size_t)rows * NB * sizeof(float), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(dQacc, 0, (size_t)qrows * D * sizeof(float), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st)) != cudaSuccess) return e;
+  count_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pb.logG, pb.tau, pb.tau_idx, cnt, rows, pb.T, NB);
+  count_launch();
+  offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(cnt, off, cursor, cap, status, NB, region);
+  count_launch();
+  fill_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pb.logG, pb.tau, pb.tau_idx, off, cap, cursor, list, rows,
+                                                          pb.T, NB);
+  count_launch();
+  pack_kernel<<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(pb.Q), reinterpret_cast<const __nv_bfloat16*>(pb.dO),
+      reinterpret_cast<const __nv_bfloat16*>(pb.O), pb.LSE, packed, qrows, pb.T, pb.G, pb.Hq, pb.Hkv, chunk);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  const QTileShape qs = qtile_shape(pb.G, pb.T, NB);
+  CUtensorMap tk, tv;
+  if (!make_tmap_bf16_3d(&tk, pb.K, pb.d, pb.T, (uint64_t)nbg, 64) ||
+      !make_tmap_bf16_3d(&tv, pb.V, pb.d, pb.T, (uint64_t)nbg, 64))
+    return cudaErrorInvalidValue;
+  Params prm;
+  prm.logG = pb.logG;
+  prm.tau = pb.tau;
+  prm.tau_idx = pb.tau_idx;
+  prm.LSE = pb.LSE;
+  prm.cnt = cnt;
+  prm.off = off;
+  prm.list = list;
+  prm.list_cap = cap;
+  prm.dQacc = dQacc;
+  prm.packed = packed;
+  prm.chunk = chunk;
+  prm.dK = reinterpret_cast<__nv_bfloat16*>(dK);
+  prm.dV = reinterpret_cast<__nv_bfloat16*>(dV);
+  prm.dLogG = dLogG;
+  prm.status = status;
+  prm.B = pb.B;
+  prm.Hq = pb.Hq;
+  prm.Hkv = pb.Hkv;
+  prm.T = pb.T;
+  prm.NB = NB;
+  prm.G = pb.G;
+  prm.P = qs.P;
+  prm.scale_log2 = pb.sm_scale * kLog2e;
+  prm.sm_scale = pb.sm_scale;
+  if ((e = cudaFuncSetAttribute(sas_bwd_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+      cudaSuccess)
+    return e;
+  sas_bwd_gather_kernel<<<(unsigned)(nbg * NB), THREADS, SMEM_BYTES, st>>>(tk, tv, prm);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long n4 = qrows * D / 4;
+  dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dQacc, reinterpret_cast<__nv_bfloat16*>(dQ), n4,
+                                                                  pb.sm_scale);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace sas

@@ -43,9 +43,11 @@ struct TcProblem {
 // bf16 tensor-core forward; ws holds the status word and the tile masks.
 cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* status, uint32_t* masks,
                           cudaStream_t st);
-// bf16 tensor-core backward.
-cudaError_t launch_bwd_tc(const TcProblem& pb, void* dQ, void* dK, void* dV, float* dLogG, int32_t* status,
-                          uint32_t* masks, float* delta, cudaStream_t st);
+// bf16 tensor-core backward (KV-block outer, gathered query rows); `scratch`
+// holds bwd_gather_workspace_bytes bytes.
+size_t bwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K);
+cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, void* dV, float* dLogG, int32_t* status,
+                              float* delta, uint8_t* scratch, cudaStream_t st);
 
 // fp32 CUDA-core forward / backward.
 cudaError_t launch_fwd_simt(const TcProblem& pb, float* O, float* LSE, cudaStream_t st);

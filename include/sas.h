@@ -114,7 +114,8 @@ SAS_API int sas_select_threshold(const float* logG, float* tau, int32_t* tau_idx
  * device status word.
  */
 SAS_API int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes);
-SAS_API int sas_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes);
+SAS_API int sas_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int K, int dtype,
+                               size_t* bytes);
 SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int block, int K, size_t* bytes);
 
 /*
@@ -143,12 +144,16 @@ SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, cons
  *   dLogG[b,g,t,m] = sum_{h in g} sum_{i in block m} dS[h,t,i] for selected m, 0 otherwise.
  * Inputs as for sas_fwd plus O (the forward output), dO and LSE (the forward's).
  * Outputs dQ [B,Hq,T,d], dK/dV [B,Hkv,T,d] of `dtype`; dLogG [B,Hkv,T,NB] fp32
- * (fully written: zero outside the selection). ws: sas_bwd_workspace_size bytes.
+ * (fully written: zero outside the selection). Kbudget: the budget K given to
+ * sas_select_threshold (the threshold keeps at most K-1 historical blocks per row;
+ * internal per-block row lists are sized by it; a threshold that keeps more is
+ * reported as a device-side bounds error). ws: sas_bwd_workspace_size bytes
+ * (for bf16 it holds an fp32 dQ accumulator and the per-block row lists).
  */
 SAS_API int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
             const float* logG, const float* tau, const int32_t* tau_idx, const float* LSE, void* dQ, void* dK,
-            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, float sm_scale, void* ws,
-            size_t ws_bytes, void* stream);
+            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget, float sm_scale,
+            void* ws, size_t ws_bytes, void* stream);
 
 /*
  * sas_decode_fwd - one sparse decode step per sequence (SAS paper §4.3

@@ -22,7 +22,7 @@ def run_gpu(inp, logG32, tau, tidx, w):
     Q, K, V, dO = (dev(inp[k]) for k in ("Q", "K", "V", "dO"))
     lg, ta, ti = dev(logG32), dev(tau), dev(tidx)
     O, LSE = binding.forward(Q, K, V, lg, ta, ti, w.sm_scale)
-    dQ, dK, dV, dLogG = binding.backward(Q, K, V, O, dO, lg, ta, ti, LSE, w.sm_scale)
+    dQ, dK, dV, dLogG = binding.backward(Q, K, V, O, dO, lg, ta, ti, LSE, w.K, w.sm_scale)
     torch.cuda.synchronize()
     return {k: to_np(v) for k, v in dict(O=O, LSE=LSE, dQ=dQ, dK=dK, dV=dV, dLogG=dLogG).items()}
 
