@@ -249,55 +249,59 @@ def run_gpu(args):
         if ev:
             ev[3].record(stream)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize(device)
-    if binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b):
-        raise RuntimeError("kernel-side timeout during warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    barrier(device)
-    torch.cuda.synchronize(device)
-    launches0 = binding.launch_count()
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.zero_()      # L2 flush between timed steps (outside the events)
-            step(evs[i])
-        torch.cuda.synchronize(device)
-    launches = binding.launch_count() - launches0
-    barrier(device)
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    gate_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    total_ms = reduce_max(sum(step_ms), device)
-    ms_per_step = total_ms / args.steps
-    value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
-
-    # Dominant call (the backward) against the tensor-core roofline.
-    bwd_avg = statistics.mean(bwd_ms)
-    fwd_avg = statistics.mean(fwd_ms)
-    dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
-        ("sas_fwd", fwd_avg, fwd_flops)
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
-                "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
-                "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
-                "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
-                "gate_select_ms": round(statistics.mean(gate_ms), 4)}
-
     legs = set(args.legs.split(","))
+    if "step" in legs:
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize(device)
+        if binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b):
+            raise RuntimeError("kernel-side timeout during warm-up")
+
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        barrier(device)
+        torch.cuda.synchronize(device)
+        launches0 = binding.launch_count()
+        with ClockSampler(local) as clk:
+            for i in range(args.steps):
+                flush.zero_()      # L2 flush between timed steps (outside the events)
+                step(evs[i])
+            torch.cuda.synchronize(device)
+        launches = binding.launch_count() - launches0
+        barrier(device)
+        step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+        fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+        bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+        gate_ms = [e[0].elapsed_time(e[1]) for e in evs]
+        total_ms = reduce_max(sum(step_ms), device)
+        ms_per_step = total_ms / args.steps
+        value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
+
+        # Dominant call (the backward) against the tensor-core roofline.
+        bwd_avg = statistics.mean(bwd_ms)
+        fwd_avg = statistics.mean(fwd_ms)
+        dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
+            ("sas_fwd", fwd_avg, fwd_flops)
+        achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                    "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
+                    "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
+                    "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
+                    "gate_select_ms": round(statistics.mean(gate_ms), 4)}
+    else:
+        value, ms_per_step, launches, roofline, clk = None, None, 0, None, ClockSampler(local)
+
     # End to end through the C ABI from pinned host buffers, results copied back.
     e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
     dec = run_decode(args, device, stream, binding, peaks) if "decode" in legs else None
 
     result = {
         "metric": "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd step)",
-        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "value": round(value, 3) if value is not None else None, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4) if ms_per_step is not None else None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "qwen3_4b_t8k layer fwd+bwd: B=1 Hq=32 Hkv=8 d=128 T=8192 block=64 K=16 "
                                "(1024-token budget), s~N(0,2) + 3 planted blocks per query",

@@ -314,13 +314,77 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp-level radix select of the H-th largest value among row[0..c) (c > H > 0),
-// 8-bit digits, most significant first, counting in a per-warp shared-memory
-// histogram. Returns the order-preserving key of that value and, in
-// *take_equal, how many values equal to it are kept (the lowest indices).
+// Top-K threshold of one row by a warp: the H-th largest value among row[0..c)
+// (c > H > 0), equal values going to the lower index.
+//
+// Keys (order-preserving uint32 images of the values, -0.0 == +0.0) are held in
+// registers, key of index m = lane + 32*i in keys[i] (rows up to 32*KREG values).
+// The H-th largest key is found by an MSB-first radix select with 8-bit digits,
+// counting in a per-warp shared-memory histogram of 256 bins.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t warp_radix_select(const float* __restrict__ row, int c, int H, uint32_t* hist,
-                                      int* take_equal) {
+constexpr int kSelectReg = 32;   // rows of up to 1024 values are selected from registers
+
+template <int KREG>
+__device__ __forceinline__ void load_row_keys(const float* __restrict__ row, int c, uint32_t (&keys)[KREG]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    const int m = lane + 32 * i;
+    keys[i] = (m < c) ? float_key(__ldg(row + m)) : 0u;
+  }
+}
+
+// Key of the H-th largest value; *take_equal = how many values equal to it are kept.
+// MSB-first bisection, one bit per step: the candidate keeps bit b when at least
+// `remaining` keys share the candidate's higher bits and have bit b set. Counts
+// use a warp reduction (no shared-memory atomics, so skewed digit distributions
+// cost nothing extra).
+template <int KREG>
+__device__ __forceinline__ uint32_t radix_select_keys(const uint32_t (&keys)[KREG], int c, int H, uint32_t* hist,
+                                                      int* take_equal) {
+  (void)hist;
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0u;
+  int remaining = H;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = (prefix | (1u << bit)) >> bit;
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) cnt += (lane + 32 * i < c && (keys[i] >> bit) == cand) ? 1 : 0;
+    cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
+    if (cnt >= remaining)
+      prefix |= 1u << bit;
+    else
+      remaining -= cnt;
+  }
+  *take_equal = remaining;
+  return prefix;
+}
+
+// Index of the take_equal-th (1-based) value equal to tkey, ascending.
+template <int KREG>
+__device__ __forceinline__ int tie_index_keys(const uint32_t (&keys)[KREG], int c, uint32_t tkey, int take_equal) {
+  const int lane = threadIdx.x & 31;
+  int run = 0;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    const int m = lane + 32 * i;
+    const uint32_t bal = __ballot_sync(0xffffffffu, m < c && keys[i] == tkey);
+    const int cnt = __popc(bal);
+    if (run + cnt >= take_equal) {
+      uint32_t bb = bal;
+      for (int k = 1; k < take_equal - run; ++k) bb &= bb - 1u;
+      return 32 * i + __ffs(bb) - 1;
+    }
+    run += cnt;
+  }
+  return -1;
+}
+
+// Generic path for rows longer than 32*kSelectReg: keys re-read from memory on every pass.
+__device__ __forceinline__ uint32_t radix_select_global(const float* __restrict__ row, int c, int H, uint32_t* hist,
+                                                        int* take_equal) {
   const int lane = threadIdx.x & 31;
   uint32_t prefix = 0u, pmask = 0u;
   int remaining = H;
@@ -335,7 +399,6 @@ __device__ __forceinline__ uint32_t warp_radix_select(const float* __restrict__ 
       if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncwarp();
-    // Lane l owns digits 255-8l down to 248-8l (descending across lanes).
     uint32_t cnt[8];
     uint32_t local = 0u;
 #pragma unroll
@@ -374,6 +437,23 @@ __device__ __forceinline__ uint32_t warp_radix_select(const float* __restrict__ 
   }
   *take_equal = remaining;
   return prefix;
+}
+
+__device__ __forceinline__ int tie_index_global(const float* __restrict__ row, int c, uint32_t tkey, int take_equal) {
+  const int lane = threadIdx.x & 31;
+  int run = 0;
+  for (int base = 0; base < c; base += 32) {
+    const int m = base + lane;
+    const uint32_t bal = __ballot_sync(0xffffffffu, m < c && float_key(row[m]) == tkey);
+    const int cnt = __popc(bal);
+    if (run + cnt >= take_equal) {
+      uint32_t bb = bal;
+      for (int k = 1; k < take_equal - run; ++k) bb &= bb - 1u;
+      return base + __ffs(bb) - 1;
+    }
+    run += cnt;
+  }
+  return -1;
 }
 
 }  // namespace sas

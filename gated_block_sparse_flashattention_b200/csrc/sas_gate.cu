@@ -35,6 +35,36 @@ __global__ void __launch_bounds__(256) gate_normalize_kernel(const float* __rest
   for (int m = lane; m < NB; m += 32) dst[m] = (m < c) ? (__ldg(src + m) - lse) : -INFINITY;
 }
 
+// Threshold (tau, tau_idx) and optional ascending index list of one row whose
+// keys fit in KREG registers per lane.
+template <int KREG>
+__device__ __forceinline__ void select_row_regs(const float* __restrict__ v, int c, int H, uint32_t* hist,
+                                                float* tau_out, int32_t* tidx_out, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t keys[KREG];
+  load_row_keys(v, c, keys);
+  int take_eq = 0;
+  const uint32_t tkey = radix_select_keys(keys, c, H, hist, &take_eq);
+  const int tidx = tie_index_keys(keys, c, tkey, take_eq);
+  if (lane == 0) {
+    *tau_out = key_float(tkey);
+    *tidx_out = tidx;
+  }
+  if (out) {
+    int pos = 0;
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) {
+      if (32 * i >= c) break;
+      const int m = lane + 32 * i;
+      const bool take = m < c && (keys[i] > tkey || (keys[i] == tkey && m <= tidx));
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(bal & ((1u << lane) - 1u))] = m;
+      pos += __popc(bal);
+    }
+    for (int k = pos + lane; k < H; k += 32) out[k] = -1;
+  }
+}
+
 __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __restrict__ logG, float* __restrict__ tau,
                                                                int32_t* __restrict__ tau_idx,
                                                                int32_t* __restrict__ sel, long long rows, int T,
@@ -66,24 +96,22 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
       for (int k = lane; k < H; k += 32) out[k] = (k < c) ? k : -1;
     return;
   }
-  int take_eq = 0;
-  const uint32_t tkey = warp_radix_select(v, c, H, hist_all[wid], &take_eq);
-  // tau_idx: the take_eq-th (1-based) index, ascending, among values whose key equals tkey.
-  int tidx = -1;
-  int run = 0;
-  for (int base = 0; base < c; base += 32) {
-    const int m = base + lane;
-    const bool eq = (m < c) && (float_key(v[m]) == tkey);
-    const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-    const int cnt = __popc(bal);
-    if (run + cnt >= take_eq) {
-      uint32_t b = bal;
-      for (int k = 1; k < take_eq - run; ++k) b &= b - 1u;   // drop the lower set bits
-      tidx = base + __ffs(b) - 1;
-      break;
-    }
-    run += cnt;
+  if (c <= 32 * kSelectReg) {
+    // Keys in registers: one read of the row, four radix passes, the tie index
+    // and the index list all work on them (register width picked by row length).
+    if (c <= 128)
+      select_row_regs<4>(v, c, H, hist_all[wid], tau + row, tau_idx + row, out);
+    else if (c <= 256)
+      select_row_regs<8>(v, c, H, hist_all[wid], tau + row, tau_idx + row, out);
+    else if (c <= 512)
+      select_row_regs<16>(v, c, H, hist_all[wid], tau + row, tau_idx + row, out);
+    else
+      select_row_regs<32>(v, c, H, hist_all[wid], tau + row, tau_idx + row, out);
+    return;
   }
+  int take_eq = 0;
+  const uint32_t tkey = radix_select_global(v, c, H, hist_all[wid], &take_eq);
+  const int tidx = tie_index_global(v, c, tkey, take_eq);
   if (lane == 0) {
     tau[row] = key_float(tkey);
     tau_idx[row] = tidx;
