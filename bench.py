@@ -366,52 +366,58 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
 
 
 def run_decode(args, device, stream, binding, peaks):
-    """Decode step (16 sequences x 1 token over a 32768-token cache) in a CUDA graph, L2 flushed between steps."""
+    """Decode step (16 sequences x 1 token over a 32768-token cache), 16 steps per CUDA graph.
+
+    The graph holds 16 decode steps back to back, each with its own seeded
+    selector-score tensor, so every step attends a different random block set:
+    one graph touches about 1 GB of distinct K/V blocks of the 2.1 GB cache, far
+    more than the 126 MB L2, and a step's blocks come from HBM as in serving. The
+    per-step time is the graph's device time / 16 (CUDA events around each
+    replay), so host launch latency is amortised as it is in a decode loop.
+    """
     w = workloads.WORKLOADS[DECODE_WORKLOAD]
-    n_rot = 4
+    n_rot = 16
     inp = workloads.make_decode_inputs(w, seed=0)
     q, Kc, Vc = inp["q"].to(device), inp["Kc"].to(device), inp["Vc"].to(device)
     seqlen = inp["seqlen"].to(device)
     gen = torch.Generator().manual_seed(1)
     s_rot = [torch.randn(w.B, w.Hkv, w.NB, generator=gen).to(device) for _ in range(n_rot)]
-    s = s_rot[0].clone()
     o = torch.empty_like(q)
     ws = binding.workspace(binding.sas_decode_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K), device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     g_stream = torch.cuda.Stream(device)
     g_stream.wait_stream(stream)
+    launches0 = binding.launch_count()
     with torch.cuda.stream(g_stream):
-        binding.sas_decode_fwd(q, Kc, Vc, seqlen, s, w.K, o, ws, w.sm_scale, stream=g_stream)
+        binding.sas_decode_fwd(q, Kc, Vc, seqlen, s_rot[0], w.K, o, ws, w.sm_scale, stream=g_stream)
+        per_call = binding.launch_count() - launches0
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=g_stream):
-            binding.sas_decode_fwd(q, Kc, Vc, seqlen, s, w.K, o, ws, w.sm_scale, stream=g_stream)
+            for i in range(n_rot):
+                binding.sas_decode_fwd(q, Kc, Vc, seqlen, s_rot[i], w.K, o, ws, w.sm_scale, stream=g_stream)
     stream.wait_stream(g_stream)
     torch.cuda.synchronize(device)
-    steps = max(args.steps, 20)
-    for i in range(max(args.warmup, 3)):
-        s.copy_(s_rot[i % n_rot])
-        flush.zero_()
+    for _ in range(max(args.warmup, 3)):
         graph.replay()
     torch.cuda.synchronize(device)
+    reps = max(4, args.steps)
     times = []
-    for i in range(steps):
-        s.copy_(s_rot[i % n_rot])   # a different selection each step
-        flush.zero_()
+    for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         graph.replay()
         b.record(stream)
         times.append((a, b))
     torch.cuda.synchronize(device)
-    ms = [a.elapsed_time(b) for a, b in times]
-    med = statistics.median(ms)
+    med = statistics.median([a.elapsed_time(b) for a, b in times]) / n_rot
     gbs = decode_bytes(w) / (med * 1e-3) / 1e9
     st = binding.sas_device_status(ws)
     del graph
     return {"workload": "decode_b16_l32k: 16 seqs x 1 token, cache 32768, Hq=32 Hkv=8 d=128 K=16",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": decode_bytes(w), "peak": peaks["hbm_gbs"],
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "graph": True, "steps": steps, "device_status": st}
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
+            "launches_per_step": per_call, "device_status": st,
+            "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
 
 
 # ----------------------------------------------------------------------------- reference arm

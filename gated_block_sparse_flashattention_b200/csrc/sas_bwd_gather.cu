@@ -18,6 +18,14 @@
 // reductions into a workspace accumulator; dLogG[t, j] is written once, by the
 // CTA of block j. Tensor-core work equals the attended work (no union waste).
 //
+// Delta from the stored (bf16) O is off by the rounding of O. dQ/dK/dV barely
+// notice, but dLogG[t, m] = sum_h (A_hm - P_h(B_m) Delta_h), with A_hm the
+// block's sum of P dP and P_h(B_m) its probability mass, is a difference of two
+// close terms when one selected block holds most of the mass. So each CTA also
+// adds its per-head block sum of dS into eps[t, h] (over all attended blocks,
+// that is exactly Delta_h - Delta_stored_h, because P sums to one) and stores
+// P_h(B_m); a finishing kernel subtracts sum_h P_h(B_m) eps[t, h] from dLogG.
+//
 // Pre-pass (three small kernels): per-block counts of selecting rows, their
 // offsets, and the position lists.
 #include <algorithm>
@@ -79,6 +87,8 @@ struct Params {
   __nv_bfloat16* dK;
   __nv_bfloat16* dV;
   float* dLogG;
+  float* eps;                // [B*Hkv*T][G] fp32, zeroed: sum over attended blocks of the block dS sums
+  float* pmass;              // [list entry][G] probability mass of the entry's block, per head
   int32_t* status;
   int B, Hq, Hkv, T, NB, G, P;
   float scale_log2;
@@ -135,7 +145,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int sel_n = min(p.cnt[(long long)bg * p.NB + j], p.list_cap[(long long)bg * p.NB + j]);
   const int total = own_n + sel_n;
   const int n_tiles = (total + PP - 1) / PP;
-  const int32_t* lst = p.list + p.off[(long long)bg * p.NB + j];
+  const long long off_j = p.off[(long long)bg * p.NB + j];
+  const int32_t* lst = p.list + off_j;
   int32_t* status = p.status;
 
   if (warp == 5) tmem_alloc(tmem_slot, TMEM_COLS);
@@ -387,7 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // P / dS shared tiles are free once tile i-1's MMAs completed.
         step_ok = warp_wait(&bars->pd_free, (i - 1) & 1, status);
       }
-      float rs = 0.f;
+      float rs = 0.f, pm = 0.f;
       if (step_ok) {
 #pragma unroll 1
         for (int hc = 0; hc < 2; ++hc) {
@@ -414,6 +425,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 pv[e] = (valid && 32 * hc + kk <= lim) ? ex2(fmaf(sv, p.scale_log2, bias2) - lse2) : 0.f;
                 dv[e] = pv[e] * (dp - dlt);
                 rs += dv[e];
+                pm += pv[e];
               }
               pw[k] = pack_bf16(pv[0], pv[1]);
               sw[k] = pack_bf16(dv[0], dv[1]);
@@ -435,6 +447,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive(&bars->qrow_full[qb]);
           mbar_arrive(&bars->p_full);
         }
+      }
+      // Delta correction terms: this block's dS sum into eps[t, hh]; for a selected
+      // block also its probability mass, at the row's list entry.
+      if (step_ok && valid) {
+        atomicAdd(p.eps + ((long long)bg * p.T + t) * G + hh, rs);
+        if (!own) p.pmass[(off_j + i * PP + (r % PP) - own_n) * G + hh] = pm;
       }
       // dLogG[t, j] for positions that selected j: sum over the G heads (rows hh*PP + pp).
       red[qb * 128 + r] = (valid && !own) ? rs : 0.f;
@@ -619,6 +637,33 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
   reinterpret_cast<uint2*>(dq)[i] = o;
 }
 
+// dLogG[t, j] -= sum_h P_h(B_j) eps[t, h] for every (position, selected block)
+// pair: one warp per (b, g, block) list.
+__global__ void __launch_bounds__(256) dlogg_fix_kernel(const int32_t* __restrict__ cnt,
+                                                        const int32_t* __restrict__ off,
+                                                        const int32_t* __restrict__ cap,
+                                                        const int32_t* __restrict__ list,
+                                                        const float* __restrict__ pmass,
+                                                        const float* __restrict__ eps, float* __restrict__ dLogG,
+                                                        long long n_lists, int T, int NB, int G) {
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // (bg, j)
+  const int lane = threadIdx.x & 31;
+  if (w >= n_lists) return;
+  const long long bg = w / NB;
+  const int j = (int)(w % NB);
+  const int n = min(cnt[w], cap[w]);
+  const long long e0 = off[w];
+  for (int k = lane; k < n; k += 32) {
+    const long long e = e0 + k;
+    const int t = list[e];
+    const float* pm = pmass + e * G;
+    const float* ep = eps + (bg * T + t) * G;
+    float corr = 0.f;
+    for (int h = 0; h < G; ++h) corr = fmaf(pm[h], ep[h], corr);
+    dLogG[(bg * T + t) * NB + j] -= corr;
+  }
+}
+
 }  // namespace gbwd
 
 // Bytes of one packed position: Q and dO rows of the G heads, then LSE and Delta padded to 16 bytes.
@@ -634,6 +679,8 @@ size_t bwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K) {
   n += 4 * a256((size_t)nbg * NB * sizeof(int32_t));       // counts, offsets, caps, cursors
   n += a256((size_t)nbg * region * sizeof(int32_t));       // position lists
   n += a256((size_t)B * Hkv * T * packed_chunk_bytes(Hq / Hkv));   // packed rows
+  n += a256((size_t)B * Hq * T * sizeof(float));           // eps [B*Hkv*T][G]
+  n += a256((size_t)nbg * region * (Hq / Hkv) * sizeof(float));    // pmass, one per list entry and head
   return n;
 }
 
@@ -660,11 +707,16 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   o += a256((size_t)nbg * region * sizeof(int32_t));
   uint8_t* packed = scratch + o;
   const int chunk = (int)packed_chunk_bytes(pb.G);
+  o += a256((size_t)rows * chunk);
+  float* eps = reinterpret_cast<float*>(scratch + o);
+  o += a256((size_t)qrows * sizeof(float));
+  float* pmass = reinterpret_cast<float*>(scratch + o);
 
   cudaError_t e;
   if ((e = cudaMemsetAsync(dLogG, 0, (size_t)rows * NB * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dQacc, 0, (size_t)qrows * D * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(eps, 0, (size_t)qrows * sizeof(float), st)) != cudaSuccess) return e;
   count_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pb.logG, pb.tau, pb.tau_idx, cnt, rows, pb.T, NB);
   count_launch();
   offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(cnt, off, cursor, cap, status, NB, region);
@@ -698,6 +750,8 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   prm.dK = reinterpret_cast<__nv_bfloat16*>(dK);
   prm.dV = reinterpret_cast<__nv_bfloat16*>(dV);
   prm.dLogG = dLogG;
+  prm.eps = eps;
+  prm.pmass = pmass;
   prm.status = status;
   prm.B = pb.B;
   prm.Hq = pb.Hq;
@@ -714,6 +768,9 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   sas_bwd_gather_kernel<<<(unsigned)(nbg * NB), THREADS, SMEM_BYTES, st>>>(tk, tv, prm);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  dlogg_fix_kernel<<<(unsigned)((nbg * NB + 7) / 8), 256, 0, st>>>(cnt, off, cap, list, pmass, eps, dLogG, nbg * NB,
+                                                                   pb.T, NB, pb.G);
+  count_launch();
   const long long n4 = qrows * D / 4;
   dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dQacc, reinterpret_cast<__nv_bfloat16*>(dQ), n4,
                                                                   pb.sm_scale);

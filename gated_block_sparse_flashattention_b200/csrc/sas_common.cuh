@@ -154,6 +154,8 @@ __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
 __device__ __forceinline__ void cp_async_commit_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -282,6 +284,18 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+__device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ small math
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -319,9 +333,7 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
 //
 // Keys (order-preserving uint32 images of the values, -0.0 == +0.0) are held in
 // registers, key of index m = lane + 32*i in keys[i] (rows up to 32*KREG values).
-// The H-th largest key is found by an MSB-first radix select with 8-bit digits,
-// counting in a per-warp shared-memory histogram of 256 bins.
-// ---------------------------------------------------------------------------
+// Key 0 (the image of a negative NaN) marks an empty slot.
 constexpr int kSelectReg = 32;   // rows of up to 1024 values are selected from registers
 
 template <int KREG>
@@ -380,6 +392,98 @@ __device__ __forceinline__ int tie_index_keys(const uint32_t (&keys)[KREG], int 
     run += cnt;
   }
   return -1;
+}
+
+// Bitonic sort of one value per lane across the warp, descending by lane.
+__device__ __forceinline__ uint32_t warp_sort_desc(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+      v = keep_max ? max(v, o) : min(v, o);
+    }
+  }
+  return v;
+}
+
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+      v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  }
+  return v;
+}
+
+// Threshold of the H largest keys (ties toward the lower index) for H <= 32,
+// without bisection. The H-th largest of the 32 per-lane maxima is a lower bound
+// of the threshold: H lanes each hold a key at least that large. Keys below it are
+// never taken, so when at most 32 keys reach it, those candidates are sorted
+// across the warp by (key descending, index ascending) and the H-th one is the
+// threshold key *tkey with its index *tidx (the largest index taken at that key).
+// *asc gets, on lane i < H, the i-th smallest selected index (when asc != null).
+// Returns false, with nothing written, when more than 32 keys reach the bound.
+// Requires c > H. `cand` is 32 uint2 of this warp's shared memory.
+template <int KREG>
+__device__ __forceinline__ bool pivot_select_keys(const uint32_t (&keys)[KREG], int c, int H, uint2* cand,
+                                                  uint32_t* tkey, int* tidx, uint32_t* asc = nullptr) {
+  const int lane = threadIdx.x & 31;
+  uint32_t lmax = 0u;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) lmax = max(lmax, keys[i]);   // empty slots hold key 0
+  const uint32_t bound = __shfl_sync(0xffffffffu, warp_sort_desc(lmax), H - 1);
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) n += (lane + 32 * i < c && keys[i] >= bound) ? 1 : 0;
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total > 32) return false;
+  int pos = incl - n;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i)
+    if (lane + 32 * i < c && keys[i] >= bound) cand[pos++] = make_uint2(keys[i], (uint32_t)(lane + 32 * i));
+  __syncwarp();
+  uint64_t v = 0ull;   // below every candidate
+  if (lane < total) {
+    const uint2 e = cand[lane];
+    v = ((uint64_t)e.x << 32) | (uint64_t)(0xffffffffu - e.y);
+  }
+  __syncwarp();
+  v = warp_sort_desc(v);
+  const uint64_t th = __shfl_sync(0xffffffffu, v, H - 1);
+  *tkey = (uint32_t)(th >> 32);
+  *tidx = (int)(0xffffffffu - (uint32_t)th);
+  if (asc) {
+    // Lanes 0..H-1 hold the selection; order it by index (complements sorted
+    // descending), the unselected lanes last.
+    const uint32_t comp = (lane < H) ? (uint32_t)v : 0u;
+    *asc = 0xffffffffu - warp_sort_desc(comp);
+  }
+  return true;
+}
+
+// Threshold key and tie index of the H largest keys (c > H): the pivot path when
+// it applies, else the bisection and the tie scan.
+template <int KREG>
+__device__ __forceinline__ void threshold_keys(const uint32_t (&keys)[KREG], int c, int H, uint2* cand,
+                                               uint32_t* tkey, int* tidx) {
+  if (H <= 32 && pivot_select_keys(keys, c, H, cand, tkey, tidx)) return;
+  int take_eq = 0;
+  *tkey = radix_select_keys(keys, c, H, nullptr, &take_eq);
+  *tidx = tie_index_keys(keys, c, *tkey, take_eq);
 }
 
 // Generic path for rows longer than 32*kSelectReg: keys re-read from memory on every pass.

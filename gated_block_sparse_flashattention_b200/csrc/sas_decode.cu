@@ -5,31 +5,33 @@
 // §5.1 "Inference implementation" (per-KV-group selection, GQA, gathering only
 // the selected KV blocks).
 //
-// Two kernels:
-//   decode_select_kernel  one warp per (b, g): radix select of the Top-(K-1)
-//                         historical blocks on the score row; the attended
-//                         list [c, selected blocks ascending] goes to the workspace.
-//   decode_attn_kernel    persistent, two CTAs per SM. Work items are (b, g,
-//                         attended block); warp 0 streams each item's K and V
-//                         block (64 keys x 128 features, two 16 KiB bulk async
-//                         copies) into a 3-stage ring, 8 compute warps score the
-//                         G heads against it, run a softmax over the block and
-//                         accumulate P V, and write an fp32 partial (row max,
-//                         row sum, unnormalised output). The CTA that finishes the
-//                         last item of a (b, g) (atomic ticket) merges its partials.
+// bf16 storage, one kernel:
+//   decode_fused_mma_kernel  persistent, two one-warp CTAs per SM, each walking
+//                         a contiguous run of work items (b, g, attended block)
+//                         with a 3-stage TMA ring; the warp selects each (b, g)'s
+//                         blocks itself on entering it, computes the G heads'
+//                         scores and P V as m16n8k16 MMAs (fp32 accumulation),
+//                         folds the items of one (b, g) online, and leaves one
+//                         fp32 partial per such segment.
+// fp32 storage, two kernels:
+//   decode_select_kernel  one warp per (b, g): the attended list [c, selected
+//                         blocks ascending] goes to the workspace.
+//   decode_attn_kernel<float> one 128-thread CTA per work item on the CUDA
+//                         cores, one bulk async copy each for K and V.
+// In both, the CTA whose ticket completes a (b, g) merges its partials into o.
 #include <algorithm>
 #include <mutex>
 
 #include "sas_common.cuh"
 #include "sas_kernels.h"
+#include "sas_tmap.h"
 
 namespace sas {
 namespace decode {
 
 constexpr int D = 128;
-constexpr int NS = 3;                    // K/V ring stages
-constexpr int COMPUTE_WARPS = 8;
-constexpr int THREADS = 32 * (1 + COMPUTE_WARPS);
+constexpr int ATT_THREADS = 128;         // attention CTA: 4 warps x 16 keys
+constexpr int HC = 4;                    // heads per register chunk
 
 struct Params {
   const void* q;
@@ -45,7 +47,7 @@ struct Params {
   int32_t* tickets;    // [B*Hkv]
   float* part_ml;      // [B*Hkv][K][G][2]
   float* part_o;       // [B*Hkv][K][G][D]
-  int B, Hq, Hkv, Lmax, NBmax, K, apply_log_gate, G, n_items;
+  int B, Hq, Hkv, Lmax, NBmax, K, apply_log_gate, G;
   float sm_scale;
 };
 
@@ -66,389 +68,914 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
                : "memory");
 }
 
+// Programmatic dependent launch: the dependent grid may start once every CTA of
+// this grid has called launch_dependents; its griddepcontrol.wait returns when
+// this grid has completed and its memory operations are visible.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ---------------------------------------------------------------------------- selection
-__global__ void __launch_bounds__(256) decode_select_kernel(const Params p) {
-  __shared__ uint32_t hist_all[8][256];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int bg = blockIdx.x * 8 + wid;
-  if (bg >= p.B * p.Hkv) return;
+// Emits the selected blocks of one score row (keys in registers) as the ascending
+// list att[1..] (and so[0..] when requested); returns how many.
+template <int KREG>
+__device__ __forceinline__ int decode_select_row(const float* __restrict__ srow, int c, int H, int mode, uint2* cand,
+                                                 int32_t* att, int32_t* so) {
+  const int lane = threadIdx.x & 31;
+  if (mode == 1) {   // every historical block
+    for (int m = lane; m < c; m += 32) {
+      att[1 + m] = m;
+      if (so) so[m] = m;
+    }
+    return c;
+  }
+  uint32_t keys[KREG];
+  load_row_keys(srow, c, keys);
+  uint32_t tk = 0u, asc = 0u;
+  int tidx = -1;
+  if (H <= 32 && pivot_select_keys(keys, c, H, cand, &tk, &tidx, &asc)) {
+    if (lane < H) {
+      att[1 + lane] = (int32_t)asc;
+      if (so) so[lane] = (int32_t)asc;
+    }
+    return H;
+  }
+  int take_eq = 0;
+  tk = radix_select_keys(keys, c, H, nullptr, &take_eq);
+  tidx = tie_index_keys(keys, c, tk, take_eq);
+  int pos = 0;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    if (32 * i >= c) break;
+    const int m = lane + 32 * i;
+    const bool take = m < c && (keys[i] > tk || (keys[i] == tk && m <= tidx));
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int lp = pos + __popc(bal & ((1u << lane) - 1u));
+      att[1 + lp] = m;
+      if (so) so[lp] = m;
+    }
+    pos += __popc(bal);
+  }
+  return pos;
+}
+
+// Selected blocks of one score row (c historical blocks, mode as below) as the
+// ascending list att[1..] (and so[0..] when requested); returns how many. Warp-
+// collective. `scratch` is 256 words of this warp's shared memory (16-byte aligned).
+// mode 0: nothing selected; 1: every historical block; 2: threshold.
+__device__ __forceinline__ int select_row(const float* __restrict__ srow, int c, int H, int mode, uint32_t* scratch,
+                                          int32_t* att, int32_t* so) {
+  const int lane = threadIdx.x & 31;
+  uint2* cand = reinterpret_cast<uint2*>(scratch);
+  if (mode == 0) return 0;
+  if (c <= 128) return decode_select_row<4>(srow, c, H, mode, cand, att, so);
+  if (c <= 256) return decode_select_row<8>(srow, c, H, mode, cand, att, so);
+  if (c <= 512) return decode_select_row<16>(srow, c, H, mode, cand, att, so);
+  if (c <= 32 * kSelectReg) return decode_select_row<kSelectReg>(srow, c, H, mode, cand, att, so);
+  uint32_t tk = 0u;
+  int tidx = -1;
+  if (mode == 2) {
+    int take_eq = 0;
+    tk = radix_select_global(srow, c, H, scratch, &take_eq);
+    tidx = tie_index_global(srow, c, tk, take_eq);
+  }
+  int pos = 0;
+  for (int base = 0; base < c; base += 32) {
+    const int m = base + lane;
+    bool take = false;
+    if (m < c) {
+      const uint32_t key = float_key(srow[m]);
+      take = mode == 1 || (key > tk) || (key == tk && m <= tidx);
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int lp = pos + __popc(bal & ((1u << lane) - 1u));
+      att[1 + lp] = m;
+      if (so) so[lp] = m;
+    }
+    pos += __popc(bal);
+  }
+  return pos;
+}
+
+// log sum_{m < c} exp(s[m]) of one score row (the log-gate option); warp-collective.
+__device__ __forceinline__ float row_lse(const float* __restrict__ srow, int c) {
+  const int lane = threadIdx.x & 31;
+  float mx = -INFINITY;
+  for (int m = lane; m < c; m += 32) mx = fmaxf(mx, srow[m]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+  for (int m = lane; m < c; m += 32) sum += expf(srow[m] - mx);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  return (c > 0) ? mx + logf(sum) : 0.f;
+}
+
+// One warp (one CTA) per (b, g), so the rows spread over the SMs.
+__global__ void __launch_bounds__(32) decode_select_kernel(const Params p) {
+  __shared__ __align__(16) uint32_t scratch[256];
+  const int lane = threadIdx.x;
+  const int bg = blockIdx.x;
+  griddep_launch_dependents();   // the attention kernel may start its prologue
   const int b = bg / p.Hkv;
   const int L = p.seqlen[b];
+  int32_t* att = p.att + (long long)bg * p.K;
+  if (lane == 0) p.tickets[bg] = 0;   // the attention kernel counts finished blocks here
+  if (L < 1 || L > p.Lmax) {   // a sequence length outside the cache: nothing attended
+    if (lane == 0) set_status(p.status, SAS_DEV_ERR_BOUNDS);
+    for (int k = lane; k < p.K; k += 32) att[k] = -1;
+    return;
+  }
   const int c = (L - 1) / kBlock;
   const int H = p.K - 1;
   const float* srow = p.s + (long long)bg * p.NBmax;
-  int32_t* att = p.att + (long long)bg * p.K;
   int32_t* so = p.sel_out ? p.sel_out + (long long)bg * H : nullptr;
-  // mode 0: nothing selected; 1: every historical block; 2: threshold (tk, tidx).
   const int mode = (min(c, H) == 0) ? 0 : (c <= H ? 1 : 2);
   if (lane == 0) att[0] = c;
-  int pos = 0;
-  if (c <= 32 * kSelectReg) {
-    uint32_t keys[kSelectReg];
-    load_row_keys(srow, c, keys);
-    uint32_t tk = 0u;
-    int tidx = -1;
-    if (mode == 2) {
-      int take_eq = 0;
-      tk = radix_select_keys(keys, c, H, hist_all[wid], &take_eq);
-      tidx = tie_index_keys(keys, c, tk, take_eq);
-    }
-#pragma unroll
-    for (int i = 0; i < kSelectReg; ++i) {
-      if (mode == 0 || 32 * i >= c) break;
-      const int m = lane + 32 * i;
-      const bool take = m < c && (mode == 1 || keys[i] > tk || (keys[i] == tk && m <= tidx));
-      const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const int lp = pos + __popc(bal & ((1u << lane) - 1u));
-        att[1 + lp] = m;
-        if (so) so[lp] = m;
-      }
-      pos += __popc(bal);
-    }
-  } else {
-    uint32_t tk = 0u;
-    int tidx = -1;
-    if (mode == 2) {
-      int take_eq = 0;
-      tk = radix_select_global(srow, c, H, hist_all[wid], &take_eq);
-      tidx = tie_index_global(srow, c, tk, take_eq);
-    }
-    for (int base = 0; mode != 0 && base < c; base += 32) {
-      const int m = base + lane;
-      bool take = false;
-      if (m < c) {
-        const uint32_t k = float_key(srow[m]);
-        take = mode == 1 || (k > tk) || (k == tk && m <= tidx);
-      }
-      const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const int lp = pos + __popc(bal & ((1u << lane) - 1u));
-        att[1 + lp] = m;
-        if (so) so[lp] = m;
-      }
-      pos += __popc(bal);
-    }
-  }
+  const int pos = select_row(srow, c, H, mode, scratch, att, so);
   for (int k = 1 + pos + lane; k < p.K; k += 32) att[k] = -1;
   if (so)
     for (int k = pos + lane; k < H; k += 32) so[k] = -1;
   if (p.apply_log_gate) {
-    float mx = -INFINITY;
-    for (int m = lane; m < c; m += 32) mx = fmaxf(mx, srow[m]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-    for (int m = lane; m < c; m += 32) sum += expf(srow[m] - mx);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) p.lse_gate[bg] = (c > 0) ? mx + logf(sum) : 0.f;
+    const float lse = row_lse(srow, c);
+    if (lane == 0) p.lse_gate[bg] = lse;
   }
 }
 
 // ---------------------------------------------------------------------------- attention
+
+// Eight consecutive features of one K or V row as fp32.
+__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&f)[8]) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void load8(const float* src, float (&f)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+__device__ __forceinline__ void load8_global(const __nv_bfloat16* src, float (&f)[8]) {
+  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void load8_global(const float* src, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+
+// Merges the K partials of (b, g) into o: weight_k = exp(max_k - max), o =
+// sum_k weight_k o_k / sum_k weight_k sum_k. Run by the NT threads of the CTA
+// that took the last ticket; `sm` holds 3*K*G + G floats of shared memory. Every
+// load of a phase is independent of the others, so the phase costs about one
+// L2 round trip.
+template <typename T, int NT, int BATCH>
+__device__ __forceinline__ void merge_partials(const Params& p, int bg, float* sm) {
+  const int tid = threadIdx.x;
+  const int G = p.G, K = p.K;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  float2* ml = reinterpret_cast<float2*>(sm);   // [K][G] (max, sum) of every partial
+  float* wt = sm + 2 * K * G;                   // [K][G] weights
+  float* inv = wt + K * G;                      // [G] 1 / denominator
+  auto sync = [] {
+    if constexpr (NT > 32)
+      __syncthreads();
+    else
+      __syncwarp();
+  };
+  const float2* pml = reinterpret_cast<const float2*>(p.part_ml + (long long)bg * K * G * 2);
+  for (int i = tid; i < K * G; i += NT) ml[i] = __ldcg(pml + i);
+  sync();
+  for (int h = tid; h < G; h += NT) {
+    float M = -INFINITY;
+    for (int kk = 0; kk < K; ++kk) M = fmaxf(M, ml[kk * G + h].x);
+    float den = 0.f;
+    for (int kk = 0; kk < K; ++kk) {
+      const float2 v = ml[kk * G + h];
+      const float w = (v.x == -INFINITY) ? 0.f : ex2((v.x - M) * kLog2e);
+      wt[kk * G + h] = w;
+      den = fmaf(w, v.y, den);
+    }
+    inv[h] = 1.f / den;
+  }
+  sync();
+  const float4* pob = reinterpret_cast<const float4*>(p.part_o + (long long)bg * K * G * D);
+  for (int idx = tid; idx < G * (D / 4); idx += NT) {
+    const int h = idx / (D / 4), d4 = idx % (D / 4);
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < K; k0 += BATCH) {
+      float4 u[BATCH];
+#pragma unroll
+      for (int kk = 0; kk < BATCH; ++kk)
+        if (k0 + kk < K) u[kk] = __ldcg(pob + ((k0 + kk) * G + h) * (D / 4) + d4);
+#pragma unroll
+      for (int kk = 0; kk < BATCH; ++kk) {
+        if (k0 + kk < K) {
+          // Empty slots were never written: weight zero, and their bits stay unused.
+          const float w = wt[(k0 + kk) * G + h];
+          if (w != 0.f) {
+            num.x = fmaf(w, u[kk].x, num.x);
+            num.y = fmaf(w, u[kk].y, num.y);
+            num.z = fmaf(w, u[kk].z, num.z);
+            num.w = fmaf(w, u[kk].w, num.w);
+          }
+        }
+      }
+    }
+    const float s = inv[h];
+    const long long oi = ((long long)b * p.Hq + g * G + h) * D + d4 * 4;
+    if constexpr (sizeof(T) == 2) {
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.o) + oi);
+      dst[0] = __floats2bfloat162_rn(num.x * s, num.y * s);
+      dst[1] = __floats2bfloat162_rn(num.z * s, num.w * s);
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(p.o) + oi) = make_float4(num.x * s, num.y * s, num.z * s, num.w * s);
+    }
+  }
+}
+
+// Merges each (b, g) listed in grp[0..n) (K partials apiece) into o with one L2
+// round trip per batch of 16 partials: every thread loads the (max, sum) pairs of
+// its head together with the partial outputs of its 4 features and combines them
+// in registers (an online rescale between batches when K > 16).
+template <int NT>
+__device__ __forceinline__ void merge_groups(const Params& p, const int* grp, int n) {
+  const int G = p.G, K = p.K;
+  const int per = G * (D / 4);
+  for (int idx = threadIdx.x; idx < n * per; idx += NT) {
+    const int bg = grp[idx / per], r = idx % per, h = r / (D / 4), d4 = r % (D / 4);
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const float2* pml = reinterpret_cast<const float2*>(p.part_ml) + (long long)bg * K * G + h;
+    const float4* pob = reinterpret_cast<const float4*>(p.part_o) + ((long long)bg * K * G + h) * (D / 4) + d4;
+    float M = -INFINITY, den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < K; k0 += 16) {
+      float2 ml[16];
+      float4 u[16];
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        if (k0 + kk < K) {
+          ml[kk] = __ldcg(pml + (k0 + kk) * G);
+          u[kk] = __ldcg(pob + (long long)(k0 + kk) * G * (D / 4));
+        } else {
+          ml[kk] = make_float2(-INFINITY, 0.f);
+        }
+      }
+      float Mb = M;
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) Mb = fmaxf(Mb, ml[kk].x);
+      if (Mb == -INFINITY) continue;
+      const float a = (M == -INFINITY) ? 0.f : ex2((M - Mb) * kLog2e);
+      den *= a;
+      num.x *= a, num.y *= a, num.z *= a, num.w *= a;
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        // Empty slots (max -inf) were never written: weight zero, bits unused.
+        if (ml[kk].x != -INFINITY) {
+          const float w = ex2((ml[kk].x - Mb) * kLog2e);
+          den = fmaf(w, ml[kk].y, den);
+          num.x = fmaf(w, u[kk].x, num.x);
+          num.y = fmaf(w, u[kk].y, num.y);
+          num.z = fmaf(w, u[kk].z, num.z);
+          num.w = fmaf(w, u[kk].w, num.w);
+        }
+      }
+      M = Mb;
+    }
+    const float s = 1.f / den;
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.o) +
+                                                            ((long long)b * p.Hq + g * G + h) * D + d4 * 4);
+    dst[0] = __floats2bfloat162_rn(num.x * s, num.y * s);
+    dst[1] = __floats2bfloat162_rn(num.z * s, num.w * s);
+  }
+}
+
+// One CTA per work item (b, g, attended block). Lane layout inside a warp: the
+// low 16 lanes and the high 16 lanes each cover one whole key row (16 chunks of
+// 8 features), so every shared-memory read of a warp is two adjacent rows.
+// Warp w owns keys 16w .. 16w+15.
 template <typename T>
-__global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const Params p) {
+__global__ void __launch_bounds__(ATT_THREADS, 4) decode_attn_kernel(const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  constexpr uint32_t BLK = 64 * D * sizeof(T);          // one K or V block
-  constexpr int CT = 32 * COMPUTE_WARPS;                // compute threads
-  uint8_t* ring = smem;                                 // [NS][K block, V block]
-  float* qf = reinterpret_cast<float*>(smem + NS * 2 * BLK);   // [G][D] of the current (b, g)
-  float* pr = qf + p.G * D;                                    // [G][64] scores, then probabilities
-  float* qsum = pr + p.G * 64;                                 // [4][G][D] partial P V sums
-  float* acc_o = qsum + 4 * p.G * D;                           // [G][D] running output of the segment
-  float* acc_ml = acc_o + p.G * D;                             // [G][2] running max / sum; [G][2] item max / sum
-  float* fac = acc_ml + 4 * p.G;                               // [G][2] rescale factors of one fold
-  uint64_t* full = reinterpret_cast<uint64_t*>(fac + 2 * p.G);
-  uint64_t* empty = full + NS;
-  int* last_flag = reinterpret_cast<int*>(empty + NS);
+  constexpr uint32_t ROW = D * sizeof(T);      // bytes of one key row
+  constexpr uint32_t BLK = kBlock * ROW;       // one K or V block
+  const int G = p.G;
+  const T* kb = reinterpret_cast<const T*>(smem);
+  const T* vb = reinterpret_cast<const T*>(smem + BLK);
+  float* red = reinterpret_cast<float*>(smem);                 // reuses the K block once scores are done
+  float* sp = reinterpret_cast<float*>(smem + 2 * BLK);        // [G][64] scores, then probabilities
+  float* mlb = sp + G * kBlock;                                // [G][2] block max / sum
+  uint64_t* bar = reinterpret_cast<uint64_t*>(mlb + 2 * G + 2);
+  int* flag = reinterpret_cast<int*>(bar + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int per_cta = (p.n_items + gridDim.x - 1) / gridDim.x;
-  const int it0 = blockIdx.x * per_cta;
-  const int it1 = min(p.n_items, it0 + per_cta);
-  const int G = p.G;
-  if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], COMPUTE_WARPS);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int it = it0; it < it1; ++it) {
-        const int n = it - it0, st = n % NS;
-        if (n >= NS && !mbar_wait(&empty[st], ((n / NS) - 1) & 1, p.status)) break;
-        const int bg = it / p.K, k = it % p.K;
-        const int m = p.att[(long long)bg * p.K + k];
-        issued = n + 1;
-        if (m < 0) {
-          mbar_arrive(&full[st]);   // empty item: nothing to copy
-          continue;
-        }
-        const int rows = min(kBlock, p.Lmax - m * kBlock);
-        const long long off = ((long long)bg * p.Lmax + (long long)m * kBlock) * D;
-        mbar_expect_tx(&full[st], 2u * rows * D * sizeof(T));
-        const uint32_t dst = smem_u32(ring + st * 2 * BLK);
-        bulk_copy_g2s(dst, static_cast<const T*>(p.Kc) + off, rows * D * sizeof(T), &full[st]);
-        bulk_copy_g2s(dst + BLK, static_cast<const T*>(p.Vc) + off, rows * D * sizeof(T), &full[st]);
-      }
-      // Copies still in flight finish before the CTA exits.
-      for (int n = max(0, issued - NS); n < issued; ++n) mbar_wait_drain(&full[n % NS], (n / NS) & 1);
-    }
+  const int dc = lane & 15, kp = lane >> 4;
+  const int bg = blockIdx.x / p.K, k = blockIdx.x % p.K;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int L = p.seqlen[b];
+  if (L < 1 || L > p.Lmax) {   // a sequence length outside the cache
+    if (threadIdx.x == 0) set_status(p.status, SAS_DEV_ERR_BOUNDS);
     return;
   }
-  // ------------------------------------------------------------ compute warps
-  // Items of one (b, g) that this CTA processes back to back form a segment; the
-  // segment keeps a running (max, sum, output) in shared memory (online softmax)
-  // and leaves one partial, in the slot of its first item.
-  const int ct = tid - 32;
-  int cur_bg = -1, seg_k0 = 0;
-  for (int it = it0; it < it1; ++it) {
-    const int n = it - it0, st = n % NS;
-    const int bg = it / p.K, k = it % p.K;
-    const int b = bg / p.Hkv, g = bg % p.Hkv;
-    const int L = p.seqlen[b];
-    const int c = (L - 1) / kBlock;
-    const int m = p.att[(long long)bg * p.K + k];
-    if (bg != cur_bg) {   // new segment: q of the group's heads (fp32), accumulator reset
-      named_bar_sync(1, CT);
-      const T* qg = static_cast<const T*>(p.q) + ((long long)b * p.Hq + g * G) * D;
-      for (int i = ct; i < G * D; i += CT) {
-        qf[i] = to_f<T>(qg[i]);
-        acc_o[i] = 0.f;
-      }
-      for (int h = ct; h < G; h += CT) {
-        acc_ml[2 * h] = -INFINITY;
-        acc_ml[2 * h + 1] = 0.f;
-      }
-      named_bar_sync(1, CT);
-      cur_bg = bg;
-      seg_k0 = k;
+  const int c = (L - 1) / kBlock;
+  const long long cache_row0 = (long long)bg * p.Lmax;
+
+  auto issue = [&](int m, int rows) {
+    mbar_expect_tx(bar, 2u * rows * ROW);
+    const long long off = (cache_row0 + (long long)m * kBlock) * D;
+    bulk_copy_g2s(smem_u32(smem), static_cast<const T*>(p.Kc) + off, rows * ROW, bar);
+    bulk_copy_g2s(smem_u32(smem + BLK), static_cast<const T*>(p.Vc) + off, rows * ROW, bar);
+  };
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    if (k == 0) issue(c, L - c * kBlock);   // the current block does not depend on the selection
+  }
+  // Everything below may read what the selection kernel wrote.
+  griddep_wait();
+  const int m = (k == 0) ? c : p.att[(long long)bg * p.K + k];
+  if (tid == 0 && k != 0 && m >= 0) issue(m, kBlock);
+  __syncthreads();
+
+  float* pm = p.part_ml + ((long long)bg * p.K + k) * G * 2;
+  float* po = p.part_o + ((long long)bg * p.K + k) * G * D;
+  if (m >= 0) {
+    const bool ok = __syncthreads_and(mbar_wait(bar, 0, p.status));
+    if (!ok) {
+      if (tid == 0) mbar_wait_drain(bar, 0);
+      return;
     }
-    // All compute warps agree on success before going on (they meet at named barriers).
-    if (!named_bar_and(2, CT, warp_wait(&full[st], (n / NS) & 1, p.status))) break;
-    if (m >= 0) {
-      const T* kb = reinterpret_cast<const T*>(ring + st * 2 * BLK);
-      const T* vb = reinterpret_cast<const T*>(ring + st * 2 * BLK + BLK);
-      const int nk = (m == c) ? (L - m * kBlock) : kBlock;   // keys present in this block
-      const float bias = (p.apply_log_gate && m != c) ? p.s[(long long)bg * p.NBmax + m] - p.lse_gate[bg] : 0.f;
-      // Scores: thread = (key, quarter of the features), four heads at a time; the
-      // four quarters of a key sit in adjacent lanes and are summed by shuffles.
-      // Chunks are read in a key-rotated order to spread the shared-memory banks.
-      {
-        const int quarter = ct & 3, key = ct >> 2;   // 256 threads = 64 keys x 4 quarters
-        const T* kr = kb + key * D + quarter * 32;
-        float kv[32];   // kv[8*j + e] = element e of chunk (j + key) & 3
+    const int nk = (m == c) ? (L - m * kBlock) : kBlock;   // keys present in this block
+    const float bias = (p.apply_log_gate && m != c) ? p.s[(long long)bg * p.NBmax + m] - p.lse_gate[bg] : 0.f;
+    const T* qg = static_cast<const T*>(p.q) + ((long long)b * p.Hq + g * G) * D;
+    // ---- scores, four heads at a time: each lane holds its 8 features of q and
+    // forms 8-feature partial dots for 8 keys; a butterfly over the 16 lanes of a
+    // row sums them and leaves each lane two finished scores.
+    for (int h0 = 0; h0 < G; h0 += HC) {
+      float qv[HC][8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int cc = (j + key) & 3;
-          if constexpr (sizeof(T) == 2) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(kr + cc * 8);
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      for (int hh = 0; hh < HC; ++hh) {
+        if (h0 + hh < G) {
+          load8_global(qg + (h0 + hh) * D + dc * 8, qv[hh]);
+        } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(h2[e]);
-              kv[j * 8 + 2 * e] = f.x;
-              kv[j * 8 + 2 * e + 1] = f.y;
-            }
-          } else {
-            const float4 a0 = *reinterpret_cast<const float4*>(kr + cc * 8);
-            const float4 a1 = *reinterpret_cast<const float4*>(kr + cc * 8 + 4);
-            kv[j * 8 + 0] = a0.x;
-            kv[j * 8 + 1] = a0.y;
-            kv[j * 8 + 2] = a0.z;
-            kv[j * 8 + 3] = a0.w;
-            kv[j * 8 + 4] = a1.x;
-            kv[j * 8 + 5] = a1.y;
-            kv[j * 8 + 6] = a1.z;
-            kv[j * 8 + 7] = a1.w;
-          }
+          for (int e = 0; e < 8; ++e) qv[hh][e] = 0.f;
         }
-        for (int h0 = 0; h0 < G; h0 += 4) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      }
+      float v[HC * 8];   // v[hh * 8 + i]: head h0+hh, key 16*warp + 2*i + kp
 #pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            if (h0 + hh < G) {
-              const float* qh = qf + (h0 + hh) * D + quarter * 32;
+      for (int i = 0; i < 8; ++i) {
+        float kf[8];
+        load8(kb + (warp * 16 + 2 * i + kp) * D + dc * 8, kf);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int cc = (j + key) & 3;
-                const float4 q0 = *reinterpret_cast<const float4*>(qh + cc * 8);
-                const float4 q1 = *reinterpret_cast<const float4*>(qh + cc * 8 + 4);
-                acc[hh] = fmaf(q0.x, kv[j * 8 + 0], acc[hh]);
-                acc[hh] = fmaf(q0.y, kv[j * 8 + 1], acc[hh]);
-                acc[hh] = fmaf(q0.z, kv[j * 8 + 2], acc[hh]);
-                acc[hh] = fmaf(q0.w, kv[j * 8 + 3], acc[hh]);
-                acc[hh] = fmaf(q1.x, kv[j * 8 + 4], acc[hh]);
-                acc[hh] = fmaf(q1.y, kv[j * 8 + 5], acc[hh]);
-                acc[hh] = fmaf(q1.z, kv[j * 8 + 6], acc[hh]);
-                acc[hh] = fmaf(q1.w, kv[j * 8 + 7], acc[hh]);
-              }
-            }
-          }
+        for (int hh = 0; hh < HC; ++hh) {
+          float a = 0.f;
 #pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            float a = acc[hh];
-            a += __shfl_xor_sync(0xffffffffu, a, 1);
-            a += __shfl_xor_sync(0xffffffffu, a, 2);
-            if (quarter == 0 && h0 + hh < G) pr[(h0 + hh) * 64 + key] = (key < nk) ? a * p.sm_scale + bias : -INFINITY;
+          for (int e = 0; e < 8; ++e) a = fmaf(qv[hh][e], kf[e], a);
+          v[hh * 8 + i] = a;
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const bool up = lane & 8;
+        const float send = up ? v[t] : v[t + 16];
+        const float keep = up ? v[t + 16] : v[t];
+        v[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const bool up = lane & 4;
+        const float send = up ? v[t] : v[t + 8];
+        const float keep = up ? v[t + 8] : v[t];
+        v[t] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const bool up = lane & 2;
+        const float send = up ? v[t] : v[t + 4];
+        const float keep = up ? v[t + 4] : v[t];
+        v[t] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const bool up = lane & 1;
+        const float send = up ? v[t] : v[t + 2];
+        const float keep = up ? v[t + 2] : v[t];
+        v[t] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+      }
+      // v[e] is the full score of entry j = 2 * dc + e.
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j = 2 * dc + e, hh = j >> 3, key = warp * 16 + 2 * (j & 7) + kp;
+        if (h0 + hh < G) sp[(h0 + hh) * kBlock + key] = (key < nk) ? v[e] * p.sm_scale + bias : -INFINITY;
+      }
+    }
+    __syncthreads();
+    // ---- softmax over the block's keys, one warp per head: probabilities relative
+    // to the block's own maximum, plus the block's (max, sum).
+    for (int h = warp; h < G; h += ATT_THREADS / 32) {
+      const float a0 = sp[h * kBlock + lane], a1 = sp[h * kBlock + 32 + lane];
+      float mx = fmaxf(a0, a1);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float e0 = (mx == -INFINITY) ? 0.f : ex2((a0 - mx) * kLog2e);
+      const float e1 = (mx == -INFINITY) ? 0.f : ex2((a1 - mx) * kLog2e);
+      sp[h * kBlock + lane] = e0;
+      sp[h * kBlock + 32 + lane] = e1;
+      float sum = e0 + e1;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) {
+        pm[2 * h] = mx;
+        pm[2 * h + 1] = sum;
+      }
+    }
+    __syncthreads();
+    // ---- P V, four heads at a time: each lane accumulates its 8 features over the
+    // warp's keys; the two half-warps are folded by one butterfly step (each half
+    // keeps two heads) and the four warps are summed through shared memory.
+    for (int h0 = 0; h0 < G; h0 += HC) {
+      float acc[HC * 8];
+#pragma unroll
+      for (int i = 0; i < HC * 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int key = warp * 16 + 2 * i + kp;
+        if (key < nk) {   // rows past the end of the cache hold stale bits
+          float vf[8];
+          load8(vb + key * D + dc * 8, vf);
+#pragma unroll
+          for (int hh = 0; hh < HC; ++hh) {
+            const float w = (h0 + hh < G) ? sp[(h0 + hh) * kBlock + key] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[hh * 8 + e] = fmaf(w, vf[e], acc[hh * 8 + e]);
           }
         }
       }
-      named_bar_sync(1, CT);
-      // Softmax over the block's 64 keys: one warp per head; the item's (max, sum)
-      // and the fold factors into the segment accumulator.
-      for (int h = ct >> 5; h < G; h += COMPUTE_WARPS) {
-        const float a0 = pr[h * 64 + lane], a1 = pr[h * 64 + 32 + lane];
-        float mx = fmaxf(a0, a1);
 #pragma unroll
-        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float e0 = (mx == -INFINITY) ? 0.f : expf(a0 - mx);
-        const float e1 = (mx == -INFINITY) ? 0.f : expf(a1 - mx);
-        pr[h * 64 + lane] = e0;
-        pr[h * 64 + 32 + lane] = e1;
-        float sum = e0 + e1;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) {
-          const float m_old = acc_ml[2 * h], l_old = acc_ml[2 * h + 1];
-          const float m_new = fmaxf(m_old, mx);
-          const float f_old = (m_old == -INFINITY) ? 0.f : expf(m_old - m_new);
-          const float f_item = (mx == -INFINITY) ? 0.f : expf(mx - m_new);
-          fac[2 * h] = f_old;
-          fac[2 * h + 1] = f_item;
-          acc_ml[2 * h] = m_new;
-          acc_ml[2 * h + 1] = l_old * f_old + sum * f_item;
-        }
+      for (int t = 0; t < HC * 4; ++t) {
+        const float send = kp ? acc[t] : acc[t + HC * 4];
+        const float keep = kp ? acc[t + HC * 4] : acc[t];
+        acc[t] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
       }
-      named_bar_sync(1, CT);
-      // P V: thread = (feature pair, quarter of the keys), features fastest across
-      // lanes (conflict-free V reads), four heads at a time; quarters summed in smem.
+      // acc[hl * 8 + e]: head h0 + 2 * kp + hl, feature 8 * dc + e, summed over the warp's keys.
+      if (h0 > 0) __syncthreads();   // the previous chunk's sums have been read
+#pragma unroll
+      for (int hl = 0; hl < 2; ++hl) {
+        float4* dst = reinterpret_cast<float4*>(red + ((warp * HC) + 2 * kp + hl) * D + dc * 8);
+        dst[0] = make_float4(acc[hl * 8 + 0], acc[hl * 8 + 1], acc[hl * 8 + 2], acc[hl * 8 + 3]);
+        dst[1] = make_float4(acc[hl * 8 + 4], acc[hl * 8 + 5], acc[hl * 8 + 6], acc[hl * 8 + 7]);
+      }
+      __syncthreads();
+      // HC * D / 4 = 128 float4 outputs, one per thread.
       {
-        const int dp = ct & 63, kq = ct >> 6;
-        const int k_lo = kq * 16, k_hi = min(nk, k_lo + 16);
-        float2* part = reinterpret_cast<float2*>(qsum);   // [4 quarters][G][64 pairs]
-        for (int h0 = 0; h0 < G; h0 += 4) {
-          float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int key = k_lo; key < k_hi; ++key) {
-            float v0, v1;
-            if constexpr (sizeof(T) == 2) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vb + key * D + 2 * dp));
-              v0 = f.x;
-              v1 = f.y;
-            } else {
-              const float2 f = *reinterpret_cast<const float2*>(vb + key * D + 2 * dp);
-              v0 = f.x;
-              v1 = f.y;
-            }
+        const int hh = tid / (D / 4), d4 = tid % (D / 4);
+        if (h0 + hh < G) {
+          float4 s4 = reinterpret_cast<const float4*>(red + hh * D)[d4];
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-              if (h0 + hh < G) {
-                const float w = pr[(h0 + hh) * 64 + key];
-                o0[hh] = fmaf(w, v0, o0[hh]);
-                o1[hh] = fmaf(w, v1, o1[hh]);
-              }
-            }
+          for (int w = 1; w < ATT_THREADS / 32; ++w) {
+            const float4 u = reinterpret_cast<const float4*>(red + (w * HC + hh) * D)[d4];
+            s4.x += u.x, s4.y += u.y, s4.z += u.z, s4.w += u.w;
           }
-#pragma unroll
-          for (int hh = 0; hh < 4; ++hh)
-            if (h0 + hh < G) part[(kq * G + h0 + hh) * 64 + dp] = make_float2(o0[hh], o1[hh]);
-        }
-        named_bar_sync(1, CT);
-        for (int idx = ct; idx < G * 64; idx += CT) {
-          const int h = idx >> 6, d2 = idx & 63;
-          float2 item = part[h * 64 + d2];
-#pragma unroll
-          for (int q = 1; q < 4; ++q) {
-            const float2 u = part[(q * G + h) * 64 + d2];
-            item.x += u.x;
-            item.y += u.y;
-          }
-          float2* ao = reinterpret_cast<float2*>(acc_o + h * D) + d2;
-          const float2 old = *ao;
-          *ao = make_float2(old.x * fac[2 * h] + item.x * fac[2 * h + 1], old.y * fac[2 * h] + item.y * fac[2 * h + 1]);
+          reinterpret_cast<float4*>(po + (h0 + hh) * D)[d4] = s4;
         }
       }
     }
-    // The stage can be refilled once every compute warp is done with it.
+  } else {
+    // An empty slot (fewer historical blocks than the budget): weight zero in the merge.
+    for (int h = tid; h < G; h += ATT_THREADS) {
+      pm[2 * h] = -INFINITY;
+      pm[2 * h + 1] = 0.f;
+    }
+  }
+  // ---- ticket: the CTA that completes the last item of (b, g) merges the K partials.
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const int ticket = atomicAdd(p.tickets + bg, 1);
+    *flag = (ticket == p.K - 1);
+  }
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  merge_partials<T, ATT_THREADS, 4>(p, bg, reinterpret_cast<float*>(smem));   // the K block is free
+}
+
+// ---------------------------------------------------------------------------- attention, bf16 (tensor cores)
+// One warp (one CTA) per work item (b, g, attended block). The block's K and V
+// rows arrive by TMA as two 64-feature boxes each, in the 128-byte swizzle, so
+// that the 8-row fragment reads below hit eight different bank groups. The G <= 16
+// heads of the group form the 16 rows of m16n8k16 MMAs (bf16 in, fp32
+// accumulate): S = q K^T over 8 key tiles and 8 feature steps, a softmax over the
+// block in registers, then O = P V over 4 key steps and 16 feature tiles, with P
+// taken straight from the S accumulators (the accumulator layout of S is the
+// operand layout of P).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..15) of key row `row` in a K or V tile:
+// two boxes of [64 rows][128 bytes] (features 0-63, 64-127), 128-byte swizzle.
+__device__ __forceinline__ uint32_t kv_tile_offset(uint32_t row, uint32_t chunk) {
+  return (chunk >> 3) * 8192u + row * 128u + (((chunk & 7u) ^ (row & 7u)) << 4);
+}
+
+constexpr uint32_t kMmaTileBytes = 2 * 8192;   // one K or V block (64 x 128 bf16)
+constexpr int kDecStages = 3;                  // K/V ring stages per CTA
+constexpr int kDecWarps = 4;                   // each owns 16 of a block's 64 keys
+constexpr uint32_t kStageBytes = 2 * kMmaTileBytes;
+
+// Shared memory of the fused kernel for G heads per group and budget K.
+constexpr int kMaxItemsPerCta = 63;            // bounds the per-CTA item and segment lists
+struct FusedLayout {
+  uint32_t q, zero, att, grp, comb, seg, bar, total;
+};
+__host__ __device__ inline FusedLayout fused_layout(int G, int K) {
+  FusedLayout l;
+  l.q = kDecStages * kStageBytes;        // 4 q slots of G rows x 256 bytes
+  l.zero = l.q + 4u * G * 256u;          // one zero row (q rows G..15 of the MMA)
+  l.att = l.zero + 256u;                 // attended block of each of the CTA's items
+  l.grp = l.att + 256u;                  // per (b, g) of the CTA: sequence length, log-gate LSE
+  l.comb = l.grp + 2u * 256u;            // [warps][16 rows] (max, sum)
+  l.seg = l.comb + kDecWarps * 16 * 2 * 4;                       // segments: (b, g), first and last item
+  l.bar = l.seg + 64u * 4u * 4u + 64u * 4u;   // segments, then the list of (b, g) to merge
+  l.total = l.bar + 128u;                // full/empty barriers, stage blocks, copies in flight
+  return l;
+}
+
+// Persistent sparse decode attention for bf16 storage: two 4-warp CTAs per SM,
+// launched as a programmatic dependent of decode_select_kernel.
+//
+// CTA i owns the work items u = (b * Hkv + g) * K + k in [u0, u1), consecutive
+// (at most 63), and walks them with a 3-stage ring: TMA copies of the next three
+// items' K and V blocks (64 keys x 128 features, 128-byte swizzle) are in flight
+// while one item is computed. Warp 0 also produces the copies, with the group's q
+// rows alongside the first block of each (b, g). Each warp owns 16 of a block's
+// 64 keys. The G <= 16 heads of the group are the 16 rows of m16n8k16 MMAs (bf16
+// in, fp32 accumulate): S = q K^T for its keys, then O += P V with P taken straight
+// from the S accumulators (their layout is the A operand layout). Each warp keeps
+// its own online softmax state over the items of one (b, g) (max, sum and output
+// in registers; the output is rescaled only when the running max grows by more
+// than 2^8). At the end of such a segment the four warps' states are combined by
+// fp32 reductions into one partial. After its last item the CTA takes one ticket
+// per segment, and the ticket that completes K items merges that (b, g) into o.
+__global__ void __launch_bounds__(32 * kDecWarps, 2)
+    decode_fused_mma_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq,
+                            const int U) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int G = p.G, K = p.K;
+  const FusedLayout lay = fused_layout(G, K);
+  uint8_t* qring = smem + lay.q;
+  uint8_t* zrow = smem + lay.zero;
+  int32_t* att_s = reinterpret_cast<int32_t*>(smem + lay.att);
+  int32_t* grp_L = reinterpret_cast<int32_t*>(smem + lay.grp);
+  float* grp_lse = reinterpret_cast<float*>(smem + lay.grp + 256u);
+  float* comb = reinterpret_cast<float*>(smem + lay.comb);
+  int4* segs = reinterpret_cast<int4*>(smem + lay.seg);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar);
+  uint64_t* empty = full + kDecStages;
+  int* stage_m = reinterpret_cast<int*>(empty + kDecStages);
+  int* issued = stage_m + kDecStages;   // last item index copied into each stage (-1: none)
+  int* nseg_s = issued + kDecStages;
+
+  const int n_units = p.B * p.Hkv * K;
+  const int u0 = blockIdx.x * U, u1 = min(n_units, u0 + U);
+  if (u0 >= u1) return;
+  const int bg0 = u0 / K, n_grp = (u1 - 1) / K - bg0 + 1;
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecWarps);
+      issued[s] = -1;
+    }
+    *nseg_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) reinterpret_cast<uint2*>(zrow)[lane] = make_uint2(0u, 0u);
+  for (int j = tid; j < n_grp; j += 32 * kDecWarps) grp_L[j] = p.seqlen[(bg0 + j) / p.Hkv];
+  // Everything below may read what the selection kernel wrote.
+  griddep_wait();
+  for (int i = tid; i < u1 - u0; i += 32 * kDecWarps) att_s[i] = p.att[u0 + i];
+  if (p.apply_log_gate)
+    for (int j = tid; j < n_grp; j += 32 * kDecWarps) grp_lse[j] = p.lse_gate[bg0 + j];
+  __syncthreads();
+
+  // ------------------------------------------------------------ producer (warp 0)
+  int pf = u0, pf_bg = -1;
+  // Fills stage s with the next item: its K/V block (and the group's q rows when
+  // the item is the first of its (b, g) here), or a bare arrival for an empty slot.
+  auto produce = [&](int s) {
+    if (pf >= u1) return;
+    if (lane == 0) {
+      const int bg = pf / K;
+      const bool newbg = bg != pf_bg;
+      const int m = att_s[pf - u0];
+      stage_m[s] = m;
+      const uint32_t bytes = (m >= 0 ? kStageBytes : 0u) + (newbg ? (uint32_t)G * 256u : 0u);
+      if (bytes) {
+        fence_proxy_async_smem();
+        mbar_expect_tx(&full[s], bytes);
+        if (newbg) {
+          const int b = bg / p.Hkv, g = bg % p.Hkv;
+          tma_load_2d(qring + ((bg - bg0) & 3) * G * 256, &tmq, &full[s], 0, b * p.Hq + g * G);
+        }
+        if (m >= 0) {
+          uint8_t* st = smem + s * kStageBytes;
+          tma_load_3d(st, &tmk, &full[s], 0, m * kBlock, bg);
+          tma_load_3d(st + 8192, &tmk, &full[s], 64, m * kBlock, bg);
+          tma_load_3d(st + kMmaTileBytes, &tmv, &full[s], 0, m * kBlock, bg);
+          tma_load_3d(st + kMmaTileBytes + 8192, &tmv, &full[s], 64, m * kBlock, bg);
+        }
+        issued[s] = pf - u0;
+      } else {
+        mbar_arrive(&full[s]);
+      }
+      pf_bg = bg;
+    }
+    ++pf;
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-    named_bar_sync(1, CT);   // pr[] / qsum[] / acc_o[] settled for this item
-    const bool seg_end = (it + 1 == it1) || ((it + 1) / p.K != bg);
-    if (!seg_end) continue;
-    // Segment end: one partial in the slot of its first item, empty marks in the
-    // other slots it covered, then a ticket for all of its items.
-    {
-      float* pm = p.part_ml + ((long long)bg * p.K) * G * 2;
-      float* po = p.part_o + ((long long)bg * p.K + seg_k0) * G * D;
-      for (int i = ct; i < G * D; i += CT) po[i] = acc_o[i];
-      for (int i = ct; i < (k - seg_k0 + 1) * G; i += CT) {
-        const int kk = seg_k0 + i / G, h = i % G;
-        pm[(kk * G + h) * 2] = (kk == seg_k0) ? acc_ml[2 * h] : -INFINITY;
-        pm[(kk * G + h) * 2 + 1] = (kk == seg_k0) ? acc_ml[2 * h + 1] : 0.f;
+  };
+  if (warp == 0)
+    for (int s = 0; s < kDecStages; ++s) produce(s);
+
+  // ------------------------------------------------------------ consumers (all warps)
+  // Per-lane parts of the fragment addresses (128-byte swizzle, row & 7 == lane & 7).
+  const int r8 = lane & 7, mi = lane >> 3;
+  const uint32_t k_row = (uint32_t)(16 * warp + (mi >> 1) * 8 + r8) * 128u;
+  const uint32_t v_row = (uint32_t)(16 * warp + (mi & 1) * 8 + r8) * 128u;
+  uint32_t k_x[4], v_x[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    k_x[j] = (uint32_t)(((2 * j + (mi & 1)) ^ r8) << 4);
+    v_x[j] = (uint32_t)(((2 * j + (mi >> 1)) ^ r8) << 4);
+  }
+  const int qrow = r8 + (mi & 1) * 8;   // head row this lane addresses in the A fragments of q
+
+  float run_m0 = -INFINITY, run_m1 = -INFINITY, run_l0 = 0.f, run_l1 = 0.f;   // log2 domain
+  float oacc[16][4];
+#pragma unroll
+  for (int nd = 0; nd < 16; ++nd) oacc[nd][0] = oacc[nd][1] = oacc[nd][2] = oacc[nd][3] = 0.f;
+  uint32_t qa[8][4];
+  int seg_bg = -1, seg_k0 = 0, seg_k1 = 0, q_bg = -1;
+  bool ok = true;
+
+  // End of a segment: the warps' states are combined into the partial of slot k0
+  // (zeroed when the segment began) and slots k0+1..k1 are marked empty. Its
+  // ticket is taken after the CTA's last item.
+  auto flush = [&](int bg, int k0, int k1) {
+    float l0 = run_l0, l1 = run_l1;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    if (tig == 0) {
+      comb[(warp * 16 + gid) * 2] = run_m0;
+      comb[(warp * 16 + gid) * 2 + 1] = l0;
+      comb[(warp * 16 + gid + 8) * 2] = run_m1;
+      comb[(warp * 16 + gid + 8) * 2 + 1] = l1;
+    }
+    ok = named_bar_and(1, 32 * kDecWarps, ok);
+    if (!ok) return;
+    float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+      M0 = fmaxf(M0, comb[(w * 16 + gid) * 2]);
+      M1 = fmaxf(M1, comb[(w * 16 + gid + 8) * 2]);
+    }
+    const float sc0 = (run_m0 == -INFINITY) ? 0.f : ex2(run_m0 - M0);
+    const float sc1 = (run_m1 == -INFINITY) ? 0.f : ex2(run_m1 - M1);
+    float* po = p.part_o + ((long long)bg * K + k0) * G * D;
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd) {
+      if (gid < G) red_add_v2(po + gid * D + nd * 8 + 2 * tig, oacc[nd][0] * sc0, oacc[nd][1] * sc0);
+      if (gid + 8 < G) red_add_v2(po + (gid + 8) * D + nd * 8 + 2 * tig, oacc[nd][2] * sc1, oacc[nd][3] * sc1);
+    }
+    if (warp == 0) {
+      float* pm = p.part_ml + (long long)bg * K * G * 2;
+      if (tig == 0) {
+        float L0 = 0.f, L1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+          const float m0 = comb[(w * 16 + gid) * 2], m1 = comb[(w * 16 + gid + 8) * 2];
+          if (m0 != -INFINITY) L0 += comb[(w * 16 + gid) * 2 + 1] * ex2(m0 - M0);
+          if (m1 != -INFINITY) L1 += comb[(w * 16 + gid + 8) * 2 + 1] * ex2(m1 - M1);
+        }
+        if (gid < G) {
+          pm[(k0 * G + gid) * 2] = (M0 == -INFINITY) ? -INFINITY : M0 * kLn2;
+          pm[(k0 * G + gid) * 2 + 1] = L0;
+        }
+        if (gid + 8 < G) {
+          pm[(k0 * G + gid + 8) * 2] = (M1 == -INFINITY) ? -INFINITY : M1 * kLn2;
+          pm[(k0 * G + gid + 8) * 2 + 1] = L1;
+        }
+      }
+      for (int i = lane; i < (k1 - k0) * G; i += 32) {
+        const int kk = k0 + 1 + i / G, h = i % G;
+        pm[(kk * G + h) * 2] = -INFINITY;
+        pm[(kk * G + h) * 2 + 1] = 0.f;
+      }
+      if (lane == 0) {
+        segs[*nseg_s] = make_int4(bg, k1 - k0 + 1, 0, 0);
+        *nseg_s += 1;
       }
     }
-    named_bar_sync(1, CT);
-    if (ct == 0) {
-      __threadfence();   // after the barrier: the whole CTA's partials precede the ticket
-      const int cnt = k - seg_k0 + 1;
-      const int ticket = atomicAdd(p.tickets + bg, cnt);
-      *last_flag = (ticket + cnt == p.K);
+    // comb[] is rewritten by the next segment only after every warp has read it.
+    named_bar_sync(2, 32 * kDecWarps);
+  };
+
+  for (int n = 0, u = u0; u < u1; ++n, ++u) {
+    const int s = n % kDecStages;
+    const uint32_t ph = (uint32_t)(n / kDecStages) & 1u;
+    const int bg = u / K, k = u % K;
+    if (bg != seg_bg) {
+      if (seg_bg >= 0) flush(seg_bg, seg_k0, seg_k1);
+      seg_bg = bg;
+      seg_k0 = k;
+      run_m0 = run_m1 = -INFINITY;
+      run_l0 = run_l1 = 0.f;
+#pragma unroll
+      for (int nd = 0; nd < 16; ++nd) oacc[nd][0] = oacc[nd][1] = oacc[nd][2] = oacc[nd][3] = 0.f;
+      if (warp == 0 && ok) {   // the segment's partial accumulates here by reductions
+        float4* po = reinterpret_cast<float4*>(p.part_o + ((long long)bg * K + k) * G * D);
+        for (int i = lane; i < G * (D / 4); i += 32) po[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
-    named_bar_sync(1, CT);
-    if (*last_flag) {
-      // Merge: slot maxima and sums into shared memory, one weight per (slot, head),
-      // then every output element sums the weighted slot outputs (loads unrolled).
+    seg_k1 = k;
+    if (ok) ok = warp_wait(&full[s], ph, p.status);
+    int m = ok ? stage_m[s] : -1;
+    const int L = grp_L[bg - bg0];
+    if (L < 1 || L > p.Lmax) m = -1;   // recorded by the selection kernel
+    bool zeroed = false;
+    if (m >= 0) {
+      const int slot = (bg - bg0) & 3;
+      const int c = (L - 1) / kBlock;
+      const int nk = (m == c) ? (L - m * kBlock) : kBlock;   // keys present in this block
+      const uint32_t st = smem_u32(smem + s * kStageBytes);
+      if (q_bg != bg) {   // the group's q rows as A fragments; rows G..15 read the zero row
+        const uint32_t qa_addr = (qrow < G) ? smem_u32(qring + slot * G * 256 + qrow * 256) + (mi >> 1) * 16u
+                                            : smem_u32(zrow);
+        const uint32_t qstep = (qrow < G) ? 32u : 0u;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) ldsm_x4(qa_addr + ks * qstep, qa[ks]);
+        q_bg = bg;
+      }
+      if (nk < 16 * warp + 16) {
+        // This warp's rows past the end of the sequence may hold any bits; P is zero
+        // there, and zero V rows keep 0 * NaN out of the P V products.
+        uint8_t* vs = smem + s * kStageBytes + kMmaTileBytes;
+        const int row0 = max(nk, 16 * warp);
+        for (int i = lane; i < (16 * warp + 16 - row0) * 16; i += 32) {
+          const int row = row0 + i / 16, chunk = i % 16;
+          *reinterpret_cast<uint4*>(vs + kv_tile_offset(row, chunk)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+        zeroed = true;
+      }
+      // ---- S = q K^T for the warp's 16 keys: sacc[j] = rows gid, gid+8, keys 16w + 8j + 2tig, +1.
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t r[4];
+        ldsm_x4(st + (ks >> 2) * 8192u + k_row + k_x[ks & 3], r);
+        mma16816(sacc[0], qa[ks], r[0], r[1]);
+        mma16816(sacc[1], qa[ks], r[2], r[3]);
+      }
+      // ---- online softmax (log2 domain).
+      const float bias =
+          (p.apply_log_gate && m != c) ? p.s[(long long)bg * p.NBmax + m] - grp_lse[bg - bg0] : 0.f;
+      const float sl2 = p.sm_scale * kLog2e, bl2 = bias * kLog2e;
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[j][e] = fmaf(sacc[j][e], sl2, bl2);
+      if (nk < kBlock) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (16 * warp + 8 * j + 2 * tig + (e & 1) >= nk) sacc[j][e] = -INFINITY;
+      }
+      float mx0 = fmaxf(fmaxf(sacc[0][0], sacc[0][1]), fmaxf(sacc[1][0], sacc[1][1]));
+      float mx1 = fmaxf(fmaxf(sacc[0][2], sacc[0][3]), fmaxf(sacc[1][2], sacc[1][3]));
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (__any_sync(0xffffffffu, mx0 > run_m0 + 8.f || mx1 > run_m1 + 8.f)) {
+        const float nm0 = fmaxf(run_m0, mx0), nm1 = fmaxf(run_m1, mx1);
+        const float a0 = (run_m0 == -INFINITY) ? 0.f : ex2(run_m0 - nm0);
+        const float a1 = (run_m1 == -INFINITY) ? 0.f : ex2(run_m1 - nm1);
+        run_m0 = nm0;
+        run_m1 = nm1;
+        run_l0 *= a0;
+        run_l1 *= a1;
+#pragma unroll
+        for (int nd = 0; nd < 16; ++nd) {
+          oacc[nd][0] *= a0;
+          oacc[nd][1] *= a0;
+          oacc[nd][2] *= a1;
+          oacc[nd][3] *= a1;
+        }
+      }
+      const float sub0 = (run_m0 == -INFINITY) ? 0.f : run_m0, sub1 = (run_m1 == -INFINITY) ? 0.f : run_m1;
+      float pv[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        pv[j][0] = ex2(sacc[j][0] - sub0);
+        pv[j][1] = ex2(sacc[j][1] - sub0);
+        pv[j][2] = ex2(sacc[j][2] - sub1);
+        pv[j][3] = ex2(sacc[j][3] - sub1);
+      }
+      run_l0 += (pv[0][0] + pv[0][1]) + (pv[1][0] + pv[1][1]);
+      run_l1 += (pv[0][2] + pv[0][3]) + (pv[1][2] + pv[1][3]);
+      const uint32_t pa[4] = {pack_bf16(pv[0][0], pv[0][1]), pack_bf16(pv[0][2], pv[0][3]),
+                              pack_bf16(pv[1][0], pv[1][1]), pack_bf16(pv[1][2], pv[1][3])};
+      // ---- O += P V over the warp's 16 keys: oacc[nd] = rows gid, gid+8, features 8nd + 2tig, +1.
+      const uint32_t vst = st + kMmaTileBytes;
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {
+        uint32_t r[4];
+        ldsm_x4_t(vst + (np >> 2) * 8192u + v_row + v_x[np & 3], r);
+        mma16816(oacc[2 * np], pa, r[0], r[1]);
+        mma16816(oacc[2 * np + 1], pa, r[2], r[3]);
+      }
+    }
+    if (zeroed) fence_proxy_async_smem();   // the generic writes come before the stage's next copy
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (warp == 0 && ok && pf < u1) {
+      // The next item goes into stage s once every warp has finished with it.
+      ok = warp_wait(&empty[s], ph, p.status);
+      if (ok) produce(s);
+    }
+  }
+  if (seg_bg >= 0) flush(seg_bg, seg_k0, seg_k1);
+  // ---- tickets: one per segment; the ticket that completes K items merges its (b, g).
+  __threadfence();
+  ok = named_bar_and(1, 32 * kDecWarps, ok);
+  if (ok) {
+    const int nseg = *nseg_s;
+    int* mlist = reinterpret_cast<int*>(segs + 64);   // the (b, g) this CTA merges
+    __syncthreads();
+    if (warp == 0) {
+      int n_last = 0;
+      for (int i0 = 0; i0 < nseg; i0 += 32) {
+        const int i = i0 + lane;
+        const int4 sg = i < nseg ? segs[i] : make_int4(0, 0, 0, 0);
+        const bool last = i < nseg && atomicAdd(p.tickets + sg.x, sg.y) + sg.y == K;
+        const uint32_t bal = __ballot_sync(0xffffffffu, last);
+        if (last) mlist[n_last + __popc(bal & ((1u << lane) - 1u))] = sg.x;
+        n_last += __popc(bal);
+      }
+      if (lane == 0) *nseg_s = n_last;
+    }
+    __syncthreads();
+    const int n_merge = *nseg_s;
+    if (n_merge > 0) {
       __threadfence();
-      float* mw = qsum;                   // [K][G] weights
-      float* den = qsum + p.K * G;        // [G]
-      for (int i = ct; i < p.K * G; i += CT)
-        mw[i] = __ldcg(p.part_ml + ((long long)bg * p.K * G + i) * 2);
-      named_bar_sync(1, CT);
-      for (int h = ct; h < G; h += CT) {
-        float M = -INFINITY;
-        for (int kk = 0; kk < p.K; ++kk) M = fmaxf(M, mw[kk * G + h]);
-        float dsum = 0.f;
-        for (int kk = 0; kk < p.K; ++kk) {
-          const float mk = mw[kk * G + h];
-          const float wgt = (mk == -INFINITY) ? 0.f : expf(mk - M);
-          dsum += wgt * __ldcg(p.part_ml + (((long long)bg * p.K + kk) * G + h) * 2 + 1);
-          mw[kk * G + h] = wgt;
-        }
-        den[h] = dsum;
-      }
-      named_bar_sync(1, CT);
-      for (int idx = ct; idx < G * D; idx += CT) {
-        const int h = idx / D, dd = idx % D;
-        float num = 0.f;
-#pragma unroll 4
-        for (int kk = 0; kk < p.K; ++kk) {
-          const float wgt = mw[kk * G + h];
-          if (wgt != 0.f) num += wgt * __ldcg(p.part_o + (((long long)bg * p.K + kk) * G + h) * D + dd);
-        }
-        const float out = num / den[h];
-        const long long oi = ((long long)b * p.Hq + g * G + h) * D + dd;
-        if constexpr (sizeof(T) == 2)
-          static_cast<__nv_bfloat16*>(p.o)[oi] = __float2bfloat16_rn(out);
-        else
-          static_cast<float*>(p.o)[oi] = out;
-      }
-      if (ct == 0) p.tickets[bg] = 0;   // ready for the next call
-      named_bar_sync(1, CT);
+      merge_groups<32 * kDecWarps>(p, mlist, n_merge);
     }
+  } else if (warp == 0 && lane == 0) {
+    // Wind down: copies still in flight finish before the CTA exits.
+    for (int t = 0; t < kDecStages; ++t)
+      if (issued[t] >= 0) mbar_wait_drain(&full[t], (uint32_t)(issued[t] / kDecStages) & 1u);
   }
 }
 
 size_t smem_bytes(int dtype, int G) {
   const size_t el = dtype == 1 ? 2 : 4;
-  return NS * 2 * 64 * D * el + ((size_t)G * D + G * 64 + 4 * G * D + G * D + 6 * G) * 4 + 2 * NS * 8 + 16 + 128;
+  return 2 * kBlock * D * el + ((size_t)G * kBlock + 2 * G + 2) * 4 + 8 + 16 + 128;
 }
 
 }  // namespace decode
@@ -499,30 +1026,53 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
   prm.K = pb.K;
   prm.apply_log_gate = pb.apply_log_gate;
   prm.G = G;
-  prm.n_items = (int)(n_bg * pb.K);
   prm.sm_scale = pb.sm_scale;
-  // Tickets start at zero on every call.
-  cudaError_t e = cudaMemsetAsync(prm.tickets, 0, n_bg * sizeof(int32_t), st);
-  if (e != cudaSuccess) return e;
-  decode_select_kernel<<<(unsigned)((n_bg + 7) / 8), 256, 0, st>>>(prm);
+  cudaError_t e;
+  // Selection first (it also clears the tickets); the attention kernel follows.
+  decode_select_kernel<<<(unsigned)n_bg, 32, 0, st>>>(prm);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const unsigned grid = (unsigned)std::min<long long>((long long)prm.n_items, 2LL * sms);
-  const size_t shm = smem_bytes(pb.dtype, G);
   if (pb.dtype == 1) {
-    if ((e = cudaFuncSetAttribute(decode_attn_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)shm)) != cudaSuccess)
-      return e;
-    decode_attn_kernel<__nv_bfloat16><<<grid, THREADS, shm, st>>>(prm);
-  } else {
-    if ((e = cudaFuncSetAttribute(decode_attn_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm)) !=
+    CUtensorMap tk, tv, tq;
+    if (!make_tmap_bf16_3d(&tk, pb.Kc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
+        !make_tmap_bf16_3d(&tv, pb.Vc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
+        !make_tmap_bf16_rows(&tq, pb.q, D, (uint64_t)pb.B * pb.Hq, (uint32_t)G))
+      return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const long long n_units = (long long)n_bg * pb.K;
+    const int per_cta = (int)std::min<long long>(kMaxItemsPerCta, (n_units + 2LL * sms - 1) / (2LL * sms));
+    const unsigned grid = (unsigned)((n_units + per_cta - 1) / per_cta);
+    const size_t shm = fused_layout(G, pb.K).total + 1024;
+    if ((e = cudaFuncSetAttribute(decode_fused_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm)) !=
         cudaSuccess)
       return e;
-    decode_attn_kernel<float><<<grid, THREADS, shm, st>>>(prm);
+    // All of the unified L1 / shared memory as shared memory: two CTAs (six ring
+    // stages of K/V blocks in flight) per SM.
+    if ((e = cudaFuncSetAttribute(decode_fused_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * kDecWarps);
+    cfg.dynamicSmemBytes = shm;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_fused_mma_kernel, prm, tk, tv, tq, per_cta);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    return cudaGetLastError();
   }
+  const size_t shm = smem_bytes(pb.dtype, G);
+  if ((e = cudaFuncSetAttribute(decode_attn_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm)) !=
+      cudaSuccess)
+    return e;
+  decode_attn_kernel<float><<<(unsigned)(n_bg * pb.K), ATT_THREADS, shm, st>>>(prm);
   count_launch();
   return cudaGetLastError();
 }
@@ -571,7 +1121,7 @@ cudaError_t launch_decode_static(const DecodeProblem& pb, cudaStream_t st) {
   void* ws = nullptr;
   cudaError_t e = decode_static::scratch_address(&ws);
   if (e != cudaSuccess) return e;
-  // The status word starts clear on every call (tickets are cleared by launch_decode).
+  // The status word starts clear on every call (the select kernel clears the tickets).
   e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   return launch_decode(pb, ws, st);

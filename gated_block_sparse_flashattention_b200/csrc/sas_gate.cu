@@ -43,9 +43,19 @@ __device__ __forceinline__ void select_row_regs(const float* __restrict__ v, int
   const int lane = threadIdx.x & 31;
   uint32_t keys[KREG];
   load_row_keys(v, c, keys);
+  uint32_t tkey = 0u, asc = 0u;
+  int tidx = -1;
+  if (H <= 32 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, &asc)) {
+    if (lane == 0) {
+      *tau_out = key_float(tkey);
+      *tidx_out = tidx;
+    }
+    if (out && lane < H) out[lane] = (int32_t)asc;   // exactly H blocks, ascending
+    return;
+  }
   int take_eq = 0;
-  const uint32_t tkey = radix_select_keys(keys, c, H, hist, &take_eq);
-  const int tidx = tie_index_keys(keys, c, tkey, take_eq);
+  tkey = radix_select_keys(keys, c, H, nullptr, &take_eq);
+  tidx = tie_index_keys(keys, c, tkey, take_eq);
   if (lane == 0) {
     *tau_out = key_float(tkey);
     *tidx_out = tidx;
@@ -69,7 +79,7 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
                                                                int32_t* __restrict__ tau_idx,
                                                                int32_t* __restrict__ sel, long long rows, int T,
                                                                int NB, int H) {
-  __shared__ uint32_t hist_all[8][256];
+  __shared__ __align__(16) uint32_t hist_all[8][256];   // per-warp scratch of the select
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const long long row = (long long)blockIdx.x * 8 + wid;
@@ -97,8 +107,8 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
     return;
   }
   if (c <= 32 * kSelectReg) {
-    // Keys in registers: one read of the row, four radix passes, the tie index
-    // and the index list all work on them (register width picked by row length).
+    // Keys in registers: one read of the row; the threshold, the tie index and
+    // the index list all work on them (register width picked by row length).
     if (c <= 128)
       select_row_regs<4>(v, c, H, hist_all[wid], tau + row, tau_idx + row, out);
     else if (c <= 256)

@@ -13,4 +13,8 @@ namespace sas {
 bool make_tmap_bf16_3d(CUtensorMap* out, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
                        uint32_t box_rows);
 
+// Encodes a 2-D map over a contiguous bf16 matrix [rows][inner] (inner <= 256)
+// with box (inner, box_rows) and no swizzle: a box lands as box_rows dense rows.
+bool make_tmap_bf16_rows(CUtensorMap* out, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows);
+
 }  // namespace sas

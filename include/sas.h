@@ -167,7 +167,8 @@ SAS_API int sas_bwd(const void* Q, const void* K, const void* V, const void* O, 
  * key/value already at position L-1); seqlen [B] int32 DEVICE, 1 <= L <= Lmax;
  * s [B,Hkv,NBmax] fp32 with NBmax >= ceil(Lmax/64); o [B,Hq,d] of `dtype`;
  * sel_out (nullable) [B,Hkv,K-1] int32 receives I in ascending order, -1 padded.
- * d == 128, 1 <= K <= 64. ws: sas_decode_workspace_size bytes.
+ * d == 128, 1 <= K <= 64. ws: sas_decode_workspace_size bytes. A seqlen
+ * outside 1..Lmax is reported as a device-side bounds error (sas_device_status).
  */
 SAS_API int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen, const float* s,
                    int K, int apply_log_gate, void* o, int32_t* sel_out, int B, int Hq, int Hkv, int Lmax, int NBmax,

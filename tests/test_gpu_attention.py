@@ -111,3 +111,69 @@ def test_full_size_qwen3_4b_layer_sampled():
     _, logG32, tau, tidx, sel = oracle_gates(inp["s"].numpy(), w.K)
     rows = np.array([0, 1, 63, 64, 100, 1023, 1024, 4095, 4096, 6000, 8127, 8128, 8191])
     _sampled_check(w, inp, logG32, tau, tidx, sel, [(0, 0), (0, 5)], rows, [0, 1, 64, 126, 127])
+
+
+def _full_size_sampled(w, groups, rows, blocks, seed=0):
+    """Full-size problem on the GPU, checked on sampled (b, g) groups.
+
+    The GPU normalises and selects the gates of every group itself; on the sampled
+    groups its gate tensor is compared with the oracle's and then replaced by the
+    oracle's fp32 gates, so that both sides attend the same blocks there. The
+    oracle evaluates the sampled rows (O, LSE, dQ, dLogG) and KV blocks (dK, dV)
+    in the gathered form, one group at a time."""
+    inp = workloads.make_training_inputs(w, seed)
+    s_cpu = inp["s"]
+    G = w.G
+    logG, tau, tidx, _ = binding.gate_and_select(dev(s_cpu), w.K)
+    ora = {}
+    for (b, g) in groups:
+        lg64 = orc.gate_normalize(s_cpu[b:b + 1, g:g + 1].numpy().astype(np.float64), w.block)
+        got = logG[b, g].cpu().numpy().astype(np.float64)
+        fin = np.isfinite(lg64[0, 0])
+        assert np.array_equal(np.isneginf(got), np.isneginf(lg64[0, 0]))
+        assert np.max(np.abs(got[fin] - lg64[0, 0][fin])) < 2e-5
+        lg32 = lg64.astype(np.float32)
+        logG[b, g] = dev(lg32[0, 0])
+        ta, ti, se = orc.select_threshold(lg32.astype(np.float64), w.K, w.block)
+        ora[(b, g)] = (lg32, ta[0, 0].astype(np.float32), ti[0, 0], se)
+    sel = torch.empty(w.B, w.Hkv, w.T, w.K - 1, dtype=torch.int32, device="cuda")
+    binding.sas_select_threshold(logG, tau, tidx, sel, w.K)
+    for (b, g), (_, ta, ti, se) in ora.items():
+        assert np.array_equal(tau[b, g].cpu().numpy(), ta)
+        assert np.array_equal(tidx[b, g].cpu().numpy(), ti)
+        assert np.array_equal(sel[b, g].cpu().numpy(), se[0, 0])
+    del sel
+    Q, K, V, dO = (dev(inp[k]) for k in ("Q", "K", "V", "dO"))
+    O, LSE = binding.forward(Q, K, V, logG, tau, tidx, w.sm_scale)
+    dQ, dK, dV, dLogG = binding.backward(Q, K, V, O, dO, logG, tau, tidx, LSE, w.K, w.sm_scale)
+    torch.cuda.synchronize()
+    tol = TOL[w.dtype]
+    r = torch.as_tensor(rows, device="cuda")
+    for (b, g), (lg32, _, _, se) in ora.items():
+        hs = slice(g * G, (g + 1) * G)
+        grp = [to_np(inp["Q"][b:b + 1, hs]), to_np(inp["K"][b:b + 1, g:g + 1]), to_np(inp["V"][b:b + 1, g:g + 1]),
+               to_np(inp["dO"][b:b + 1, hs])]
+        ref = orc.rows_gathered(*grp, lg32, se, 0, 0, rows, w.block, w.sm_scale)
+        assert max_abs(to_np(O[b, hs][:, r]), ref["O"]) <= tol["o"]
+        assert max_abs(to_np(LSE[b, hs][:, r]), ref["LSE"]) <= tol["lse"]
+        assert rel_l2(to_np(dQ[b, hs][:, r]), ref["dQ"]) <= tol["rel"]
+        assert rel_l2(to_np(dLogG[b, g][r]), ref["dLogG"]) <= tol["rel"]
+        for j in blocks:
+            rdK, rdV = orc.kv_block_gathered(*grp, lg32, se, 0, 0, j, w.block, w.sm_scale)
+            ks = slice(j * w.block, (j + 1) * w.block)
+            assert rel_l2(to_np(dK[b, g, ks]), rdK) <= tol["rel"], ("dK", j)
+            assert rel_l2(to_np(dV[b, g, ks]), rdV) <= tol["rel"], ("dV", j)
+
+
+def test_full_size_qwen3_8b_layer_sampled():
+    """B=2, Hq=32, Hkv=8, d=128, T=32768, K=32, Student-t selector scores, at full size."""
+    w = workloads.WORKLOADS["qwen3_8b_t32k"]
+    rows = np.array([0, 1, 63, 64, 2047, 2048, 16384, 20001, 32703, 32704, 32767])
+    _full_size_sampled(w, [(0, 0), (1, 7)], rows, [0, 3, 256, 510, 511])
+
+
+def test_full_size_qwen3_14b_layer_sampled():
+    """B=1, Hq=40 (G=5), Hkv=8, d=128, T=65536, K=16, N(0, 1) selector scores, at full size."""
+    w = workloads.WORKLOADS["qwen3_14b_t64k"]
+    rows = np.array([0, 1, 63, 64, 65, 1000, 4095, 4096, 32768, 50001, 65471, 65472, 65535])
+    _full_size_sampled(w, [(0, 3)], rows, [0, 1, 500, 1022, 1023])
