@@ -89,6 +89,7 @@ struct Params {
   float* dLogG;
   float* eps;                // [B*Hkv*T][G] fp32, zeroed: sum over attended blocks of the block dS sums
   float* pmass;              // [list entry][G] probability mass of the entry's block, per head
+  int32_t* dl_idx;           // [list entry] t * NB + j of the entry's dLogG element within its (b, g)
   int32_t* status;
   int B, Hq, Hkv, T, NB, G, P;
   float scale_log2;
@@ -133,11 +134,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Group-major order: the CTAs running at the same time mostly belong to one
-  // (b, g), so the Q/dO rows they gather (that group's heads only) stay in L2.
-  // Within a group, small j (longest row lists) first.
-  const int bg = blockIdx.x / p.NB;
-  const int j = blockIdx.x % p.NB;
+  // Block-major order: block j is attended by its own positions and by the later
+  // positions that select it, so small j carry the longest row lists. Launching
+  // them first (all groups' block 0, then block 1, ...) leaves the short lists to
+  // fill the SMs at the end.
+  const int n_bg = p.B * p.Hkv;
+  const int bg = blockIdx.x % n_bg;
+  const int j = blockIdx.x / n_bg;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int PP = p.P, G = p.G;
   const int rows_used = G * PP;
@@ -452,7 +455,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       // block also its probability mass, at the row's list entry.
       if (step_ok && valid) {
         atomicAdd(p.eps + ((long long)bg * p.T + t) * G + hh, rs);
-        if (!own) p.pmass[(off_j + i * PP + (r % PP) - own_n) * G + hh] = pm;
+        if (!own) {
+          const long long e = off_j + i * PP + (r % PP) - own_n;
+          p.pmass[e * G + hh] = pm;
+          if (hh == 0) p.dl_idx[e] = t * p.NB + j;
+        }
       }
       // dLogG[t, j] for positions that selected j: sum over the G heads (rows hh*PP + pp).
       red[qb * 128 + r] = (valid && !own) ? rs : 0.f;
@@ -498,29 +505,54 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------- pre-pass
+// The pre-pass works on chunks of kChunkRows positions of one (b, g): each CTA
+// counts its chunk's (position, selected block) pairs per block in shared memory
+// and touches the global counters once per (chunk, block), so the global atomics
+// do not pile up on the few thousand block counters.
+constexpr int kChunkRows = 256;
+
+// Calls f(t, m) for every selected historical block m of every position t of the
+// chunk (one warp per position, blocks strided over the lanes).
+template <typename F>
+__device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, const float* __restrict__ tau,
+                                              const int32_t* __restrict__ tau_idx, long long bg, int t0, int T,
+                                              int NB, F&& f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = t0 + warp; t < min(T, t0 + kChunkRows); t += blockDim.x >> 5) {
+    const long long row = bg * T + t;
+    const int c = min(t / kBlock, NB);
+    if (c == 0) continue;
+    const float tv = tau[row];
+    const int ti = tau_idx[row];
+    const float* v = logG + row * (long long)NB;
+    for (int m = lane; m < c; m += 32) {
+      const float x = v[m];
+      if (x > tv || (x == tv && m <= ti)) f(t, m);
+    }
+  }
+}
+
 // Count, per (b, g, block), the positions whose selection contains the block.
+// Grid: (chunks of T, B * Hkv); dynamic shared memory: NB ints.
 __global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
                                                     const int32_t* __restrict__ tau_idx, int32_t* __restrict__ cnt,
-                                                    long long rows, int T, int NB) {
-  const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const long long bg = row / T;
-  const int t = (int)(row % T);
-  const int c = min(t / kBlock, NB);
-  const float tv = tau[row];
-  const int ti = tau_idx[row];
-  const float* v = logG + row * (long long)NB;
-  for (int m = lane; m < c; m += 32) {
-    const float x = v[m];
-    if (x > tv || (x == tv && m <= ti)) atomicAdd(cnt + bg * NB + m, 1);
-  }
+                                                    int T, int NB) {
+  extern __shared__ int32_t hist[];
+  const long long bg = blockIdx.y;
+  const int t0 = blockIdx.x * kChunkRows;
+  for (int m = threadIdx.x; m < NB; m += blockDim.x) hist[m] = 0;
+  __syncthreads();
+  for_each_pair(logG, tau, tau_idx, bg, t0, T, NB, [&](int, int m) { atomicAdd(hist + m, 1); });
+  __syncthreads();
+  for (int m = threadIdx.x; m < NB; m += blockDim.x)
+    if (hist[m]) atomicAdd(cnt + bg * NB + m, hist[m]);
 }
 
 // Offsets: each (b, g) owns a region of T * min(H, NB) entries; off = region + prefix of counts.
 __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ cnt, int32_t* __restrict__ off,
                                                        int32_t* __restrict__ cursor, int32_t* __restrict__ cap,
-                                                       int32_t* status, int NB, long long region) {
+                                                       int32_t* __restrict__ total, int32_t* status, int NB,
+                                                       long long region) {
   __shared__ int32_t warp_sums[32];
   const long long bg = blockIdx.x;
   int base = 0;
@@ -560,29 +592,37 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
     base += warp_sums[31];
     __syncthreads();
   }
+  if (threadIdx.x == 0) total[bg] = (int32_t)(base < region ? base : region);   // entries in use
 }
 
+// Writes the position lists: the chunk's pairs are counted per block in shared
+// memory, each (chunk, block) reserves its range of the block's list with one
+// global atomic, and the positions are placed in that range.
+// Grid: (chunks of T, B * Hkv); dynamic shared memory: 2 * NB ints.
 __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
                                                    const int32_t* __restrict__ tau_idx,
                                                    const int32_t* __restrict__ off, const int32_t* __restrict__ cap,
-                                                   int32_t* __restrict__ cursor, int32_t* __restrict__ list,
-                                                   long long rows, int T, int NB) {
-  const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const long long bg = row / T;
-  const int t = (int)(row % T);
-  const int c = min(t / kBlock, NB);
-  const float tv = tau[row];
-  const int ti = tau_idx[row];
-  const float* v = logG + row * (long long)NB;
-  for (int m = lane; m < c; m += 32) {
-    const float x = v[m];
-    if (x > tv || (x == tv && m <= ti)) {
-      const int slot = atomicAdd(cursor + bg * NB + m, 1);
-      if (slot < cap[bg * NB + m]) list[off[bg * NB + m] + slot] = t;
-    }
+                                                   int32_t* __restrict__ cursor, int32_t* __restrict__ list, int T,
+                                                   int NB) {
+  extern __shared__ int32_t sm[];
+  int32_t* lcnt = sm;        // pairs of the chunk per block, then the running slot
+  int32_t* lbase = sm + NB;  // the chunk's first slot in each block's list
+  const long long bg = blockIdx.y;
+  const int t0 = blockIdx.x * kChunkRows;
+  for (int m = threadIdx.x; m < NB; m += blockDim.x) lcnt[m] = 0;
+  __syncthreads();
+  for_each_pair(logG, tau, tau_idx, bg, t0, T, NB, [&](int, int m) { atomicAdd(lcnt + m, 1); });
+  __syncthreads();
+  for (int m = threadIdx.x; m < NB; m += blockDim.x) {
+    const int n = lcnt[m];
+    lbase[m] = n ? atomicAdd(cursor + bg * NB + m, n) : 0;
+    lcnt[m] = 0;
   }
+  __syncthreads();
+  for_each_pair(logG, tau, tau_idx, bg, t0, T, NB, [&](int t, int m) {
+    const int slot = lbase[m] + atomicAdd(lcnt + m, 1);
+    if (slot < cap[bg * NB + m]) list[off[bg * NB + m] + slot] = t;
+  });
 }
 
 // Packs the rows of each (b, g, position) into one chunk: Q [G][D], dO [G][D]
@@ -638,30 +678,23 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
 }
 
 // dLogG[t, j] -= sum_h P_h(B_j) eps[t, h] for every (position, selected block)
-// pair: one warp per (b, g, block) list.
-__global__ void __launch_bounds__(256) dlogg_fix_kernel(const int32_t* __restrict__ cnt,
-                                                        const int32_t* __restrict__ off,
-                                                        const int32_t* __restrict__ cap,
-                                                        const int32_t* __restrict__ list,
+// pair: one thread per list entry.
+__global__ void __launch_bounds__(256) dlogg_fix_kernel(const int32_t* __restrict__ total,
+                                                        const int32_t* __restrict__ dl_idx,
                                                         const float* __restrict__ pmass,
                                                         const float* __restrict__ eps, float* __restrict__ dLogG,
-                                                        long long n_lists, int T, int NB, int G) {
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // (bg, j)
-  const int lane = threadIdx.x & 31;
-  if (w >= n_lists) return;
-  const long long bg = w / NB;
-  const int j = (int)(w % NB);
-  const int n = min(cnt[w], cap[w]);
-  const long long e0 = off[w];
-  for (int k = lane; k < n; k += 32) {
-    const long long e = e0 + k;
-    const int t = list[e];
-    const float* pm = pmass + e * G;
-    const float* ep = eps + (bg * T + t) * G;
-    float corr = 0.f;
-    for (int h = 0; h < G; ++h) corr = fmaf(pm[h], ep[h], corr);
-    dLogG[(bg * T + t) * NB + j] -= corr;
-  }
+                                                        long long n_entries, long long region, int T, int NB, int G) {
+  const long long e = (long long)blockIdx.x * 256 + threadIdx.x;
+  if (e >= n_entries) return;
+  const long long bg = e / region;
+  if (e - bg * region >= total[bg]) return;
+  const int idx = dl_idx[e];
+  const int t = idx / NB;
+  const float* pm = pmass + e * G;
+  const float* ep = eps + (bg * T + t) * G;
+  float corr = 0.f;
+  for (int h = 0; h < G; ++h) corr = fmaf(pm[h], ep[h], corr);
+  dLogG[bg * T * NB + idx] -= corr;
 }
 
 }  // namespace gbwd
@@ -681,6 +714,8 @@ size_t bwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K) {
   n += a256((size_t)B * Hkv * T * packed_chunk_bytes(Hq / Hkv));   // packed rows
   n += a256((size_t)B * Hq * T * sizeof(float));           // eps [B*Hkv*T][G]
   n += a256((size_t)nbg * region * (Hq / Hkv) * sizeof(float));    // pmass, one per list entry and head
+  n += a256((size_t)nbg * region * sizeof(int32_t));       // dLogG element of each list entry
+  n += a256((size_t)nbg * sizeof(int32_t));                // entries in use per (b, g)
   return n;
 }
 
@@ -711,18 +746,23 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   float* eps = reinterpret_cast<float*>(scratch + o);
   o += a256((size_t)qrows * sizeof(float));
   float* pmass = reinterpret_cast<float*>(scratch + o);
+  o += a256((size_t)nbg * region * pb.G * sizeof(float));
+  int32_t* dl_idx = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * region * sizeof(int32_t));
+  int32_t* total = reinterpret_cast<int32_t*>(scratch + o);
 
   cudaError_t e;
   if ((e = cudaMemsetAsync(dLogG, 0, (size_t)rows * NB * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dQacc, 0, (size_t)qrows * D * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(eps, 0, (size_t)qrows * sizeof(float), st)) != cudaSuccess) return e;
-  count_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pb.logG, pb.tau, pb.tau_idx, cnt, rows, pb.T, NB);
+  const dim3 chunks((unsigned)((pb.T + kChunkRows - 1) / kChunkRows), (unsigned)nbg);
+  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(pb.logG, pb.tau, pb.tau_idx, cnt, pb.T, NB);
   count_launch();
-  offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(cnt, off, cursor, cap, status, NB, region);
+  offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(cnt, off, cursor, cap, total, status, NB, region);
   count_launch();
-  fill_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pb.logG, pb.tau, pb.tau_idx, off, cap, cursor, list, rows,
-                                                          pb.T, NB);
+  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(pb.logG, pb.tau, pb.tau_idx, off, cap, cursor, list,
+                                                              pb.T, NB);
   count_launch();
   pack_kernel<<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(pb.Q), reinterpret_cast<const __nv_bfloat16*>(pb.dO),
@@ -752,6 +792,7 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   prm.dLogG = dLogG;
   prm.eps = eps;
   prm.pmass = pmass;
+  prm.dl_idx = dl_idx;
   prm.status = status;
   prm.B = pb.B;
   prm.Hq = pb.Hq;
@@ -768,8 +809,8 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   sas_bwd_gather_kernel<<<(unsigned)(nbg * NB), THREADS, SMEM_BYTES, st>>>(tk, tv, prm);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dlogg_fix_kernel<<<(unsigned)((nbg * NB + 7) / 8), 256, 0, st>>>(cnt, off, cap, list, pmass, eps, dLogG, nbg * NB,
-                                                                   pb.T, NB, pb.G);
+  dlogg_fix_kernel<<<(unsigned)((nbg * region + 255) / 256), 256, 0, st>>>(total, dl_idx, pmass, eps, dLogG,
+                                                                          nbg * region, region, pb.T, NB, pb.G);
   count_launch();
   const long long n4 = qrows * D / 4;
   dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dQacc, reinterpret_cast<__nv_bfloat16*>(dQ), n4,
