@@ -36,6 +36,27 @@ import torch  # noqa: E402
 
 from gated_block_sparse_flashattention_b200 import workloads  # noqa: E402
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture, cold caches),
+# reported as the roofline "traffic" only while the kernel sources still match the ones measured
+# (sha256 prefixes); after any change they read as unmeasured (null).
+MEASURED_TRAFFIC = {
+    "sas_bwd": (2504363520, {"sas_bwd_gather.cu": "a11aea369e42324c", "sas_common.cuh": "e4093c08909732ee"}),
+    "decode": (72220000, {"sas_decode.cu": "f89db8d077393a35", "sas_common.cuh": "e4093c08909732ee"}),
+}
+
+
+def measured_traffic(name: str):
+    import hashlib
+
+    nbytes, sources = MEASURED_TRAFFIC[name]
+    csrc = os.path.join(ROOT, "gated_block_sparse_flashattention_b200", "csrc")
+    for fname, digest in sources.items():
+        with open(os.path.join(csrc, fname), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
+                return None
+    return nbytes
+
+
 BENCH_WORKLOAD = "qwen3_4b_t8k"
 DECODE_WORKLOAD = "decode_b16_l32k"
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2, written between timed steps
@@ -285,7 +306,8 @@ def run_gpu(args):
         achieved = dom_flops / (dom_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                    "frac": round(achieved / peaks["bf16_tflops"], 4),
+                    "traffic": measured_traffic(dom_name) if dom_name == "sas_bwd" else None,
                     "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
                     "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
                     "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
@@ -415,7 +437,8 @@ def run_decode(args, device, stream, binding, peaks):
     return {"workload": "decode_b16_l32k: 16 seqs x 1 token, cache 32768, Hq=32 Hkv=8 d=128 K=16",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": decode_bytes(w), "peak": peaks["hbm_gbs"],
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": measured_traffic("decode"),
+            "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
             "launches_per_step": per_call, "device_status": st,
             "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
 
