@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Block-major order: block j is attended by its own positions and by the later
   // positions that select it, so small j carry the longest row lists. Launching
   // them first (all groups' block 0, then block 1, ...) leaves the short lists to
-  // fill the SMs at the end.
+  // fill the SMs at the end. (Measured: group-major and pairs-of-groups orders,
+  // which keep fewer groups' rows in L2, were 17% and 11% slower.)
   const int n_bg = p.B * p.Hkv;
   const int bg = blockIdx.x % n_bg;
   const int j = blockIdx.x / n_bg;
