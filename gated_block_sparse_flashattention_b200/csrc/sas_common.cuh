@@ -429,12 +429,15 @@ __device__ __forceinline__ uint64_t warp_sort_desc(uint64_t v) {
 // never taken, so when at most 32 keys reach it, those candidates are sorted
 // across the warp by (key descending, index ascending) and the H-th one is the
 // threshold key *tkey with its index *tidx (the largest index taken at that key).
-// *asc gets, on lane i < H, the i-th smallest selected index (when asc != null).
+// *asc gets, on lane i < H, the i-th smallest selected index (when asc != null);
+// *top gets, on lane i < H, the index of the i-th selected key in (key descending,
+// index ascending) order (when top != null).
 // Returns false, with nothing written, when more than 32 keys reach the bound.
 // Requires c > H. `cand` is 32 uint2 of this warp's shared memory.
 template <int KREG>
 __device__ __forceinline__ bool pivot_select_keys(const uint32_t (&keys)[KREG], int c, int H, uint2* cand,
-                                                  uint32_t* tkey, int* tidx, uint32_t* asc = nullptr) {
+                                                  uint32_t* tkey, int* tidx, uint32_t* asc = nullptr,
+                                                  uint32_t* top = nullptr) {
   const int lane = threadIdx.x & 31;
   uint32_t lmax = 0u;
 #pragma unroll
@@ -466,6 +469,7 @@ __device__ __forceinline__ bool pivot_select_keys(const uint32_t (&keys)[KREG], 
   const uint64_t th = __shfl_sync(0xffffffffu, v, H - 1);
   *tkey = (uint32_t)(th >> 32);
   *tidx = (int)(0xffffffffu - (uint32_t)th);
+  if (top) *top = 0xffffffffu - (uint32_t)v;
   if (asc) {
     // Lanes 0..H-1 hold the selection; order it by index (complements sorted
     // descending), the unselected lanes last.

@@ -5,20 +5,20 @@
 // §5.1 "Inference implementation" (per-KV-group selection, GQA, gathering only
 // the selected KV blocks).
 //
-// bf16 storage, one kernel:
-//   decode_fused_mma_kernel  persistent, two one-warp CTAs per SM, each walking
-//                         a contiguous run of work items (b, g, attended block)
-//                         with a 3-stage TMA ring; the warp selects each (b, g)'s
-//                         blocks itself on entering it, computes the G heads'
-//                         scores and P V as m16n8k16 MMAs (fp32 accumulation),
-//                         folds the items of one (b, g) online, and leaves one
-//                         fp32 partial per such segment.
-// fp32 storage, two kernels:
-//   decode_select_kernel  one warp per (b, g): the attended list [c, selected
-//                         blocks ascending] goes to the workspace.
-//   decode_attn_kernel<float> one 128-thread CTA per work item on the CUDA
-//                         cores, one bulk async copy each for K and V.
-// In both, the CTA whose ticket completes a (b, g) merges its partials into o.
+// bf16 storage, three kernels:
+//   decode_select_kernel    one warp (one CTA) per (b, g): Top-(K-1) of the score
+//                           row; the attended list [c, selected blocks] goes to
+//                           the workspace.
+//   decode_fused_mma_kernel persistent, two 4-warp CTAs per SM, each walking a
+//                           contiguous run of items (b, g, attended block) with a
+//                           3-stage TMA ring; the G heads' scores and P V run as
+//                           m16n8k16 MMAs (fp32 accumulation); the items of one
+//                           (b, g) are folded online and leave one fp32 partial.
+//   decode_merge_kernel     one CTA per (b, g): merges the partials into o.
+// The second and third are programmatic dependents of the one before them.
+// fp32 storage: decode_select_kernel, then decode_attn_kernel<float> (one
+// 128-thread CTA per item on the CUDA cores, one bulk copy each for K and V),
+// whose CTA taking the last ticket of a (b, g) merges its partials.
 #include <algorithm>
 #include <mutex>
 
@@ -44,10 +44,12 @@ struct Params {
   int32_t* status;     // device status word (first word of the workspace)
   int32_t* att;        // [B*Hkv][K] attended blocks: [current, selected ascending], -1 padded
   float* lse_gate;     // [B*Hkv] log-sum-exp of the historical scores (log-gate option)
-  int32_t* tickets;    // [B*Hkv]
-  float* part_ml;      // [B*Hkv][K][G][2]
-  float* part_o;       // [B*Hkv][K][G][D]
+  int32_t* tickets;    // [B*Hkv] (fp32 attention kernel)
+  int32_t* work;       // a counter the select kernel clears (unused by the current kernels)
+  float* part_ml;      // [B*Hkv][n_slots][G][2]
+  float* part_o;       // [B*Hkv][n_slots][G][D]
   int B, Hq, Hkv, Lmax, NBmax, K, apply_log_gate, G;
+  int n_slots;         // partial slots per (b, g)
   float sm_scale;
 };
 
@@ -172,16 +174,26 @@ __device__ __forceinline__ float row_lse(const float* __restrict__ srow, int c) 
   return (c > 0) ? mx + logf(sum) : 0.f;
 }
 
-// One warp (one CTA) per (b, g), so the rows spread over the SMs.
+// One warp (one CTA) per (b, g), so the rows spread over the SMs. KREG (from
+// the score-row length NBmax) lets the row be loaded before the sequence length
+// is known, so the two loads are in flight together; KREG = 0 is the generic
+// path for rows longer than 32 * kSelectReg. The attended list is [c, then the
+// selected blocks]: ascending when sel_out is requested, else in selection order.
+template <int KREG>
 __global__ void __launch_bounds__(32) decode_select_kernel(const Params p) {
   __shared__ __align__(16) uint32_t scratch[256];
   const int lane = threadIdx.x;
   const int bg = blockIdx.x;
   griddep_launch_dependents();   // the attention kernel may start its prologue
+  const float* srow = p.s + (long long)bg * p.NBmax;
+  float sv[KREG > 0 ? KREG : 1];
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) sv[i] = (lane + 32 * i < p.NBmax) ? __ldg(srow + lane + 32 * i) : 0.f;
   const int b = bg / p.Hkv;
   const int L = p.seqlen[b];
   int32_t* att = p.att + (long long)bg * p.K;
-  if (lane == 0) p.tickets[bg] = 0;   // the attention kernel counts finished blocks here
+  if (lane == 0) p.tickets[bg] = 0;   // the fp32 attention kernel counts finished blocks here
+  if (lane == 0 && bg == 0) *p.work = 0;
   if (L < 1 || L > p.Lmax) {   // a sequence length outside the cache: nothing attended
     if (lane == 0) set_status(p.status, SAS_DEV_ERR_BOUNDS);
     for (int k = lane; k < p.K; k += 32) att[k] = -1;
@@ -189,11 +201,28 @@ __global__ void __launch_bounds__(32) decode_select_kernel(const Params p) {
   }
   const int c = (L - 1) / kBlock;
   const int H = p.K - 1;
-  const float* srow = p.s + (long long)bg * p.NBmax;
   int32_t* so = p.sel_out ? p.sel_out + (long long)bg * H : nullptr;
   const int mode = (min(c, H) == 0) ? 0 : (c <= H ? 1 : 2);
   if (lane == 0) att[0] = c;
-  const int pos = select_row(srow, c, H, mode, scratch, att, so);
+  int pos = -1;
+  if constexpr (KREG > 0) {
+    if (mode == 2 && H <= 32) {
+      uint32_t keys[KREG];
+#pragma unroll
+      for (int i = 0; i < KREG; ++i) keys[i] = (lane + 32 * i < c) ? float_key(sv[i]) : 0u;
+      uint32_t tk = 0u, asc = 0u, top = 0u;
+      int tidx = -1;
+      if (pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(scratch), &tk, &tidx, so ? &asc : nullptr,
+                            so ? nullptr : &top)) {
+        if (lane < H) {
+          att[1 + lane] = (int32_t)(so ? asc : top);
+          if (so) so[lane] = (int32_t)asc;
+        }
+        pos = H;
+      }
+    }
+  }
+  if (pos < 0) pos = select_row(srow, c, H, mode, scratch, att, so);
   for (int k = 1 + pos + lane; k < p.K; k += 32) att[k] = -1;
   if (so)
     for (int k = pos + lane; k < H; k += 32) so[k] = -1;
@@ -305,15 +334,15 @@ __device__ __forceinline__ void merge_partials(const Params& p, int bg, float* s
   }
 }
 
-// Merges each (b, g) listed in grp[0..n) (K partials apiece) into o with one L2
+// Merges each (b, g) listed in grp[0..n) (n_slots partials apiece) into o with one L2
 // round trip per batch of 16 partials: every thread loads the (max, sum) pairs of
 // its head together with the partial outputs of its 4 features and combines them
-// in registers (an online rescale between batches when K > 16).
+// in registers (an online rescale between batches when there are more than 16).
 template <int NT>
 __device__ __forceinline__ void merge_groups(const Params& p, const int* grp, int n) {
-  const int G = p.G, K = p.K;
+  const int G = p.G, K = p.n_slots;
   const int per = G * (D / 4);
-  for (int idx = threadIdx.x; idx < n * per; idx += NT) {
+  for (int idx = threadIdx.x; idx < n * per; idx += (NT > 0 ? NT : (int)blockDim.x)) {
     const int bg = grp[idx / per], r = idx % per, h = r / (D / 4), d4 = r % (D / 4);
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const float2* pml = reinterpret_cast<const float2*>(p.part_ml) + (long long)bg * K * G + h;
@@ -359,6 +388,15 @@ __device__ __forceinline__ void merge_groups(const Params& p, const int* grp, in
     dst[0] = __floats2bfloat162_rn(num.x * s, num.y * s);
     dst[1] = __floats2bfloat162_rn(num.z * s, num.w * s);
   }
+}
+
+// Merges each (b, g)'s partials (n_slots apiece) into o: one 128-thread CTA per
+// (b, g) (a float4 of o per thread and pass), launched as a programmatic dependent
+// of the bf16 attention kernel.
+__global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
+  griddep_wait();   // the attention kernel's partials are complete and visible
+  const int grp = blockIdx.x;
+  merge_groups<0>(p, &grp, 1);
 }
 
 // One CTA per work item (b, g, attended block). Lane layout inside a warp: the
@@ -612,9 +650,9 @@ constexpr int kDecWarps = 4;                   // each owns 16 of a block's 64 k
 constexpr uint32_t kStageBytes = 2 * kMmaTileBytes;
 
 // Shared memory of the fused kernel for G heads per group and budget K.
-constexpr int kMaxItemsPerCta = 63;            // bounds the per-CTA item and segment lists
+constexpr int kMaxItemsPerCta = 63;            // bounds the per-CTA item and group lists
 struct FusedLayout {
-  uint32_t q, zero, att, grp, comb, seg, bar, total;
+  uint32_t q, zero, att, grp, comb, bar, total;
 };
 __host__ __device__ inline FusedLayout fused_layout(int G, int K) {
   FusedLayout l;
@@ -623,8 +661,7 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int K) {
   l.att = l.zero + 256u;                 // attended block of each of the CTA's items
   l.grp = l.att + 256u;                  // per (b, g) of the CTA: sequence length, log-gate LSE
   l.comb = l.grp + 2u * 256u;            // [warps][16 rows] (max, sum)
-  l.seg = l.comb + kDecWarps * 16 * 2 * 4;                       // segments: (b, g), first and last item
-  l.bar = l.seg + 64u * 4u * 4u + 64u * 4u;   // segments, then the list of (b, g) to merge
+  l.bar = l.comb + kDecWarps * 16 * 2 * 4;
   l.total = l.bar + 128u;                // full/empty barriers, stage blocks, copies in flight
   return l;
 }
@@ -643,8 +680,8 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int K) {
 // its own online softmax state over the items of one (b, g) (max, sum and output
 // in registers; the output is rescaled only when the running max grows by more
 // than 2^8). At the end of such a segment the four warps' states are combined by
-// fp32 reductions into one partial. After its last item the CTA takes one ticket
-// per segment, and the ticket that completes K items merges that (b, g) into o.
+// fp32 reductions into one partial. decode_merge_kernel, launched as a programmatic
+// dependent, merges every (b, g) once all partials are written.
 __global__ void __launch_bounds__(32 * kDecWarps, 2)
     decode_fused_mma_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq,
@@ -660,12 +697,10 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
   int32_t* grp_L = reinterpret_cast<int32_t*>(smem + lay.grp);
   float* grp_lse = reinterpret_cast<float*>(smem + lay.grp + 256u);
   float* comb = reinterpret_cast<float*>(smem + lay.comb);
-  int4* segs = reinterpret_cast<int4*>(smem + lay.seg);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar);
   uint64_t* empty = full + kDecStages;
   int* stage_m = reinterpret_cast<int*>(empty + kDecStages);
   int* issued = stage_m + kDecStages;   // last item index copied into each stage (-1: none)
-  int* nseg_s = issued + kDecStages;
 
   const int n_units = p.B * p.Hkv * K;
   const int u0 = blockIdx.x * U, u1 = min(n_units, u0 + U);
@@ -677,11 +712,11 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
       mbar_init(&empty[s], kDecWarps);
       issued[s] = -1;
     }
-    *nseg_s = 0;
     fence_barrier_init();
   }
   if (warp == 0) reinterpret_cast<uint2*>(zrow)[lane] = make_uint2(0u, 0u);
   for (int j = tid; j < n_grp; j += 32 * kDecWarps) grp_L[j] = p.seqlen[(bg0 + j) / p.Hkv];
+  griddep_launch_dependents();   // the merge kernel may be scheduled as CTAs finish
   // Everything below may read what the selection kernel wrote.
   griddep_wait();
   for (int i = tid; i < u1 - u0; i += 32 * kDecWarps) att_s[i] = p.att[u0 + i];
@@ -749,8 +784,7 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
   bool ok = true;
 
   // End of a segment: the warps' states are combined into the partial of slot k0
-  // (zeroed when the segment began) and slots k0+1..k1 are marked empty. Its
-  // ticket is taken after the CTA's last item.
+  // (zeroed when the segment began) and slots k0+1..k1 are marked empty.
   auto flush = [&](int bg, int k0, int k1) {
     float l0 = run_l0, l1 = run_l1;
 #pragma unroll
@@ -803,10 +837,6 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
         const int kk = k0 + 1 + i / G, h = i % G;
         pm[(kk * G + h) * 2] = -INFINITY;
         pm[(kk * G + h) * 2 + 1] = 0.f;
-      }
-      if (lane == 0) {
-        segs[*nseg_s] = make_int4(bg, k1 - k0 + 1, 0, 0);
-        *nseg_s += 1;
       }
     }
     // comb[] is rewritten by the next segment only after every warp has read it.
@@ -941,32 +971,7 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
     }
   }
   if (seg_bg >= 0) flush(seg_bg, seg_k0, seg_k1);
-  // ---- tickets: one per segment; the ticket that completes K items merges its (b, g).
-  __threadfence();
-  ok = named_bar_and(1, 32 * kDecWarps, ok);
-  if (ok) {
-    const int nseg = *nseg_s;
-    int* mlist = reinterpret_cast<int*>(segs + 64);   // the (b, g) this CTA merges
-    __syncthreads();
-    if (warp == 0) {
-      int n_last = 0;
-      for (int i0 = 0; i0 < nseg; i0 += 32) {
-        const int i = i0 + lane;
-        const int4 sg = i < nseg ? segs[i] : make_int4(0, 0, 0, 0);
-        const bool last = i < nseg && atomicAdd(p.tickets + sg.x, sg.y) + sg.y == K;
-        const uint32_t bal = __ballot_sync(0xffffffffu, last);
-        if (last) mlist[n_last + __popc(bal & ((1u << lane) - 1u))] = sg.x;
-        n_last += __popc(bal);
-      }
-      if (lane == 0) *nseg_s = n_last;
-    }
-    __syncthreads();
-    const int n_merge = *nseg_s;
-    if (n_merge > 0) {
-      __threadfence();
-      merge_groups<32 * kDecWarps>(p, mlist, n_merge);
-    }
-  } else if (warp == 0 && lane == 0) {
+  if (!ok && warp == 0 && lane == 0) {
     // Wind down: copies still in flight finish before the CTA exits.
     for (int t = 0; t < kDecStages; ++t)
       if (issued[t] >= 0) mbar_wait_drain(&full[t], (uint32_t)(issued[t] / kDecStages) & 1u);
@@ -988,7 +993,7 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int K) {
   size_t bytes = 256;                                      // status word
   bytes += a256(n_bg * K * sizeof(int32_t));               // attended lists
   bytes += a256(n_bg * sizeof(float));                     // log-gate LSE
-  bytes += a256(n_bg * sizeof(int32_t));                   // tickets
+  bytes += a256((n_bg + 1) * sizeof(int32_t));             // tickets, counter
   bytes += a256(n_bg * K * G * 2 * sizeof(float));         // partial max / sum
   bytes += n_bg * K * G * decode::D * sizeof(float);       // partial outputs
   return bytes;
@@ -1014,7 +1019,8 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
   prm.lse_gate = reinterpret_cast<float*>(w + off);
   off += a256(n_bg * sizeof(float));
   prm.tickets = reinterpret_cast<int32_t*>(w + off);
-  off += a256(n_bg * sizeof(int32_t));
+  prm.work = prm.tickets + n_bg;
+  off += a256((n_bg + 1) * sizeof(int32_t));
   prm.part_ml = reinterpret_cast<float*>(w + off);
   off += a256(n_bg * pb.K * G * 2 * sizeof(float));
   prm.part_o = reinterpret_cast<float*>(w + off);
@@ -1026,12 +1032,33 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
   prm.K = pb.K;
   prm.apply_log_gate = pb.apply_log_gate;
   prm.G = G;
+  prm.n_slots = pb.K;
   prm.sm_scale = pb.sm_scale;
   cudaError_t e;
-  // Selection first (it also clears the tickets); the attention kernel follows.
-  decode_select_kernel<<<(unsigned)n_bg, 32, 0, st>>>(prm);
-  count_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // Selection first (it also clears the counters); the attention kernel follows.
+  // Both prefer all of L1 as shared memory, so that attention CTAs can start on
+  // an SM while a selection CTA still runs there (a carveout change would have to
+  // wait for the SM to drain).
+  auto select = [&](auto kernel) -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (r != cudaSuccess) return r;
+    kernel<<<(unsigned)n_bg, 32, 0, st>>>(prm);
+    count_launch();
+    return cudaGetLastError();
+  };
+  // Registers per lane for the score row: the row is loaded before its length is known.
+  if (pb.NBmax <= 128)
+    e = select(decode_select_kernel<4>);
+  else if (pb.NBmax <= 256)
+    e = select(decode_select_kernel<8>);
+  else if (pb.NBmax <= 512)
+    e = select(decode_select_kernel<16>);
+  else if (pb.NBmax <= 32 * kSelectReg)
+    e = select(decode_select_kernel<kSelectReg>);
+  else
+    e = select(decode_select_kernel<0>);
+  if (e != cudaSuccess) return e;
   if (pb.dtype == 1) {
     CUtensorMap tk, tv, tq;
     if (!make_tmap_bf16_3d(&tk, pb.Kc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
@@ -1064,6 +1091,13 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, decode_fused_mma_kernel, prm, tk, tv, tq, per_cta);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    // The merge of every (b, g), as a programmatic dependent of the attention kernel.
+    cfg.gridDim = dim3((unsigned)n_bg);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, decode_merge_kernel, prm);
     if (e != cudaSuccess) return e;
     count_launch();
     return cudaGetLastError();
