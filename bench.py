@@ -120,7 +120,8 @@ def barrier(device=None):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    """nvidia-smi clocks / throttle reasons, sampled every 50 ms; only the samples taken while
+    `active` is set (the GPU running timed or warm-up work) are kept."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -131,12 +132,13 @@ class ClockSampler:
         self.proc = None
         self.lines: list[str] = []
         self._thr = None
+        self.active = False
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._thr = threading.Thread(target=self._read, daemon=True)
             self._thr.start()
         except (FileNotFoundError, OSError):
@@ -145,7 +147,8 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            if self.active:
+                self.lines.append(line.strip())
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -271,7 +274,10 @@ def run_gpu(args):
             ev[3].record(stream)
 
     legs = set(args.legs.split(","))
+    clk = ClockSampler(local).__enter__()   # running through every leg; samples kept while active
+    time.sleep(0.3)
     if "step" in legs:
+        clk.active = True
         for _ in range(args.warmup):
             flush.zero_()
             step()
@@ -283,11 +289,11 @@ def run_gpu(args):
         barrier(device)
         torch.cuda.synchronize(device)
         launches0 = binding.launch_count()
-        with ClockSampler(local) as clk:
-            for i in range(args.steps):
-                flush.zero_()      # L2 flush between timed steps (outside the events)
-                step(evs[i])
-            torch.cuda.synchronize(device)
+        for i in range(args.steps):
+            flush.zero_()      # L2 flush between timed steps (outside the events)
+            step(evs[i])
+        torch.cuda.synchronize(device)
+        clk.active = False
         launches = binding.launch_count() - launches0
         barrier(device)
         step_ms = [e[0].elapsed_time(e[3]) for e in evs]
@@ -313,11 +319,14 @@ def run_gpu(args):
                     "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
                     "gate_select_ms": round(statistics.mean(gate_ms), 4)}
     else:
-        value, ms_per_step, launches, roofline, clk = None, None, 0, None, ClockSampler(local)
+        value, ms_per_step, launches, roofline = None, None, 0, None
 
     # End to end through the C ABI from pinned host buffers, results copied back.
+    clk.active = True   # the e2e leg keeps the GPU busy too
     e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
-    dec = run_decode(args, device, stream, binding, peaks) if "decode" in legs else None
+    clk.active = False
+    dec = run_decode(args, device, stream, binding, peaks, clk) if "decode" in legs else None
+    clk.__exit__(None, None, None)
 
     result = {
         "metric": "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd step)",
@@ -387,7 +396,7 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(total / args.steps, 4)}
 
 
-def run_decode(args, device, stream, binding, peaks):
+def run_decode(args, device, stream, binding, peaks, clk=None):
     """Decode step (16 sequences x 1 token over a 32768-token cache), 16 steps per CUDA graph.
 
     The graph holds 16 decode steps back to back, each with its own seeded
@@ -418,11 +427,15 @@ def run_decode(args, device, stream, binding, peaks):
                 binding.sas_decode_fwd(q, Kc, Vc, seqlen, s_rot[i], w.K, o, ws, w.sm_scale, stream=g_stream)
     stream.wait_stream(g_stream)
     torch.cuda.synchronize(device)
+    if clk is not None:
+        clk.active = True
     for _ in range(max(args.warmup, 3)):
         graph.replay()
     torch.cuda.synchronize(device)
     reps = max(4, args.steps)
     times = []
+    if clk is not None:
+        clk.active = True
     for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -430,6 +443,8 @@ def run_decode(args, device, stream, binding, peaks):
         b.record(stream)
         times.append((a, b))
     torch.cuda.synchronize(device)
+    if clk is not None:
+        clk.active = False
     med = statistics.median([a.elapsed_time(b) for a, b in times]) / n_rot
     gbs = decode_bytes(w) / (med * 1e-3) / 1e9
     st = binding.sas_device_status(ws)
