@@ -120,8 +120,9 @@ def barrier(device=None):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons, sampled every 50 ms; only the samples taken while
-    `active` is set (the GPU running timed or warm-up work) are kept."""
+    """nvidia-smi clocks / throttle reasons, sampled every 50 ms while `active` is set (from the first
+    warm-up step to the end of the decode leg). The summary keeps the samples drawn under load (power
+    draw at least half of the largest seen): the timed regions themselves are tens of milliseconds."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -163,16 +164,22 @@ class ClockSampler:
     def summary(self):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in self.lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
             except ValueError:
                 continue
-            for name, val in zip(names, f[5:9]):
+        pmax = max((r[2] for r in rows), default=0.0)
+        for clock, cmax, power, flags in rows:
+            if power < 0.5 * pmax:
+                continue
+            sm.append(clock)
+            smax = cmax
+            for name, val in zip(names, flags):
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
@@ -293,7 +300,6 @@ def run_gpu(args):
             flush.zero_()      # L2 flush between timed steps (outside the events)
             step(evs[i])
         torch.cuda.synchronize(device)
-        clk.active = False
         launches = binding.launch_count() - launches0
         barrier(device)
         step_ms = [e[0].elapsed_time(e[3]) for e in evs]
@@ -322,10 +328,10 @@ def run_gpu(args):
         value, ms_per_step, launches, roofline = None, None, 0, None
 
     # End to end through the C ABI from pinned host buffers, results copied back.
-    clk.active = True   # the e2e leg keeps the GPU busy too
+    clk.active = True
     e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
-    clk.active = False
     dec = run_decode(args, device, stream, binding, peaks, clk) if "decode" in legs else None
+    clk.active = False
     clk.__exit__(None, None, None)
 
     result = {
@@ -443,8 +449,6 @@ def run_decode(args, device, stream, binding, peaks, clk=None):
         b.record(stream)
         times.append((a, b))
     torch.cuda.synchronize(device)
-    if clk is not None:
-        clk.active = False
     med = statistics.median([a.elapsed_time(b) for a, b in times]) / n_rot
     gbs = decode_bytes(w) / (med * 1e-3) / 1e9
     st = binding.sas_device_status(ws)

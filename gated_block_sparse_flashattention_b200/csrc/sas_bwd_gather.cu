@@ -513,22 +513,35 @@ __global__ void __launch_bounds__(THREADS, 1)
 constexpr int kChunkRows = 256;
 
 // Calls f(t, m) for every selected historical block m of every position t of the
-// chunk (one warp per position, blocks strided over the lanes).
+// chunk. One warp per group of 4 positions (blocks strided over the lanes): the
+// loads of the 4 rows are issued together, so a warp pays one round trip per
+// group instead of one per row.
 template <typename F>
 __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, const float* __restrict__ tau,
                                               const int32_t* __restrict__ tau_idx, long long bg, int t0, int T,
                                               int NB, F&& f) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int t = t0 + warp; t < min(T, t0 + kChunkRows); t += blockDim.x >> 5) {
-    const long long row = bg * T + t;
-    const int c = min(t / kBlock, NB);
-    if (c == 0) continue;
-    const float tv = tau[row];
-    const int ti = tau_idx[row];
-    const float* v = logG + row * (long long)NB;
-    for (int m = lane; m < c; m += 32) {
-      const float x = v[m];
-      if (x > tv || (x == tv && m <= ti)) f(t, m);
+  constexpr int R = 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+  const int t_end = min(T, t0 + kChunkRows);
+  for (int tb = t0 + warp * R; tb < t_end; tb += n_warps * R) {
+    float tv[R];
+    int ti[R], c[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int t = tb + r;
+      c[r] = (t < t_end) ? min(t / kBlock, NB) : 0;
+      tv[r] = c[r] ? tau[bg * T + t] : 0.f;
+      ti[r] = c[r] ? tau_idx[bg * T + t] : 0;
+    }
+    const int cmax = max(max(c[0], c[1]), max(c[2], c[3]));
+    for (int m0 = 0; m0 < cmax; m0 += 32) {
+      const int m = m0 + lane;
+      float x[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) x[r] = (m < c[r]) ? logG[(bg * T + tb + r) * (long long)NB + m] : 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if (m < c[r] && (x[r] > tv[r] || (x[r] == tv[r] && m <= ti[r]))) f(tb + r, m);
     }
   }
 }
