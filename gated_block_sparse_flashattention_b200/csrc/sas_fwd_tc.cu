@@ -15,6 +15,10 @@
 //   warp 5     MMA issuer (one thread): S = Q K^T (M=128, N=64, K=128) into a
 //              double-buffered TMEM S, O += P V (A = P from TMEM, N=128) into
 //              the TMEM O accumulator. Also owns the TMEM allocation.
+// Two CTAs share an SM (256 TMEM columns and about 107 KB of shared memory
+// each), so one tile's softmax runs while the other's waits on its MMAs. P is
+// written over the first half of its S buffer; S of block j+2 reuses that buffer
+// only after the P V of block j has completed.
 #include "sas_common.cuh"
 #include "sas_kernels.h"
 #include "sas_tmap.h"
@@ -23,7 +27,7 @@ namespace sas {
 namespace fwd {
 
 constexpr int D = 128;
-constexpr int NST = 3;                      // K/V ring stages
+constexpr int NST = 2;                      // K/V ring stages
 constexpr int THREADS = 192;
 constexpr uint32_t Q_BYTES = 128 * D * 2;   // 32 KiB: 2 halves of [128 rows][128 B]
 constexpr uint32_t KV_HALF = 64 * 128;      // one 64-row x 128-byte half tile (8 KiB)
@@ -39,8 +43,8 @@ constexpr uint32_t SMEM_BYTES = OFF_WORDS + (MAX_NB / 32) * 4 + 1024;   // +1024
 // TMEM columns.
 constexpr uint32_t COL_O = 0;
 constexpr uint32_t COL_S0 = 128;    // S buffers: 128 + 64*sb
-constexpr uint32_t COL_P0 = 256;    // P buffers (bf16 pairs): 256 + 32*sb
-constexpr uint32_t TMEM_COLS = 512;
+// P (bf16 pairs) of block j goes over the first 32 columns of S buffer j & 1.
+constexpr uint32_t TMEM_COLS = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 
 struct Params {
@@ -59,7 +63,7 @@ struct Bars {
   uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2], pv_done[2], fin;
 };
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     sas_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -199,7 +203,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int st = j % NST;
           const int sb = j & 1;
           ok = mbar_wait(&bars->k_full[st], (j / NST) & 1, status);
-          if (ok && j >= 2) ok = mbar_wait(&bars->p_full[sb], ((j - 2) >> 1) & 1, status);
+          // S buffer sb held S and then P of block j-2: free once that P V has completed.
+          if (ok && j >= 2) ok = mbar_wait(&bars->pv_done[sb], ((j - 2) >> 1) & 1, status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = s_base + OFF_KV + st * STAGE_BYTES;
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t bd = make_sdesc(vb + ks * 2048, KV_HALF, 1024);
-            umma_ts(tmem + COL_O, tmem + COL_P0 + 32 * pb + ks * 8, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
+            umma_ts(tmem + COL_O, tmem + COL_S0 + 64 * pb + ks * 8, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&bars->pv_done[pb]);
           umma_commit(&bars->kv_empty[st]);
@@ -331,7 +336,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         pk[k] = pack_bf16(a0, a1);
       }
       l += rs;
-      tmem_st32(tmem + lane_base + COL_P0 + 32 * sb, pk);
+      tmem_st32(tmem + lane_base + COL_S0 + 64 * sb, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -405,6 +410,10 @@ cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* sta
   prm.n_ptiles = qs.n_ptiles;
   prm.scale_log2 = pb.sm_scale * kLog2e;
   e = cudaFuncSetAttribute(fwd::sas_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  // All of L1 as shared memory, so that two CTAs fit on an SM.
+  e = cudaFuncSetAttribute(fwd::sas_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long long)pb.B * pb.Hkv * qs.n_ptiles);
   fwd::sas_fwd_tc_kernel<<<grid, fwd::THREADS, fwd::SMEM_BYTES, st>>>(tq, tk, tv, prm);
