@@ -76,6 +76,47 @@ def attended_flops(w) -> tuple[float, float]:
     return fwd, 2.5 * fwd
 
 
+def executed_flops(w, sel):
+    """(forward, backward) FLOPs the tensor cores execute for one step, from the selection sel [B,Hkv,T,K-1].
+
+    Forward: every q-tile (P positions x G heads = 128 rows) runs S = Q K^T and O += P V (128 x 64 x 128 MACs
+    each) over its block list: the current block(s) plus the union of its rows' selected blocks. Backward: the
+    CTA of block j runs 5 MMAs of 128 x 64 x 128 MACs per tile of P positions over the positions that attend j
+    (its own 64 and those that selected it). The ratio to the attended FLOPs is the waste of the tiling.
+    """
+    G = w.G
+    P = (128 // G) & ~7
+    B, Hkv, T, H = sel.shape
+    nbg = B * Hkv
+    mma = 2.0 * 128 * 64 * 128
+    n_pt = (T + P - 1) // P
+    s2 = sel.reshape(nbg, T, H).long()
+    if n_pt * P > T:
+        s2 = torch.cat([s2, torch.full((nbg, n_pt * P - T, H), -1, dtype=s2.dtype, device=s2.device)], 1)
+    s2 = s2.reshape(nbg, n_pt, P * H) + 1                     # 0: no block
+    hit = torch.zeros(nbg, n_pt, w.NB + 1, dtype=torch.bool, device=sel.device)
+    hit.scatter_(2, s2, True)
+    t0 = torch.arange(n_pt, device=sel.device) * P
+    t1 = torch.clamp(t0 + P, max=T) - 1
+    n_cur = (t1 // w.block - t0 // w.block + 1).to(torch.float64)
+    fwd = float((hit[:, :, 1:].sum(-1).to(torch.float64) + n_cur).sum()) * 2 * mma
+    counts = torch.zeros(nbg, w.NB + 1, dtype=torch.float64, device=sel.device)
+    counts.scatter_add_(1, sel.reshape(nbg, T * H).long() + 1, torch.ones(nbg, T * H, dtype=torch.float64,
+                                                                        device=sel.device))
+    own = torch.clamp(T - torch.arange(w.NB, device=sel.device) * w.block, max=w.block).to(torch.float64)
+    tiles = torch.ceil((counts[:, 1:] + own) / P)
+    bwd = float(tiles.sum()) * 5 * mma
+    return fwd, bwd
+
+
+def gate_select_bytes(w) -> float:
+    """HBM bytes of normalise + select: the causal part of s read, logG written, its causal part read again,
+    tau and tau_idx written."""
+    c = np.minimum(np.arange(w.T) // w.block, w.NB).astype(np.float64)
+    rows = w.B * w.Hkv
+    return rows * (4.0 * c.sum() * 2 + 4.0 * w.NB * w.T + 8.0 * w.T)
+
+
 def decode_bytes(w) -> float:
     """Algorithmic bytes of one decode step: selected K/V blocks, q, o and the score rows."""
     el = 2 if w.dtype == "bf16" else 4
@@ -316,6 +357,12 @@ def run_gpu(args):
         dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
             ("sas_fwd", fwd_avg, fwd_flops)
         achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+        sel = torch.empty(w.B, w.Hkv, w.T, w.K - 1, dtype=torch.int32, device=device)
+        binding.sas_select_threshold(logG, tau, tidx, sel, w.K, stream=stream)
+        torch.cuda.synchronize(device)
+        ex_fwd, ex_bwd = executed_flops(w, sel)
+        del sel
+        gate_avg = statistics.mean(gate_ms)
         roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": round(achieved / peaks["bf16_tflops"], 4),
@@ -323,7 +370,12 @@ def run_gpu(args):
                     "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
                     "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
                     "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
-                    "gate_select_ms": round(statistics.mean(gate_ms), 4)}
+                    "fwd_executed_tflops": round(ex_fwd / (fwd_avg * 1e-3) / 1e12, 2),
+                    "fwd_inflation": round(ex_fwd / fwd_flops, 3),
+                    "bwd_executed_tflops": round(ex_bwd / (bwd_avg * 1e-3) / 1e12, 2),
+                    "bwd_inflation": round(ex_bwd / bwd_flops, 3),
+                    "gate_select_ms": round(gate_avg, 4),
+                    "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1)}
     else:
         value, ms_per_step, launches, roofline = None, None, 0, None
 

@@ -48,6 +48,8 @@ SMALL = [
     workloads.custom("bf16_g1", "bf16", B=2, Hq=2, Hkv=2, d=128, T=384, K=2),
     workloads.custom("bf16_g8", "bf16", B=1, Hq=8, Hkv=1, d=128, T=640, K=5, s_dist="normal2_planted3"),
     workloads.custom("f32_d128", "f32", B=1, Hq=4, Hkv=2, d=128, T=320, K=3),
+    workloads.custom("bf16_g16", "bf16", B=1, Hq=16, Hkv=1, d=128, T=512, K=4),
+    workloads.custom("bf16_g2_k33", "bf16", B=1, Hq=4, Hkv=2, d=128, T=2304, K=33),
 ]
 
 

@@ -52,3 +52,21 @@ def test_decode_full_size():
     w = workloads.WORKLOADS["decode_b16_l32k"]
     inp = workloads.make_decode_inputs(w)
     check(w, inp)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (10, 2), (16, 1)])
+def test_decode_group_sizes(dtype, Hq, Hkv):
+    """G = 1, 5 and 16 heads per group (the MMA rows past G are padding), ragged lengths incl. 1 and Lmax."""
+    w = workloads.custom("dec_g", dtype, B=4, Hq=Hq, Hkv=Hkv, d=128, T=1600, K=6, decode=True)
+    inp = workloads.make_decode_inputs(w, seed=Hq, seqlen=[1600, 1, 129, 1000])
+    check(w, inp)
+
+
+@pytest.mark.parametrize("K", [2, 64])
+def test_decode_budget_extremes(K):
+    """K = 2 (one selected block) and the largest budget, 64, with lengths that leave fewer historical
+    blocks than the budget (every historical block taken) and lengths that do not."""
+    w = workloads.custom("dec_k", "bf16", B=3, Hq=8, Hkv=2, d=128, T=8192, K=K, decode=True)
+    inp = workloads.make_decode_inputs(w, seed=K, seqlen=[8192, 3000, 700])
+    check(w, inp)
