@@ -73,6 +73,37 @@ def gate_normalize(s, block: int):
 
 
 # --------------------------------------------------------------------------------------
+# Selector-score gradient: SAS paper Appendix D.3 "Gradient Derivation for Training
+# Scope" (the softmax backward ds_m = g_m (dg_m - sum_l g_l dg_l)) and §4.2 eq. 8.
+# With the gate gradient given in log form, dLogG_l = g_l dg_l, this is
+# ds_m = dLogG_m - g_m * sum_l dLogG_l over the historical blocks l < c_t.
+# --------------------------------------------------------------------------------------
+def gate_grad(s, dLogG, block: int):
+    """Return ``ds = dL/ds`` given ``dLogG = dL/dlogG`` for ``logG = gate_normalize(s)``.
+
+    For each row, over the historical blocks m < c_t: the Jacobian of
+    log g_l = s_l - LSE(s) is d log g_l / d s_m = [l == m] - g_m, so
+    ds_m = sum_l dLogG_l ([l == m] - g_m). Entries m >= c_t are 0.
+    s, dLogG: [B, Hkv, T, NB]. Returns float64 of the same shape.
+    """
+    s = _f64(s)
+    dl = _f64(dLogG)
+    B, Hkv, T, NB = s.shape
+    ds = np.zeros(s.shape)
+    for t in range(T):
+        c = min(t // block, NB)
+        if c == 0:
+            continue
+        hist = s[:, :, t, :c]
+        g = np.exp(hist - hist.max(axis=-1, keepdims=True))
+        g = g / g.sum(axis=-1, keepdims=True)
+        d = dl[:, :, t, :c]
+        jac = np.eye(c)[None, None] - g[:, :, None, :]          # [.., l, m] = [l == m] - g_m
+        ds[:, :, t, :c] = np.einsum("bgl,bglm->bgm", d, jac)
+    return ds
+
+
+# --------------------------------------------------------------------------------------
 # Top-K as a per-query threshold: SAS paper §4.3 "Kernel Design" and Appendix E
 # (a block is active when its log gate reaches the per-query threshold tau).
 # Exactly H = K-1 blocks are kept; equal values are broken toward the lower index,

@@ -443,3 +443,59 @@ def test_pins_catch_planted_mistakes(monkeypatch, mistake, target):
     monkeypatch.setattr(orc, bad[0], bad[1])
     with pytest.raises(AssertionError):
         target()
+
+
+# ---------------------------------------------------------------- selector-score gradient
+def _gate_loss(s, w, block):
+    lg = orc.gate_normalize(s, block)
+    return float(np.sum(np.where(np.isfinite(lg), lg * w, 0.0)))
+
+
+def test_gate_grad_matches_central_differences():
+    """ds from gate_grad against central differences of L(s) = sum_m w_m logG_m(s) on every entry."""
+    rng = np.random.default_rng(11)
+    block, T, NB = 4, 20, 5
+    s = rng.standard_normal((1, 2, T, NB)) * 1.5
+    w = rng.standard_normal((1, 2, T, NB))
+    ds = orc.gate_grad(s, w, block)
+    h = 1e-6
+    fd = np.zeros_like(s)
+    for idx in np.ndindex(s.shape):
+        sp, sm = s.copy(), s.copy()
+        sp[idx] += h
+        sm[idx] -= h
+        fd[idx] = (_gate_loss(sp, w, block) - _gate_loss(sm, w, block)) / (2 * h)
+    np.testing.assert_allclose(ds, fd, atol=1e-8)
+
+
+def test_gate_grad_rows_sum_to_zero_and_single_block_rows_vanish():
+    """Shifting a row of s by a constant leaves logG unchanged, so each row of ds sums to zero; a row with a
+    single historical block has logG = 0 whatever s is, so its ds is zero; future blocks get zero."""
+    rng = np.random.default_rng(12)
+    block, T, NB = 8, 64, 8
+    s = rng.standard_normal((2, 1, T, NB))
+    d = rng.standard_normal((2, 1, T, NB))
+    ds = orc.gate_grad(s, d, block)
+    np.testing.assert_allclose(ds.sum(axis=-1), 0.0, atol=1e-12)
+    one = (np.arange(T) // block) == 1
+    assert np.all(ds[:, :, one] == 0.0)
+    c = (np.arange(T) // block)[None, None, :, None]
+    assert np.all(ds[np.broadcast_to(np.arange(NB)[None, None, None, :] >= c, ds.shape)] == 0.0)
+
+
+def _bad_gate_grad(s, dLogG, block):
+    """Mistake: the softmax Jacobian applied without the gate weights (ds = dLogG - mean(dLogG))."""
+    s = np.asarray(s, float)
+    d = np.asarray(dLogG, float)
+    ds = np.zeros(s.shape)
+    for t in range(s.shape[2]):
+        c = min(t // block, s.shape[3])
+        if c:
+            ds[:, :, t, :c] = d[:, :, t, :c] - d[:, :, t, :c].mean(axis=-1, keepdims=True)
+    return ds
+
+
+def test_gate_grad_pin_catches_planted_mistake(monkeypatch):
+    monkeypatch.setattr(orc, "gate_grad", _bad_gate_grad)
+    with pytest.raises(AssertionError):
+        test_gate_grad_matches_central_differences()
