@@ -2,8 +2,8 @@
 
 One step = one pass of the whole training-side path over one batch of the
 Qwen3-4B-like layer (B=1, Hq=32, Hkv=8, d=128, T=8192, block 64, K=16 blocks):
-gate normalisation, Top-K threshold selection, forward and backward
-(dQ/dK/dV/dLogG). The metric is attended-block TFLOP/s: 4*d*sum_rows(n_t) for
+gate normalisation fused with Top-K threshold selection, forward, backward
+(dQ/dK/dV/dLogG) and the selector-score gradient ds. The metric is attended-block TFLOP/s: 4*d*sum_rows(n_t) for
 the forward and 2.5x that for the backward, n_t = (t mod 64) + 1 + 64*min(K-1, c_t)
 attended keys of row t. The memory-bound decode step (16 sequences over a
 32768-token cache) is reported beside it in GB/s.
@@ -59,6 +59,7 @@ def measured_traffic(name: str):
 
 BENCH_WORKLOAD = "qwen3_4b_t8k"
 DECODE_WORKLOAD = "decode_b16_l32k"
+METRIC = "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd+gate-grad step)"
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2, written between timed steps
 
 
@@ -110,11 +111,19 @@ def executed_flops(w, sel):
 
 
 def gate_select_bytes(w) -> float:
-    """HBM bytes of normalise + select: the causal part of s read, logG written, its causal part read again,
+    """HBM bytes of the fused normalise + select: the causal part of s read once, the full logG row written,
     tau and tau_idx written."""
     c = np.minimum(np.arange(w.T) // w.block, w.NB).astype(np.float64)
     rows = w.B * w.Hkv
-    return rows * (4.0 * c.sum() * 2 + 4.0 * w.NB * w.T + 8.0 * w.T)
+    return rows * (4.0 * c.sum() + 4.0 * w.NB * w.T + 8.0 * w.T)
+
+
+def gate_grad_bytes(w) -> float:
+    """HBM bytes of the selector-score gradient: the causal parts of logG and dLogG read, the full ds row
+    written."""
+    c = np.minimum(np.arange(w.T) // w.block, w.NB).astype(np.float64)
+    rows = w.B * w.Hkv
+    return rows * (4.0 * c.sum() * 2 + 4.0 * w.NB * w.T)
 
 
 def decode_bytes(w) -> float:
@@ -271,7 +280,8 @@ def oracle_sample(w, seconds: float, seed: int = 0):
         rows_done += len(rows)
         hi -= 128
     desc = (f"oracle fwd+bwd (materialised, fp64) on {rows_done} query positions x {w.G} heads of one "
-            f"(batch, KV group) of {w.name}; gates normalised/selected by the oracle outside the timing")
+            f"(batch, KV group) of {w.name}; gates normalised/selected by the oracle outside the timing, "
+            f"selector-score gradient not sampled (O(NB) per row against O(n_t d) attention work)")
     return work / elapsed / 1e12, threads, desc
 
 
@@ -301,6 +311,7 @@ def run_gpu(args):
     O = torch.empty_like(Q)
     LSE = torch.empty(w.B, w.Hq, w.T, device=device)
     dQ, dK, dV, dLogG = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s)
+    ds = torch.empty_like(s)
     ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
     ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -309,8 +320,7 @@ def run_gpu(args):
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        binding.sas_gate_normalize(s, logG, stream=stream)
-        binding.sas_select_threshold(logG, tau, tidx, None, w.K, stream=stream)
+        binding.sas_gate_normalize_select(s, logG, tau, tidx, None, w.K, stream=stream)
         if ev:
             ev[1].record(stream)
         binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.sm_scale, ws_f, stream=stream)
@@ -320,6 +330,9 @@ def run_gpu(args):
                         stream=stream)
         if ev:
             ev[3].record(stream)
+        binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
+        if ev:
+            ev[4].record(stream)
 
     legs = set(args.legs.split(","))
     clk = ClockSampler(local).__enter__()   # running through every leg; samples kept while active
@@ -333,7 +346,7 @@ def run_gpu(args):
         if binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b):
             raise RuntimeError("kernel-side timeout during warm-up")
 
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
         barrier(device)
         torch.cuda.synchronize(device)
         launches0 = binding.launch_count()
@@ -343,10 +356,11 @@ def run_gpu(args):
         torch.cuda.synchronize(device)
         launches = binding.launch_count() - launches0
         barrier(device)
-        step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+        step_ms = [e[0].elapsed_time(e[4]) for e in evs]
         fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
         bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
         gate_ms = [e[0].elapsed_time(e[1]) for e in evs]
+        grad_ms = [e[3].elapsed_time(e[4]) for e in evs]
         total_ms = reduce_max(sum(step_ms), device)
         ms_per_step = total_ms / args.steps
         value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
@@ -363,6 +377,7 @@ def run_gpu(args):
         ex_fwd, ex_bwd = executed_flops(w, sel)
         del sel
         gate_avg = statistics.mean(gate_ms)
+        grad_avg = statistics.mean(grad_ms)
         roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": round(achieved / peaks["bf16_tflops"], 4),
@@ -375,7 +390,9 @@ def run_gpu(args):
                     "bwd_executed_tflops": round(ex_bwd / (bwd_avg * 1e-3) / 1e12, 2),
                     "bwd_inflation": round(ex_bwd / bwd_flops, 3),
                     "gate_select_ms": round(gate_avg, 4),
-                    "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1)}
+                    "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1),
+                    "gate_grad_ms": round(grad_avg, 4),
+                    "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1)}
     else:
         value, ms_per_step, launches, roofline = None, None, 0, None
 
@@ -387,7 +404,7 @@ def run_gpu(args):
     clk.__exit__(None, None, None)
 
     result = {
-        "metric": "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd step)",
+        "metric": METRIC,
         "value": round(value, 3) if value is not None else None, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4) if ms_per_step is not None else None, "higher_is_better": True,
@@ -420,7 +437,7 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
                 "dQ": torch.empty(host["Q"].shape, dtype=host["Q"].dtype).pin_memory(),
                 "dK": torch.empty(host["K"].shape, dtype=host["K"].dtype).pin_memory(),
                 "dV": torch.empty(host["V"].shape, dtype=host["V"].dtype).pin_memory(),
-                "dLogG": torch.empty(host["s"].shape, dtype=torch.float32).pin_memory()}
+                "ds": torch.empty(host["s"].shape, dtype=torch.float32).pin_memory()}
     dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in pinned.items()}
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = sum(v.numel() * v.element_size() for v in out_host.values())
@@ -434,7 +451,8 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
                                  check=False)
         dQ, dK, dV, dLogG = binding.backward(dev_in["Q"], dev_in["K"], dev_in["V"], O, dev_in["dO"], logG, tau,
                                              tidx, LSE, w.K, w.sm_scale, stream=stream, check=False)
-        for k, v in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV), ("dLogG", dLogG)):
+        ds = binding.gate_grad(logG, dLogG, stream=stream)
+        for k, v in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV), ("ds", ds)):
             out_host[k].copy_(v, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -531,7 +549,7 @@ def run_reference(args):
     wall = time.perf_counter() - t0
     value = statistics.mean(vals)
     print(json.dumps({
-        "impl": "reference", "metric": "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd step)",
+        "impl": "reference", "metric": METRIC,
         "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",

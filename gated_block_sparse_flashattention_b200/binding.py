@@ -31,6 +31,9 @@ _SIGNATURES = {
     "sas_launch_count": (ctypes.c_uint64, []),
     "sas_gate_normalize": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "sas_gate_normalize_select": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                           _vp]),
+    "sas_gate_grad": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_fwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
     "sas_bwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_decode_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
@@ -119,6 +122,18 @@ def sas_select_threshold(logG, tau, tau_idx, sel, K, block=BLOCK, stream=None):
         _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
 
 
+def sas_gate_normalize_select(s, logG, tau, tau_idx, sel, K, block=BLOCK, stream=None):
+    B, Hkv, T, NB = s.shape
+    _check("sas_gate_normalize_select", lib().sas_gate_normalize_select(
+        _ptr(s), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
+
+
+def sas_gate_grad(logG, dLogG, ds, block=BLOCK, stream=None):
+    B, Hkv, T, NB = logG.shape
+    _check("sas_gate_grad", lib().sas_gate_grad(
+        _ptr(logG), _ptr(dLogG), _ptr(ds), B, Hkv, T, NB, block, _stream(stream)))
+
+
 def _ws_size(name, *args) -> int:
     out = _sz(0)
     _check(name, getattr(lib(), name)(*args, ctypes.byref(out)))
@@ -202,9 +217,15 @@ def gate_and_select(s, K, block=BLOCK, want_sel=False, stream=None):
     tau = torch.empty(B, Hkv, T, dtype=torch.float32, device=s.device)
     tidx = torch.empty(B, Hkv, T, dtype=torch.int32, device=s.device)
     sel = torch.empty(B, Hkv, T, max(K - 1, 1), dtype=torch.int32, device=s.device) if want_sel else None
-    sas_gate_normalize(s, logG, block, stream)
-    sas_select_threshold(logG, tau, tidx, sel, K, block, stream)
+    sas_gate_normalize_select(s, logG, tau, tidx, sel, K, block, stream)
     return logG, tau, tidx, sel
+
+
+def gate_grad(logG, dLogG, block=BLOCK, stream=None):
+    """ds = dL/ds [B,Hkv,T,NB] from the log-gate gradient of ``backward`` and the gates of ``gate_and_select``."""
+    ds = torch.empty_like(dLogG)
+    sas_gate_grad(logG, dLogG, ds, block, stream)
+    return ds
 
 
 def _check_device_status(fn, ws, stream):

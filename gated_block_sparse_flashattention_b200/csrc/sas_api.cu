@@ -99,6 +99,26 @@ int sas_select_threshold(const float* logG, float* tau, int32_t* tau_idx, int32_
       launch_select_threshold(logG, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB, K - 1, as_stream(stream)));
 }
 
+int sas_gate_normalize_select(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel, int B, int Hkv,
+                              int T, int NB, int block, int K, void* stream) {
+  if (!s || !logG || !tau || !tau_idx || s == logG) return SAS_ERR_INVALID_ARG;
+  if (!aligned16(s) || !aligned16(logG) || !aligned16(tau) || !aligned16(tau_idx)) return SAS_ERR_INVALID_ARG;
+  if (sel && !aligned16(sel)) return SAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || T <= 0 || NB <= 0 || block != 64 || K < 1) return SAS_ERR_INVALID_ARG;
+  if ((long long)NB * 64 < T) return SAS_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_normalize_select(s, logG, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB, K - 1, as_stream(stream)));
+}
+
+int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int B, int Hkv, int T, int NB, int block,
+                  void* stream) {
+  if (!logG || !dLogG || !ds || ds == logG || ds == dLogG) return SAS_ERR_INVALID_ARG;
+  if (!aligned16(logG) || !aligned16(dLogG) || !aligned16(ds)) return SAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || T <= 0 || NB <= 0 || block != 64) return SAS_ERR_INVALID_ARG;
+  if ((long long)NB * 64 < T) return SAS_ERR_INVALID_ARG;
+  return cuda_status(launch_gate_grad(logG, dLogG, ds, (long long)B * Hkv * T, T, NB, as_stream(stream)));
+}
+
 int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes) {
   if (!bytes) return SAS_ERR_INVALID_ARG;
   const int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);

@@ -36,13 +36,11 @@ __global__ void __launch_bounds__(256) gate_normalize_kernel(const float* __rest
 }
 
 // Threshold (tau, tau_idx) and optional ascending index list of one row whose
-// keys fit in KREG registers per lane.
+// keys are in KREG registers per lane (key of block m = lane + 32 i in keys[i]).
 template <int KREG>
-__device__ __forceinline__ void select_row_regs(const float* __restrict__ v, int c, int H, uint32_t* hist,
-                                                float* tau_out, int32_t* tidx_out, int32_t* out) {
+__device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], int c, int H, uint32_t* hist,
+                                                 float* tau_out, int32_t* tidx_out, int32_t* out) {
   const int lane = threadIdx.x & 31;
-  uint32_t keys[KREG];
-  load_row_keys(v, c, keys);
   uint32_t tkey = 0u, asc = 0u;
   int tidx = -1;
   if (H <= 32 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, &asc)) {
@@ -75,6 +73,38 @@ __device__ __forceinline__ void select_row_regs(const float* __restrict__ v, int
   }
 }
 
+template <int KREG>
+__device__ __forceinline__ void select_row_regs(const float* __restrict__ v, int c, int H, uint32_t* hist,
+                                                float* tau_out, int32_t* tidx_out, int32_t* out) {
+  uint32_t keys[KREG];
+  load_row_keys(v, c, keys);
+  select_keys_regs(keys, c, H, hist, tau_out, tidx_out, out);
+}
+
+// Rows that select nothing or everything: (+inf, -1) / (-inf, c-1) and the list.
+__device__ __forceinline__ bool select_trivial_row(int c, int H, float* tau_out, int32_t* tidx_out, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  if (min(c, H) == 0) {
+    if (lane == 0) {
+      *tau_out = INFINITY;
+      *tidx_out = -1;
+    }
+    if (out)
+      for (int k = lane; k < H; k += 32) out[k] = -1;
+    return true;
+  }
+  if (c <= H) {
+    if (lane == 0) {
+      *tau_out = -INFINITY;
+      *tidx_out = c - 1;
+    }
+    if (out)
+      for (int k = lane; k < H; k += 32) out[k] = (k < c) ? k : -1;
+    return true;
+  }
+  return false;
+}
+
 __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __restrict__ logG, float* __restrict__ tau,
                                                                int32_t* __restrict__ tau_idx,
                                                                int32_t* __restrict__ sel, long long rows, int T,
@@ -88,24 +118,7 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
   const int c = min(t / kBlock, NB);
   const float* v = logG + row * (long long)NB;
   int32_t* out = sel ? sel + row * (long long)H : nullptr;
-  if (min(c, H) == 0) {
-    if (lane == 0) {
-      tau[row] = INFINITY;
-      tau_idx[row] = -1;
-    }
-    if (out)
-      for (int k = lane; k < H; k += 32) out[k] = -1;
-    return;
-  }
-  if (c <= H) {
-    if (lane == 0) {
-      tau[row] = -INFINITY;
-      tau_idx[row] = c - 1;
-    }
-    if (out)
-      for (int k = lane; k < H; k += 32) out[k] = (k < c) ? k : -1;
-    return;
-  }
+  if (select_trivial_row(c, H, tau + row, tau_idx + row, out)) return;
   if (c <= 32 * kSelectReg) {
     // Keys in registers: one read of the row; the threshold, the tie index and
     // the index list all work on them (register width picked by row length).
@@ -141,6 +154,86 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
     }
     for (int k = pos + lane; k < H; k += 32) out[k] = -1;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Normalisation and selection in one pass (one warp per row, the row in
+// registers): the same logG values as gate_normalize_kernel (same arithmetic,
+// same summation order) written once, and the selection taken on them, so the
+// outputs equal the two separate calls bit for bit. Rows longer than
+// 32 * kSelectReg blocks use the two kernels.
+// ---------------------------------------------------------------------------
+template <int KREG>
+__device__ __forceinline__ void normalize_select_row(const float* __restrict__ src, float* __restrict__ dst, int c,
+                                                     int NB, int H, uint32_t* hist, float* tau_out,
+                                                     int32_t* tidx_out, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  float v[KREG];
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) v[i] = (lane + 32 * i < c) ? __ldg(src + lane + 32 * i) : -INFINITY;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) mx = fmaxf(mx, v[i]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i)
+    if (lane + 32 * i < c) sum += expf(v[i] - mx);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float lse = mx + logf(sum);
+  uint32_t keys[KREG];
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    const int m = lane + 32 * i;
+    const float lg = (m < c) ? v[i] - lse : -INFINITY;
+    if (m < NB) dst[m] = lg;
+    keys[i] = (m < c) ? float_key(lg) : 0u;
+  }
+  for (int m = lane + 32 * KREG; m < NB; m += 32) dst[m] = -INFINITY;
+  if (select_trivial_row(c, H, tau_out, tidx_out, out)) return;
+  select_keys_regs(keys, c, H, hist, tau_out, tidx_out, out);
+}
+
+// KREG from the row length NB on the host, so short rows run with few registers
+// (and many warps per SM): the pivot select is instruction-bound.
+template <int KREG>
+__global__ void __launch_bounds__(256) normalize_select_kernel(const float* __restrict__ s, float* __restrict__ logG,
+                                                               float* __restrict__ tau, int32_t* __restrict__ tau_idx,
+                                                               int32_t* __restrict__ sel, long long rows, int T,
+                                                               int NB, int H) {
+  __shared__ __align__(16) uint32_t hist_all[8][256];   // per-warp scratch of the select
+  const int wid = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * 8 + wid;
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  int32_t* out = sel ? sel + row * (long long)H : nullptr;
+  normalize_select_row<KREG>(s + row * (long long)NB, logG + row * (long long)NB, c, NB, H, hist_all[wid],
+                             tau + row, tau_idx + row, out);
+}
+
+// ---------------------------------------------------------------------------
+// Selector-score gradient (SAS paper Appendix D.3, the softmax backward, with the
+// gate gradient in log form): ds[m] = dLogG[m] - exp(logG[m]) * sum_{l<c} dLogG[l]
+// for m < c_t, 0 otherwise. One warp per row; HBM-bound.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gate_grad_kernel(const float* __restrict__ logG, const float* __restrict__ dLogG,
+                                                        float* __restrict__ ds, long long rows, int T, int NB) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  const float* lg = logG + row * (long long)NB;
+  const float* dl = dLogG + row * (long long)NB;
+  float* out = ds + row * (long long)NB;
+  float sum = 0.f;
+  for (int m = lane; m < c; m += 32) sum += __ldg(dl + m);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  for (int m = lane; m < NB; m += 32) out[m] = (m < c) ? __ldg(dl + m) - expf(__ldg(lg + m)) * sum : 0.f;
 }
 
 // ---------------------------------------------------------------------------
@@ -199,6 +292,33 @@ cudaError_t launch_select_threshold(const float* logG, float* tau, int32_t* tau_
                                     int T, int NB, int H, cudaStream_t st) {
   const long long blocks = (rows + 7) / 8;
   select_threshold_kernel<<<(unsigned)blocks, 256, 0, st>>>(logG, tau, tau_idx, sel, rows, T, NB, H);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_normalize_select(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel,
+                                    long long rows, int T, int NB, int H, cudaStream_t st) {
+  if (NB > 32 * kSelectReg) {   // rows longer than the registers hold: two passes
+    cudaError_t e = launch_gate_normalize(s, logG, rows, T, NB, st);
+    if (e != cudaSuccess) return e;
+    return launch_select_threshold(logG, tau, tau_idx, sel, rows, T, NB, H, st);
+  }
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (NB <= 128)
+    normalize_select_kernel<4><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 256)
+    normalize_select_kernel<8><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 512)
+    normalize_select_kernel<16><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
+  else
+    normalize_select_kernel<kSelectReg><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_grad(const float* logG, const float* dLogG, float* ds, long long rows, int T, int NB,
+                             cudaStream_t st) {
+  gate_grad_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(logG, dLogG, ds, rows, T, NB);
   count_launch();
   return cudaGetLastError();
 }

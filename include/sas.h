@@ -108,6 +108,29 @@ SAS_API int sas_select_threshold(const float* logG, float* tau, int32_t* tau_idx
                          int NB, int block, int K, void* stream);
 
 /*
+ * sas_gate_normalize_select - sas_gate_normalize followed by sas_select_threshold
+ * in one pass over s: logG, tau, tau_idx and sel are bit for bit the values the
+ * two calls produce (same arithmetic and summation order), with s read once and
+ * logG not read back. Arguments, layouts and errors are those of the two calls
+ * (s and logG may not alias).
+ */
+SAS_API int sas_gate_normalize_select(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel, int B,
+                                      int Hkv, int T, int NB, int block, int K, void* stream);
+
+/*
+ * sas_gate_grad - gradient with respect to the selector scores s through the
+ * gate normalisation (SAS paper Appendix D.3, the softmax backward
+ * ds_m = g_m (dg_m - sum_l g_l dg_l), with the gate gradient given in log form
+ * dLogG_l = g_l dg_l as sas_bwd returns it, and g = exp(logG)):
+ *   ds[b,g,t,m] = dLogG[b,g,t,m] - exp(logG[b,g,t,m]) * sum_{l < c_t} dLogG[b,g,t,l]  for m < c_t,
+ *   ds[b,g,t,m] = 0                                                                   for m >= c_t.
+ * logG (from sas_gate_normalize), dLogG, ds: [B,Hkv,T,NB] fp32; ds may not alias
+ * either input. NB >= ceil(T / block), block == 64.
+ */
+SAS_API int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int B, int Hkv, int T, int NB, int block,
+                          void* stream);
+
+/*
  * Workspace sizes (bytes) for sas_fwd, sas_bwd and sas_decode_fwd with the given
  * sizes. The workspace is caller-owned device memory, at least 256-byte aligned,
  * and may be reused across calls on the same stream. Its first word is the

@@ -406,3 +406,38 @@ def decode(q, Kc, Vc, seqlen, s, K: int, block: int, sm_scale: float, apply_log_
                 e = np.exp(z - z.max())
                 o[b, h] = (e / e.sum()) @ Vc[b, g, idx]
     return o, sel
+
+
+def paged_cache(pool, page_table, block: int):
+    """Logical KV cache [B, Hkv, max_pages*block, d] of a paged pool.
+
+    pool [num_pages, Hkv, block, d] holds one block of ``block`` tokens of every
+    KV head per page; page_table [B, max_pages] names, for each sequence and
+    logical block m, the page holding its tokens m*block .. m*block+block-1
+    (-1 for blocks the sequence does not reach; they read as zeros and are never
+    attended). Plain gather, one page at a time.
+    """
+    pool = _f64(pool)
+    num_pages, Hkv, bl, d = pool.shape
+    assert bl == block
+    B, max_pages = page_table.shape
+    out = np.zeros((B, Hkv, max_pages * block, d))
+    for b in range(B):
+        for m in range(max_pages):
+            pg = int(page_table[b, m])
+            if pg >= 0:
+                out[b, :, m * block:(m + 1) * block] = pool[pg]
+    return out
+
+
+def decode_paged(q, Kpool, Vpool, page_table, seqlen, s, K: int, block: int, sm_scale: float,
+                 apply_log_gate: bool = False):
+    """The decode step of ``decode`` over a paged KV cache (pages of one block).
+
+    The paged layout only changes where a token's key and value are stored, not
+    what is computed (§5.1 "Inference implementation": only the selected KV
+    blocks are gathered), so this is ``decode`` on the logical cache that
+    ``paged_cache`` rebuilds.
+    """
+    return decode(q, paged_cache(Kpool, page_table, block), paged_cache(Vpool, page_table, block), seqlen, s, K,
+                  block, sm_scale, apply_log_gate)

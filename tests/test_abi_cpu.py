@@ -79,6 +79,15 @@ def test_invalid_calls_return_errors_without_launching(lib):
     assert lib.sas_gate_normalize(fake, fake + 64, 1, 1, 64, 1, 32, None) == -1     # block != 64
     assert lib.sas_gate_normalize(fake + 4, fake + 64, 1, 1, 64, 1, 64, None) == -1  # misaligned
     assert lib.sas_select_threshold(fake, fake, fake, None, 1, 1, 128, 2, 64, 0, None) == -1  # K < 1
+    assert lib.sas_gate_normalize_select(fake, fake + 64, fake + 128, fake + 192, None, 1, 1, 128, 2, 64, 0,
+                                         None) == -1                                # K < 1
+    assert lib.sas_gate_normalize_select(fake, fake, fake + 128, fake + 192, None, 1, 1, 128, 2, 64, 4,
+                                         None) == -1                                # s aliases logG
+    assert lib.sas_gate_normalize_select(fake, fake + 64, fake + 128, fake + 192, None, 1, 1, 192, 2, 64, 4,
+                                         None) == -1                                # NB * 64 < T
+    assert lib.sas_gate_grad(fake, fake + 64, fake + 64, 1, 1, 128, 2, 64, None) == -1   # ds aliases dLogG
+    assert lib.sas_gate_grad(fake, fake + 64, fake + 132, 1, 1, 128, 2, 64, None) == -1  # misaligned ds
+    assert lib.sas_gate_grad(fake, fake + 64, fake + 128, 1, 1, 128, 2, 32, None) == -1  # block != 64
     # sas_fwd: missing workspace / bad sizes
     args = [fake] * 3 + [binding.SAS_DT_BF16] + [fake] * 5 + [1, 4, 1, 128, 128, 64, ctypes.c_float(0.1), None, 0, None]
     assert lib.sas_fwd(*args) == -5

@@ -499,3 +499,60 @@ def test_gate_grad_pin_catches_planted_mistake(monkeypatch):
     monkeypatch.setattr(orc, "gate_grad", _bad_gate_grad)
     with pytest.raises(AssertionError):
         test_gate_grad_matches_central_differences()
+
+
+# ---------------------------------------------------------------- paged decode
+def _paged_layout(Kc, Vc, seqlen, block, rng, spare=5):
+    """Scatter a contiguous cache into a shuffled pool of one-block pages (plus unused pages)."""
+    B, Hkv, Lmax, d = Kc.shape
+    max_pages = Lmax // block
+    used = [(b, m) for b in range(B) for m in range((int(seqlen[b]) + block - 1) // block)]
+    num_pages = len(used) + spare
+    perm = rng.permutation(num_pages)
+    Kp = rng.standard_normal((num_pages, Hkv, block, d))     # unused pages hold noise
+    Vp = rng.standard_normal((num_pages, Hkv, block, d))
+    pt = np.full((B, max_pages), -1, dtype=np.int32)
+    for i, (b, m) in enumerate(used):
+        pt[b, m] = perm[i]
+        Kp[perm[i]] = Kc[b, :, m * block:(m + 1) * block]
+        Vp[perm[i]] = Vc[b, :, m * block:(m + 1) * block]
+    return Kp, Vp, pt
+
+
+def test_paged_decode_equals_contiguous_decode_under_a_page_shuffle():
+    B, Hq, Hkv, Lmax, d, block = 3, 4, 2, 256, 8, 16
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((B, Hq, d))
+    Kc, Vc = rng.standard_normal((B, Hkv, Lmax, d)), rng.standard_normal((B, Hkv, Lmax, d))
+    seqlen = np.array([256, 131, 16])
+    s = rng.standard_normal((B, Hkv, Lmax // block))
+    Kp, Vp, pt = _paged_layout(Kc, Vc, seqlen, block, rng)
+    for Kb, gate in ((4, False), (3, True), (100, False)):
+        o_ref, sel_ref = orc.decode(q, Kc, Vc, seqlen, s, Kb, block, 0.3, apply_log_gate=gate)
+        o, sel = orc.decode_paged(q, Kp, Vp, pt, seqlen, s, Kb, block, 0.3, apply_log_gate=gate)
+        np.testing.assert_allclose(o, o_ref, atol=1e-12)
+        assert np.array_equal(sel, sel_ref)
+    # the logical cache itself, token by token
+    Kl = orc.paged_cache(Kp, pt, block)
+    for b in range(B):
+        for p in range(int(seqlen[b])):
+            np.testing.assert_array_equal(Kl[b, :, p], Kc[b, :, p])
+
+
+def _bad_paged_cache(pool, page_table, block):
+    """Mistake: the page table read with sequence and block swapped."""
+    pool = np.asarray(pool, float)
+    B, max_pages = page_table.shape
+    out = np.zeros((B, pool.shape[1], max_pages * block, pool.shape[3]))
+    for b in range(B):
+        for m in range(max_pages):
+            pg = int(page_table.T.reshape(B, max_pages)[b, m])
+            if pg >= 0:
+                out[b, :, m * block:(m + 1) * block] = pool[pg]
+    return out
+
+
+def test_paged_pin_catches_planted_mistake(monkeypatch):
+    monkeypatch.setattr(orc, "paged_cache", _bad_paged_cache)
+    with pytest.raises(AssertionError):
+        test_paged_decode_equals_contiguous_decode_under_a_page_shuffle()
