@@ -59,6 +59,7 @@ def measured_traffic(name: str):
 
 BENCH_WORKLOAD = "qwen3_4b_t8k"
 DECODE_WORKLOAD = "decode_b16_l32k"
+PAGED_DECODE_WORKLOAD = "decode_b8_l512k_paged"
 METRIC = "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd+gate-grad step)"
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2, written between timed steps
 
@@ -400,6 +401,7 @@ def run_gpu(args):
     clk.active = True
     e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
     dec = run_decode(args, device, stream, binding, peaks, clk) if "decode" in legs else None
+    dec_paged = run_decode_paged(args, device, stream, binding, peaks, clk) if "paged" in legs else None
     clk.active = False
     clk.__exit__(None, None, None)
 
@@ -418,6 +420,7 @@ def run_gpu(args):
         "e2e": e2e,
         "gpu_launches": launches,
         "decode": dec,
+        "decode_paged": dec_paged,
     }
     if rank == 0 and world == 1 and "cpu" in legs:
         tf, threads, desc = oracle_sample(w, args.cpu_seconds)
@@ -472,6 +475,40 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(total / args.steps, 4)}
 
 
+def _time_decode_graph(call, n_rot, args, device, stream, binding, clk):
+    """Captures n_rot back-to-back calls call(i) in one CUDA graph and returns the median device time per
+    call (ms) over max(4, steps) replays, and the kernels one call launches."""
+    g_stream = torch.cuda.Stream(device)
+    g_stream.wait_stream(stream)
+    launches0 = binding.launch_count()
+    with torch.cuda.stream(g_stream):
+        call(0, g_stream)
+        per_call = binding.launch_count() - launches0
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=g_stream):
+            for i in range(n_rot):
+                call(i, g_stream)
+    stream.wait_stream(g_stream)
+    torch.cuda.synchronize(device)
+    if clk is not None:
+        clk.active = True
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize(device)
+    reps = max(4, args.steps)
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize(device)
+    med = statistics.median([a.elapsed_time(b) for a, b in times]) / n_rot
+    del graph
+    return med, per_call, reps
+
+
 def run_decode(args, device, stream, binding, peaks, clk=None):
     """Decode step (16 sequences x 1 token over a 32768-token cache), 16 steps per CUDA graph.
 
@@ -491,44 +528,48 @@ def run_decode(args, device, stream, binding, peaks, clk=None):
     s_rot = [torch.randn(w.B, w.Hkv, w.NB, generator=gen).to(device) for _ in range(n_rot)]
     o = torch.empty_like(q)
     ws = binding.workspace(binding.sas_decode_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K), device)
-    g_stream = torch.cuda.Stream(device)
-    g_stream.wait_stream(stream)
-    launches0 = binding.launch_count()
-    with torch.cuda.stream(g_stream):
-        binding.sas_decode_fwd(q, Kc, Vc, seqlen, s_rot[0], w.K, o, ws, w.sm_scale, stream=g_stream)
-        per_call = binding.launch_count() - launches0
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=g_stream):
-            for i in range(n_rot):
-                binding.sas_decode_fwd(q, Kc, Vc, seqlen, s_rot[i], w.K, o, ws, w.sm_scale, stream=g_stream)
-    stream.wait_stream(g_stream)
-    torch.cuda.synchronize(device)
-    if clk is not None:
-        clk.active = True
-    for _ in range(max(args.warmup, 3)):
-        graph.replay()
-    torch.cuda.synchronize(device)
-    reps = max(4, args.steps)
-    times = []
-    if clk is not None:
-        clk.active = True
-    for _ in range(reps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        graph.replay()
-        b.record(stream)
-        times.append((a, b))
-    torch.cuda.synchronize(device)
-    med = statistics.median([a.elapsed_time(b) for a, b in times]) / n_rot
+
+    def call(i, st):
+        binding.sas_decode_fwd(q, Kc, Vc, seqlen, s_rot[i], w.K, o, ws, w.sm_scale, stream=st)
+
+    med, per_call, reps = _time_decode_graph(call, n_rot, args, device, stream, binding, clk)
     gbs = decode_bytes(w) / (med * 1e-3) / 1e9
-    st = binding.sas_device_status(ws)
-    del graph
     return {"workload": "decode_b16_l32k: 16 seqs x 1 token, cache 32768, Hq=32 Hkv=8 d=128 K=16",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": decode_bytes(w), "peak": peaks["hbm_gbs"],
             "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": measured_traffic("decode"),
             "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
-            "launches_per_step": per_call, "device_status": st,
+            "launches_per_step": per_call, "device_status": binding.sas_device_status(ws),
+            "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
+
+
+def run_decode_paged(args, device, stream, binding, peaks, clk=None):
+    """Long-context decode over a paged cache: 8 sequences x 1 token at 524288 tokens of context (8192 pages
+    of 64 tokens per sequence, shuffled in a 19 GB pool), budget 32 blocks, 16 steps per CUDA graph with
+    rotating seeded score tensors as in run_decode."""
+    w = workloads.WORKLOADS[PAGED_DECODE_WORKLOAD]
+    n_rot = 16
+    inp = workloads.make_paged_decode_inputs(w, seed=0, device=device)
+    gen = torch.Generator(device=device).manual_seed(1)
+    s_rot = [torch.randn(w.B, w.Hkv, w.NB, generator=gen, device=device) for _ in range(n_rot)]
+    o = torch.empty_like(inp["q"])
+    ws = binding.workspace(binding.sas_decode_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K), device)
+
+    def call(i, st):
+        binding.sas_decode_fwd_paged(inp["q"], inp["Kp"], inp["Vp"], inp["page_table"], inp["seqlen"], s_rot[i],
+                                     w.K, o, ws, w.sm_scale, stream=st)
+
+    med, per_call, reps = _time_decode_graph(call, n_rot, args, device, stream, binding, clk)
+    nbytes = decode_bytes(w) + w.B * w.Hkv * w.K * 4.0   # + the page-table entries of the attended blocks
+    gbs = nbytes / (med * 1e-3) / 1e9
+    pool_gb = 2 * inp["Kp"].numel() * inp["Kp"].element_size() / 1e9
+    del inp
+    return {"workload": f"decode_b8_l512k_paged: 8 seqs x 1 token, context 524288 (8192 pages of 64 tokens "
+                        f"each, {pool_gb:.1f} GB K/V pool), Hq=32 Hkv=8 d=128 K=32",
+            "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
+            "bytes_per_step": nbytes, "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "traffic": None, "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
+            "launches_per_step": per_call, "device_status": binding.sas_device_status(ws),
             "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
 
 
@@ -567,9 +608,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--legs", default="step,e2e,decode,cpu",
+    ap.add_argument("--legs", default="step,e2e,decode,paged,cpu",
                     help="comma list of what to measure and report: step (device-resident timed steps), e2e "
-                         "(host buffers through the C ABI), decode, cpu (oracle baseline)")
+                         "(host buffers through the C ABI), decode, paged (long-context paged decode), cpu (oracle "
+                         "baseline)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3

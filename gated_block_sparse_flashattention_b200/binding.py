@@ -42,6 +42,8 @@ _SIGNATURES = {
                 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                        + [_c_f, _vp, _sz, _vp]),
+    "sas_decode_fwd_paged": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _c_int, _c_int, _vp,
+                                      _vp] + [_c_int] * 6 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd_static": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                               + [_c_f, _vp]),
     "sas_device_status": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
@@ -184,6 +186,19 @@ def sas_decode_fwd(q, Kc, Vc, seqlen, s, K, o, ws, sm_scale, sel_out=None, apply
         _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(seqlen), _ptr(s), K, 1 if apply_log_gate else 0,
         _ptr(o), _ptr(sel_out), B, Hq, Hkv, Lmax, NBmax, d, block, float(sm_scale), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sas_decode_fwd_paged(q, Kp, Vp, page_table, seqlen, s, K, o, ws, sm_scale, sel_out=None, apply_log_gate=False,
+                         block=BLOCK, stream=None):
+    """Kp/Vp [num_pages, Hkv, 64, d]; page_table [B, max_pages] int32 on the device."""
+    B, Hq, d = q.shape
+    num_pages, Hkv = Kp.shape[0], Kp.shape[1]
+    max_pages = page_table.shape[1]
+    NBmax = s.shape[-1]
+    _check("sas_decode_fwd_paged", lib().sas_decode_fwd_paged(
+        _ptr(q), _ptr(Kp), _ptr(Vp), _dtype_code(q), _ptr(page_table), max_pages, num_pages, _ptr(seqlen), _ptr(s),
+        K, 1 if apply_log_gate else 0, _ptr(o), _ptr(sel_out), B, Hq, Hkv, NBmax, d, block, float(sm_scale),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def sas_decode_fwd_static(q, Kc, Vc, seqlen, s, K, o, sm_scale, sel_out=None, apply_log_gate=False, block=BLOCK,

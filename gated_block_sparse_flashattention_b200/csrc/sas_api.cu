@@ -256,6 +256,48 @@ int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dtype, con
   return cuda_status(launch_decode(pb, ws, as_stream(stream)));
 }
 
+int sas_decode_fwd_paged(const void* q, const void* Kp, const void* Vp, int dtype, const int32_t* page_table,
+                         int max_pages, int num_pages, const int32_t* seqlen, const float* s, int K, int apply_log_gate,
+                         void* o, int32_t* sel_out, int B, int Hq, int Hkv, int NBmax, int d, int block,
+                         float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+  const void* ptrs[] = {q, Kp, Vp, page_table, seqlen, s, o};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return SAS_ERR_INVALID_ARG;
+  if (dtype != SAS_DT_F32 && dtype != SAS_DT_BF16) return SAS_ERR_INVALID_ARG;
+  if (dtype != SAS_DT_BF16) return SAS_ERR_UNSUPPORTED;   // the paged path is the tensor-core kernel
+  if (max_pages < 1 || num_pages < 1 || Hkv <= 0) return SAS_ERR_INVALID_ARG;
+  if ((long long)max_pages * 64 > INT32_MAX || (long long)num_pages * Hkv > INT32_MAX) return SAS_ERR_INVALID_ARG;
+  if (NBmax < max_pages || !(sm_scale > 0.f)) return SAS_ERR_INVALID_ARG;
+  const int Lmax = max_pages * 64;
+  size_t need = 0;
+  int st = sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, block, K, &need);
+  if (st != SAS_OK) return st;
+  if (!ws || !aligned256(ws) || ws_bytes < need) return SAS_ERR_WORKSPACE;
+  DecodeProblem pb{};
+  pb.B = B;
+  pb.Hq = Hq;
+  pb.Hkv = Hkv;
+  pb.Lmax = Lmax;
+  pb.NBmax = NBmax;
+  pb.d = d;
+  pb.K = K;
+  pb.apply_log_gate = apply_log_gate ? 1 : 0;
+  pb.dtype = dtype;
+  pb.sm_scale = sm_scale;
+  pb.q = q;
+  pb.Kc = Kp;
+  pb.Vc = Vp;
+  pb.seqlen = seqlen;
+  pb.s = s;
+  pb.o = o;
+  pb.sel_out = sel_out;
+  pb.page_table = page_table;
+  pb.max_pages = max_pages;
+  pb.num_pages = num_pages;
+  return cuda_status(launch_decode(pb, ws, as_stream(stream)));
+}
+
 int sas_decode_fwd_static(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen,
                           const float* s, int K, int apply_log_gate, void* o, int32_t* sel_out, int B, int Hq,
                           int Hkv, int Lmax, int NBmax, int d, int block, float sm_scale, void* stream) {

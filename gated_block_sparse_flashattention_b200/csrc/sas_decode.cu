@@ -44,11 +44,14 @@ struct Params {
   int32_t* status;     // device status word (first word of the workspace)
   int32_t* att;        // [B*Hkv][K] attended blocks: [current, selected ascending], -1 padded
   float* lse_gate;     // [B*Hkv] log-sum-exp of the historical scores (log-gate option)
+  int32_t* att_z;      // [B*Hkv][K] paged cache: plane (page * Hkv + g) of each attended block, -1 none
+  const int32_t* page_table;   // [B][max_pages] page of each logical block (null: contiguous cache)
   int32_t* tickets;    // [B*Hkv] (fp32 attention kernel)
   int32_t* work;       // a counter the select kernel clears (unused by the current kernels)
   float* part_ml;      // [B*Hkv][n_slots][G][2]
   float* part_o;       // [B*Hkv][n_slots][G][D]
   int B, Hq, Hkv, Lmax, NBmax, K, apply_log_gate, G;
+  int max_pages, num_pages;   // paged cache only
   int n_slots;         // partial slots per (b, g)
   float sm_scale;
 };
@@ -77,6 +80,61 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 // ---------------------------------------------------------------------------- selection
+// Emits the H largest of n keys held in registers (position q = lane + 32 i in
+// keys[i]; ties toward the lower position) as the list out[0..) of idx(q) in
+// ascending q, also to so[0..) when requested; returns how many (min(n, H)).
+// idx must be increasing in q, so the list is ascending in idx too. Warp-collective.
+template <int KREG, typename Idx>
+__device__ __forceinline__ int select_keys_list(const uint32_t (&keys)[KREG], int n, int H, uint2* cand, Idx idx,
+                                                int32_t* out, int32_t* so) {
+  const int lane = threadIdx.x & 31;
+  if (n <= H) {   // every key
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) {
+      const int q = lane + 32 * i;
+      if (q < n) {
+        const int v = idx(q);
+        out[q] = v;
+        if (so) so[q] = v;
+      }
+    }
+    return n;
+  }
+  uint32_t tk = 0u, asc = 0u;
+  int tidx = -1;
+  if (H <= 32 && pivot_select_keys(keys, n, H, cand, &tk, &tidx, &asc)) {
+    if (lane < H) {
+      const int v = idx((int)asc);
+      out[lane] = v;
+      if (so) so[lane] = v;
+    }
+    return H;
+  }
+  int take_eq = 0;
+  tk = radix_select_keys(keys, n, H, nullptr, &take_eq);
+  tidx = tie_index_keys(keys, n, tk, take_eq);
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    if (32 * i >= n) break;
+    const int q = lane + 32 * i;
+    const bool take = q < n && (keys[i] > tk || (keys[i] == tk && q <= tidx));
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int lp = cnt + __popc(bal & ((1u << lane) - 1u));
+      const int v = idx(q);
+      out[lp] = v;
+      if (so) so[lp] = v;
+    }
+    cnt += __popc(bal);
+  }
+  return cnt;
+}
+
+struct IdentityIdx {
+  __device__ int operator()(int q) const { return q; }
+};
+
 // Emits the selected blocks of one score row (keys in registers) as the ascending
 // list att[1..] (and so[0..] when requested); returns how many.
 template <int KREG>
@@ -92,33 +150,32 @@ __device__ __forceinline__ int decode_select_row(const float* __restrict__ srow,
   }
   uint32_t keys[KREG];
   load_row_keys(srow, c, keys);
-  uint32_t tk = 0u, asc = 0u;
-  int tidx = -1;
-  if (H <= 32 && pivot_select_keys(keys, c, H, cand, &tk, &tidx, &asc)) {
-    if (lane < H) {
-      att[1 + lane] = (int32_t)asc;
-      if (so) so[lane] = (int32_t)asc;
+  return select_keys_list(keys, c, H, cand, IdentityIdx{}, att + 1, so);
+}
+
+// Paged cache: the plane (page * Hkv + g) of every attended block of (b, g) for
+// the attention kernel's copies. A page outside 0..num_pages-1 is reported as a
+// bounds error and its block dropped from the list. Warp-collective; the warp
+// wrote att itself (visible to its lanes after the __syncwarp).
+__device__ __forceinline__ void map_pages(const Params& p, int bg, int32_t* att) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  int32_t* z = p.att_z + (long long)bg * p.K;
+  for (int k = lane; k < p.K; k += 32) {
+    const int m = att[k];
+    int zz = -1;
+    if (m >= 0) {
+      const int pg = (m < p.max_pages) ? __ldg(p.page_table + (long long)b * p.max_pages + m) : -1;
+      if (pg < 0 || pg >= p.num_pages) {
+        set_status(p.status, SAS_DEV_ERR_BOUNDS);
+        att[k] = -1;
+      } else {
+        zz = pg * p.Hkv + g;
+      }
     }
-    return H;
+    z[k] = zz;
   }
-  int take_eq = 0;
-  tk = radix_select_keys(keys, c, H, nullptr, &take_eq);
-  tidx = tie_index_keys(keys, c, tk, take_eq);
-  int pos = 0;
-#pragma unroll
-  for (int i = 0; i < KREG; ++i) {
-    if (32 * i >= c) break;
-    const int m = lane + 32 * i;
-    const bool take = m < c && (keys[i] > tk || (keys[i] == tk && m <= tidx));
-    const uint32_t bal = __ballot_sync(0xffffffffu, take);
-    if (take) {
-      const int lp = pos + __popc(bal & ((1u << lane) - 1u));
-      att[1 + lp] = m;
-      if (so) so[lp] = m;
-    }
-    pos += __popc(bal);
-  }
-  return pos;
 }
 
 // Selected blocks of one score row (c historical blocks, mode as below) as the
@@ -230,6 +287,291 @@ __global__ void __launch_bounds__(32) decode_select_kernel(const Params p) {
     const float lse = row_lse(srow, c);
     if (lane == 0) p.lse_gate[bg] = lse;
   }
+  if (p.page_table) map_pages(p, bg, att);
+}
+
+constexpr int kLongWarps = 16;   // warps of the long-row selection CTA
+
+// Rows longer than 32 * kSelectReg blocks, any budget: one CTA of kRadixThreads
+// threads per (b, g), the row in registers (block m = t + kRadixThreads * i on
+// thread t). First a lower bound of the H-th largest key from the warps' four
+// largest thread maxima (64 keys of distinct threads): the lesser of the
+// ceil(H/2)-th largest of warps 0-7's and of warps 8-15's, so that at least H
+// keys of the row are at or above it (0 when some warp holds fewer than four
+// keys, which filters nothing). The keys at or above the
+// bound are the candidates. When at most kMaxCand of them remain (the usual
+// case), each candidate's rank under (key descending, block ascending) is
+// counted directly, and the H best are placed by how many taken blocks precede
+// them. Otherwise (many keys tied at the bound) an MSB-first radix select over
+// shared-memory histograms of the candidates (digits of 11, 11 and 10 bits) finds
+// the H-th largest key and how many keys equal to it are taken (the first ones in
+// block order), and a scan of the per-(row, warp) counts of larger and of equal
+// keys gives each selected block its rank. Either way the list comes out in
+// ascending block order.
+constexpr int kRadixThreads = 32 * kLongWarps;
+constexpr int kRadixBins = 2048;
+static_assert(kRadixBins == 4 * kRadixThreads, "each thread owns four histogram bins");
+constexpr int kMaxCand = kRadixThreads;   // candidates ranked by counting (one to four threads each)
+
+template <int KR>
+__global__ void __launch_bounds__(kRadixThreads) decode_select_radix_kernel(const Params p) {
+  __shared__ uint32_t hist[2][kRadixBins];
+  __shared__ uint32_t cnt[KR][kLongWarps];   // (larger << 16 | equal) per (row, warp), then exclusive prefixes
+  __shared__ int wsum[kLongWarps];
+  __shared__ float red[kLongWarps];
+  __shared__ uint32_t wtop[4 * kLongWarps];  // per warp: its four largest thread maxima (bound of the select)
+  __shared__ uint2 cand[kMaxCand];           // (key, block) of the keys at or above the bound
+  __shared__ int taken_flag[kMaxCand];
+  __shared__ uint32_t sh_digit, sh_bound;
+  __shared__ int sh_rem, n_cand;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bg = blockIdx.x;
+  griddep_launch_dependents();   // the attention kernel may start its prologue
+  const float* srow = p.s + (long long)bg * p.NBmax;
+  float sv[KR];
+#pragma unroll
+  for (int i = 0; i < KR; ++i) {
+    const int m = tid + kRadixThreads * i;
+    sv[i] = (m < p.NBmax) ? __ldg(srow + m) : 0.f;
+  }
+  if (p.page_table) {
+    // The sequence's page-table row toward L2 (its Hkv CTAs take a share each), so
+    // that the lookups of the selected blocks at the end are L2 hits.
+    const int b0 = bg / p.Hkv, g0 = bg % p.Hkv;
+    const int lines = (p.max_pages + 31) / 32;   // 128-byte lines of the row
+    const int32_t* row = p.page_table + (long long)b0 * p.max_pages;
+    for (int l = g0 + p.Hkv * tid; l < lines; l += p.Hkv * kRadixThreads)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(row + min(32 * l, p.max_pages - 1)));
+  }
+  const int b = bg / p.Hkv;
+  const int L = p.seqlen[b];
+  int32_t* att = p.att + (long long)bg * p.K;
+  if (tid == 0) {
+    p.tickets[bg] = 0;
+    if (bg == 0) *p.work = 0;
+  }
+  if (L < 1 || L > p.Lmax) {   // a sequence length outside the cache: nothing attended
+    if (tid == 0) set_status(p.status, SAS_DEV_ERR_BOUNDS);
+    for (int k = tid; k < p.K; k += kRadixThreads) att[k] = -1;
+    return;
+  }
+  const int c = (L - 1) / kBlock;
+  const int H = p.K - 1;
+  int32_t* so = p.sel_out ? p.sel_out + (long long)bg * H : nullptr;
+  if (tid == 0) att[0] = c;
+  if (p.apply_log_gate) {   // log sum_{m < c} exp(s[m]) over the whole CTA
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < KR; ++i)
+      if (tid + kRadixThreads * i < c) mx = fmaxf(mx, sv[i]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kLongWarps; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < KR; ++i)
+      if (tid + kRadixThreads * i < c) sum += expf(sv[i] - M);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) red[warp] = sum;
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < kLongWarps; ++w) tot += red[w];
+      p.lse_gate[bg] = (c > 0) ? M + logf(tot) : 0.f;
+    }
+  }
+  if (c > H && H > 0) {
+    uint32_t keys[KR];
+#pragma unroll
+    for (int i = 0; i < KR; ++i) keys[i] = (tid + kRadixThreads * i < c) ? float_key(sv[i]) : 0u;
+    // Lower bound of the H-th largest key (0, no filtering, when some warp holds too few keys).
+    uint32_t tmax = 0u;
+#pragma unroll
+    for (int i = 0; i < KR; ++i) tmax = max(tmax, keys[i]);
+    const uint32_t srt = warp_sort_desc(tmax);   // lane j: the warp's j-th largest thread maximum
+    if (lane < 4) wtop[4 * warp + lane] = srt;
+    if (tid == 0) n_cand = 0;
+    __syncthreads();
+    if (warp == 0) {
+      // Warps 0-7's and warps 8-15's 32 values, each sorted: the k-th largest of
+      // each half has k keys of its half at or above it, so the lesser of the two
+      // has 2k >= H keys at or above it.
+      const uint32_t ha = warp_sort_desc(wtop[lane]);
+      const uint32_t hb = warp_sort_desc(wtop[lane + 32]);
+      const int k = (H + 1) / 2;   // 1..32
+      const uint32_t bnd = min(__shfl_sync(0xffffffffu, ha, k - 1), __shfl_sync(0xffffffffu, hb, k - 1));
+      if (lane == 0) sh_bound = bnd;
+    }
+    __syncthreads();
+    const uint32_t bound = sh_bound;
+    // The keys at or above the bound (the Top-H among them) go to a shared list.
+#pragma unroll
+    for (int i = 0; i < KR; ++i) {
+      const int m = tid + kRadixThreads * i;
+      if (m < c && keys[i] >= bound) {
+        const int slot = atomicAdd(&n_cand, 1);
+        if (slot < kMaxCand) cand[slot] = make_uint2(keys[i], (uint32_t)m);
+      }
+    }
+    __syncthreads();
+    const int n = n_cand;
+    if (n <= kMaxCand) {
+      // Few candidates: each one's rank under (key descending, block ascending) by
+      // counting (tpc threads per candidate); the H best are taken and placed by how
+      // many taken blocks precede them.
+      const int tpc = n <= kRadixThreads / 4 ? 4 : (n <= kRadixThreads / 2 ? 2 : 1);
+      const int j = tid / tpc, q = tid % tpc;
+      const bool mine = j < n;
+      const uint2 cj = mine ? cand[j] : make_uint2(0u, 0u);
+      const uint64_t vj = ((uint64_t)cj.x << 32) | (uint64_t)(0xFFFFFFFFu - cj.y);
+      int r = 0;
+      if (mine)
+        for (int i = q; i < n; i += tpc) {
+          const uint2 ci = cand[i];
+          r += (((uint64_t)ci.x << 32) | (uint64_t)(0xFFFFFFFFu - ci.y)) > vj ? 1 : 0;
+        }
+      for (int o = 1; o < tpc; o <<= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+      const bool taken = mine && r < H;
+      if (mine && q == 0) taken_flag[j] = taken ? 1 : 0;
+      __syncthreads();
+      int pc = 0;
+      if (taken)
+        for (int i = q; i < n; i += tpc) pc += (taken_flag[i] && cand[i].y < cj.y) ? 1 : 0;
+      for (int o = 1; o < tpc; o <<= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
+      if (taken && q == 0) {
+        att[1 + pc] = (int32_t)cj.y;
+        if (so) so[pc] = (int32_t)cj.y;
+      }
+    } else {
+      // Many keys at the bound (ties): radix select over the keys at or above it.
+      for (int jb = tid; jb < kRadixBins; jb += kRadixThreads) hist[0][jb] = 0u;
+      __syncthreads();
+      uint32_t prefix = 0u;
+      int remaining = H;
+#pragma unroll 1
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const uint32_t hi_mask = pass == 0 ? 0u : (pass == 1 ? 0xFFE00000u : 0xFFFFFC00u);
+        const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
+        uint32_t* h = hist[pass & 1];
+        if (pass < 2)   // the other histogram, for the next pass (its last reader passed a barrier since)
+          for (int jb = tid; jb < kRadixBins; jb += kRadixThreads) hist[(pass + 1) & 1][jb] = 0u;
+#pragma unroll
+        for (int i = 0; i < KR; ++i)
+          if (tid + kRadixThreads * i < c && keys[i] >= bound && (keys[i] & hi_mask) == prefix)
+            atomicAdd(&h[(keys[i] >> shift) & dmask], 1u);
+        __syncthreads();
+        // Thread t owns bins 2047-4t .. 2044-4t (descending); a block-wide exclusive
+        // scan of the owned counts finds the bin holding the remaining-th largest key.
+        int b4[4];
+        int loc = 0;
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb) {
+          b4[jb] = (int)h[kRadixBins - 1 - 4 * tid - jb];
+          loc += b4[jb];
+        }
+        int incl = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int before = incl - loc;
+#pragma unroll
+        for (int w = 0; w < kLongWarps; ++w) before += (w < warp) ? wsum[w] : 0;
+        if (before < remaining && remaining <= before + loc) {
+          int run = before;
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) {
+            if (run + b4[jb] >= remaining) {
+              sh_digit = (uint32_t)(kRadixBins - 1 - 4 * tid - jb);
+              sh_rem = remaining - run;
+              break;
+            }
+            run += b4[jb];
+          }
+        }
+        __syncthreads();
+        prefix |= sh_digit << shift;
+        remaining = sh_rem;
+      }
+      const uint32_t tkey = prefix;
+      const int take_eq = remaining;
+      const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+      for (int i = 0; i < KR; ++i) {
+        const bool in = tid + kRadixThreads * i < c;
+        const uint32_t bgt = __ballot_sync(0xffffffffu, in && keys[i] > tkey);
+        const uint32_t beq = __ballot_sync(0xffffffffu, in && keys[i] == tkey);
+        if (lane == 0) cnt[i][warp] = ((uint32_t)__popc(bgt) << 16) | (uint32_t)__popc(beq);
+      }
+      __syncthreads();
+      if (warp == 0) {   // exclusive scan over (row, warp) in row-major order = ascending block order
+        constexpr int E = KR * kLongWarps;
+        constexpr int PER = (E + 31) / 32;
+        uint32_t* flat = &cnt[0][0];
+        uint32_t v[PER];
+        uint32_t lsum = 0u;
+#pragma unroll
+        for (int jb = 0; jb < PER; ++jb) {
+          const int e = lane * PER + jb;
+          v[jb] = (e < E) ? flat[e] : 0u;
+          lsum += v[jb];
+        }
+        uint32_t incl = lsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        uint32_t run = incl - lsum;
+#pragma unroll
+        for (int jb = 0; jb < PER; ++jb) {
+          const int e = lane * PER + jb;
+          if (e < E) flat[e] = run;
+          run += v[jb];
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < KR; ++i) {
+        const int m = tid + kRadixThreads * i;
+        const bool in = m < c;
+        const bool gt = in && keys[i] > tkey, eq = in && keys[i] == tkey;
+        const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
+        const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+        const uint32_t base = cnt[i][warp];
+        const int gt_before = (int)(base >> 16) + __popc(bgt & lt);
+        const int eq_before = (int)(base & 0xFFFFu) + __popc(beq & lt);
+        if (gt || (eq && eq_before < take_eq)) {
+          const int pos = gt_before + min(eq_before, take_eq);
+          att[1 + pos] = m;
+          if (so) so[pos] = m;
+        }
+      }
+    }
+  } else if (warp == 0) {   // nothing to choose: every historical block (c <= H), or none (H == 0)
+    const int n = min(c, H);
+    for (int m = lane; m < n; m += 32) {
+      att[1 + m] = m;
+      if (so) so[m] = m;
+    }
+    for (int k = 1 + n + lane; k < p.K; k += 32) att[k] = -1;
+    if (so)
+      for (int k = n + lane; k < H; k += 32) so[k] = -1;
+  }
+  if (p.page_table) {
+    __syncthreads();   // every warp wrote part of the list
+    if (warp == 0) map_pages(p, bg, att);
+  }
 }
 
 // ---------------------------------------------------------------------------- attention
@@ -334,69 +676,89 @@ __device__ __forceinline__ void merge_partials(const Params& p, int bg, float* s
   }
 }
 
-// Merges each (b, g) listed in grp[0..n) (n_slots partials apiece) into o with one L2
-// round trip per batch of 16 partials: every thread loads the (max, sum) pairs of
-// its head together with the partial outputs of its 4 features and combines them
-// in registers (an online rescale between batches when there are more than 16).
-template <int NT>
-__device__ __forceinline__ void merge_groups(const Params& p, const int* grp, int n) {
+// Merges each (b, g)'s partials (n_slots apiece) into o: one CTA per (b, g),
+// launched as a programmatic dependent of the bf16 attention kernel. S adjacent
+// threads share one float4 of o, each folding up to 16 slots (one batch of loads
+// in flight), and combine their (max, sum, output) states by shuffles.
+template <int S>
+__host__ __device__ constexpr int merge_threads() {
+  return S >= 4 ? 256 : 128 * S;   // up to 16 float4 + 16 float2 loads in flight per thread
+}
+
+template <int S>
+__global__ void __launch_bounds__(merge_threads<S>()) decode_merge_kernel(const Params p) {
+  constexpr int kGroups = merge_threads<S>() / S;   // float4s of o per pass
+  griddep_wait();   // the attention kernel's partials are complete and visible
+  const int bg = blockIdx.x;
   const int G = p.G, K = p.n_slots;
   const int per = G * (D / 4);
-  for (int idx = threadIdx.x; idx < n * per; idx += (NT > 0 ? NT : (int)blockDim.x)) {
-    const int bg = grp[idx / per], r = idx % per, h = r / (D / 4), d4 = r % (D / 4);
-    const int b = bg / p.Hkv, g = bg % p.Hkv;
-    const float2* pml = reinterpret_cast<const float2*>(p.part_ml) + (long long)bg * K * G + h;
-    const float4* pob = reinterpret_cast<const float4*>(p.part_o) + ((long long)bg * K * G + h) * (D / 4) + d4;
+  const int sg = threadIdx.x % S;
+  const int k_begin = 16 * sg, k_end = min(K, 16 * sg + 16);
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  for (int base = 0; base < per; base += kGroups) {   // every lane runs every pass (the shuffles)
+    const int idx = base + (int)threadIdx.x / S;
+    const bool active = idx < per;
+    const int h = idx / (D / 4), d4 = idx % (D / 4);
     float M = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k0 = 0; k0 < K; k0 += 16) {
+    if (active && k_begin < k_end) {
+      const float2* pml = reinterpret_cast<const float2*>(p.part_ml) + (long long)bg * K * G + h;
+      const float4* pob = reinterpret_cast<const float4*>(p.part_o) + ((long long)bg * K * G + h) * (D / 4) + d4;
       float2 ml[16];
       float4 u[16];
 #pragma unroll
       for (int kk = 0; kk < 16; ++kk) {
-        if (k0 + kk < K) {
-          ml[kk] = __ldcg(pml + (k0 + kk) * G);
-          u[kk] = __ldcg(pob + (long long)(k0 + kk) * G * (D / 4));
+        if (k_begin + kk < k_end) {
+          ml[kk] = __ldcg(pml + (k_begin + kk) * G);
+          u[kk] = __ldcg(pob + (long long)(k_begin + kk) * G * (D / 4));
         } else {
           ml[kk] = make_float2(-INFINITY, 0.f);
         }
       }
-      float Mb = M;
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) Mb = fmaxf(Mb, ml[kk].x);
-      if (Mb == -INFINITY) continue;
-      const float a = (M == -INFINITY) ? 0.f : ex2((M - Mb) * kLog2e);
-      den *= a;
-      num.x *= a, num.y *= a, num.z *= a, num.w *= a;
+      for (int kk = 0; kk < 16; ++kk) M = fmaxf(M, ml[kk].x);
+      if (M != -INFINITY) {
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) {
-        // Empty slots (max -inf) were never written: weight zero, bits unused.
-        if (ml[kk].x != -INFINITY) {
-          const float w = ex2((ml[kk].x - Mb) * kLog2e);
-          den = fmaf(w, ml[kk].y, den);
-          num.x = fmaf(w, u[kk].x, num.x);
-          num.y = fmaf(w, u[kk].y, num.y);
-          num.z = fmaf(w, u[kk].z, num.z);
-          num.w = fmaf(w, u[kk].w, num.w);
+        for (int kk = 0; kk < 16; ++kk) {
+          // Empty slots (max -inf) were never written: weight zero, bits unused.
+          if (ml[kk].x != -INFINITY) {
+            const float w = ex2((ml[kk].x - M) * kLog2e);
+            den = fmaf(w, ml[kk].y, den);
+            num.x = fmaf(w, u[kk].x, num.x);
+            num.y = fmaf(w, u[kk].y, num.y);
+            num.z = fmaf(w, u[kk].z, num.z);
+            num.w = fmaf(w, u[kk].w, num.w);
+          }
         }
       }
-      M = Mb;
     }
-    const float s = 1.f / den;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.o) +
-                                                            ((long long)b * p.Hq + g * G + h) * D + d4 * 4);
-    dst[0] = __floats2bfloat162_rn(num.x * s, num.y * s);
-    dst[1] = __floats2bfloat162_rn(num.z * s, num.w * s);
+#pragma unroll
+    for (int o = 1; o < S; o <<= 1) {
+      const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
+      const float deno = __shfl_xor_sync(0xffffffffu, den, o);
+      float4 nu;
+      nu.x = __shfl_xor_sync(0xffffffffu, num.x, o);
+      nu.y = __shfl_xor_sync(0xffffffffu, num.y, o);
+      nu.z = __shfl_xor_sync(0xffffffffu, num.z, o);
+      nu.w = __shfl_xor_sync(0xffffffffu, num.w, o);
+      const float Mn = fmaxf(M, Mo);
+      const float a = (M == -INFINITY) ? 0.f : ex2((M - Mn) * kLog2e);
+      const float ao = (Mo == -INFINITY) ? 0.f : ex2((Mo - Mn) * kLog2e);
+      den = den * a + deno * ao;
+      num.x = num.x * a + nu.x * ao;
+      num.y = num.y * a + nu.y * ao;
+      num.z = num.z * a + nu.z * ao;
+      num.w = num.w * a + nu.w * ao;
+      M = Mn;
+    }
+    if (active && sg == 0) {
+      const float sc = 1.f / den;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.o) +
+                                                              ((long long)b * p.Hq + g * G + h) * D + d4 * 4);
+      dst[0] = __floats2bfloat162_rn(num.x * sc, num.y * sc);
+      dst[1] = __floats2bfloat162_rn(num.z * sc, num.w * sc);
+    }
   }
-}
-
-// Merges each (b, g)'s partials (n_slots apiece) into o: one 128-thread CTA per
-// (b, g) (a float4 of o per thread and pass), launched as a programmatic dependent
-// of the bf16 attention kernel.
-__global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
-  griddep_wait();   // the attention kernel's partials are complete and visible
-  const int grp = blockIdx.x;
-  merge_groups<0>(p, &grp, 1);
 }
 
 // One CTA per work item (b, g, attended block). Lane layout inside a warp: the
@@ -652,14 +1014,15 @@ constexpr uint32_t kStageBytes = 2 * kMmaTileBytes;
 // Shared memory of the fused kernel for G heads per group and budget K.
 constexpr int kMaxItemsPerCta = 63;            // bounds the per-CTA item and group lists
 struct FusedLayout {
-  uint32_t q, zero, att, grp, comb, bar, total;
+  uint32_t q, zero, att, attz, grp, comb, bar, total;
 };
 __host__ __device__ inline FusedLayout fused_layout(int G, int K) {
   FusedLayout l;
   l.q = kDecStages * kStageBytes;        // 4 q slots of G rows x 256 bytes
   l.zero = l.q + 4u * G * 256u;          // one zero row (q rows G..15 of the MMA)
   l.att = l.zero + 256u;                 // attended block of each of the CTA's items
-  l.grp = l.att + 256u;                  // per (b, g) of the CTA: sequence length, log-gate LSE
+  l.attz = l.att + 256u;                 // its plane in a paged cache
+  l.grp = l.attz + 256u;                 // per (b, g) of the CTA: sequence length, log-gate LSE
   l.comb = l.grp + 2u * 256u;            // [warps][16 rows] (max, sum)
   l.bar = l.comb + kDecWarps * 16 * 2 * 4;
   l.total = l.bar + 128u;                // full/empty barriers, stage blocks, copies in flight
@@ -694,6 +1057,7 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
   uint8_t* qring = smem + lay.q;
   uint8_t* zrow = smem + lay.zero;
   int32_t* att_s = reinterpret_cast<int32_t*>(smem + lay.att);
+  int32_t* attz_s = reinterpret_cast<int32_t*>(smem + lay.attz);
   int32_t* grp_L = reinterpret_cast<int32_t*>(smem + lay.grp);
   float* grp_lse = reinterpret_cast<float*>(smem + lay.grp + 256u);
   float* comb = reinterpret_cast<float*>(smem + lay.comb);
@@ -720,6 +1084,8 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
   // Everything below may read what the selection kernel wrote.
   griddep_wait();
   for (int i = tid; i < u1 - u0; i += 32 * kDecWarps) att_s[i] = p.att[u0 + i];
+  if (p.page_table)
+    for (int i = tid; i < u1 - u0; i += 32 * kDecWarps) attz_s[i] = p.att_z[u0 + i];
   if (p.apply_log_gate)
     for (int j = tid; j < n_grp; j += 32 * kDecWarps) grp_lse[j] = p.lse_gate[bg0 + j];
   __syncthreads();
@@ -744,11 +1110,14 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
           tma_load_2d(qring + ((bg - bg0) & 3) * G * 256, &tmq, &full[s], 0, b * p.Hq + g * G);
         }
         if (m >= 0) {
+          // Contiguous cache: plane bg, rows m*64..; paged: the block's own plane, rows 0..63.
+          const int z = p.page_table ? attz_s[pf - u0] : bg;
+          const int y = p.page_table ? 0 : m * kBlock;
           uint8_t* st = smem + s * kStageBytes;
-          tma_load_3d(st, &tmk, &full[s], 0, m * kBlock, bg);
-          tma_load_3d(st + 8192, &tmk, &full[s], 64, m * kBlock, bg);
-          tma_load_3d(st + kMmaTileBytes, &tmv, &full[s], 0, m * kBlock, bg);
-          tma_load_3d(st + kMmaTileBytes + 8192, &tmv, &full[s], 64, m * kBlock, bg);
+          tma_load_3d(st, &tmk, &full[s], 0, y, z);
+          tma_load_3d(st + 8192, &tmk, &full[s], 64, y, z);
+          tma_load_3d(st + kMmaTileBytes, &tmv, &full[s], 0, y, z);
+          tma_load_3d(st + kMmaTileBytes + 8192, &tmv, &full[s], 64, y, z);
         }
         issued[s] = pf - u0;
       } else {
@@ -992,6 +1361,7 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int K) {
   const size_t n_bg = (size_t)B * Hkv;
   size_t bytes = 256;                                      // status word
   bytes += a256(n_bg * K * sizeof(int32_t));               // attended lists
+  bytes += a256(n_bg * K * sizeof(int32_t));               // their planes in a paged cache
   bytes += a256(n_bg * sizeof(float));                     // log-gate LSE
   bytes += a256((n_bg + 1) * sizeof(int32_t));             // tickets, counter
   bytes += a256(n_bg * K * G * 2 * sizeof(float));         // partial max / sum
@@ -1016,6 +1386,11 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
   size_t off = 256;
   prm.att = reinterpret_cast<int32_t*>(w + off);
   off += a256(n_bg * pb.K * sizeof(int32_t));
+  prm.att_z = reinterpret_cast<int32_t*>(w + off);
+  off += a256(n_bg * pb.K * sizeof(int32_t));
+  prm.page_table = pb.page_table;
+  prm.max_pages = pb.max_pages;
+  prm.num_pages = pb.num_pages;
   prm.lse_gate = reinterpret_cast<float*>(w + off);
   off += a256(n_bg * sizeof(float));
   prm.tickets = reinterpret_cast<int32_t*>(w + off);
@@ -1047,7 +1422,16 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
     count_launch();
     return cudaGetLastError();
   };
+  auto select_long = [&](auto kernel) -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (r != cudaSuccess) return r;
+    kernel<<<(unsigned)n_bg, 32 * kLongWarps, 0, st>>>(prm);
+    count_launch();
+    return cudaGetLastError();
+  };
   // Registers per lane for the score row: the row is loaded before its length is known.
+  constexpr int kLongSlice = 32 * kLongWarps;   // blocks per CTA and register per lane
   if (pb.NBmax <= 128)
     e = select(decode_select_kernel<4>);
   else if (pb.NBmax <= 256)
@@ -1056,13 +1440,24 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
     e = select(decode_select_kernel<16>);
   else if (pb.NBmax <= 32 * kSelectReg)
     e = select(decode_select_kernel<kSelectReg>);
+  else if (pb.NBmax <= 4 * kLongSlice)
+    e = select_long(decode_select_radix_kernel<4>);
+  else if (pb.NBmax <= 8 * kLongSlice)
+    e = select_long(decode_select_radix_kernel<8>);
+  else if (pb.NBmax <= 16 * kLongSlice)
+    e = select_long(decode_select_radix_kernel<16>);
+  else if (pb.NBmax <= 32 * kLongSlice)
+    e = select_long(decode_select_radix_kernel<32>);
   else
     e = select(decode_select_kernel<0>);
   if (e != cudaSuccess) return e;
   if (pb.dtype == 1) {
     CUtensorMap tk, tv, tq;
-    if (!make_tmap_bf16_3d(&tk, pb.Kc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
-        !make_tmap_bf16_3d(&tv, pb.Vc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
+    // Contiguous cache: planes (b, g) of Lmax rows; paged: planes (page, g) of one block.
+    const uint64_t rows = pb.page_table ? (uint64_t)kBlock : (uint64_t)pb.Lmax;
+    const uint64_t planes = pb.page_table ? (uint64_t)pb.num_pages * pb.Hkv : (uint64_t)n_bg;
+    if (!make_tmap_bf16_3d(&tk, pb.Kc, D, rows, planes, kBlock) ||
+        !make_tmap_bf16_3d(&tv, pb.Vc, D, rows, planes, kBlock) ||
         !make_tmap_bf16_rows(&tq, pb.q, D, (uint64_t)pb.B * pb.Hq, (uint32_t)G))
       return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
@@ -1093,11 +1488,20 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
     e = cudaLaunchKernelEx(&cfg, decode_fused_mma_kernel, prm, tk, tv, tq, per_cta);
     if (e != cudaSuccess) return e;
     count_launch();
-    // The merge of every (b, g), as a programmatic dependent of the attention kernel.
+    // The merge of every (b, g), as a programmatic dependent of the attention kernel;
+    // S threads per float4 of o, each over at most 16 of the K slots.
     cfg.gridDim = dim3((unsigned)n_bg);
-    cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = 0;
-    e = cudaLaunchKernelEx(&cfg, decode_merge_kernel, prm);
+    if (pb.K <= 16) {
+      cfg.blockDim = dim3(merge_threads<1>());
+      e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<1>, prm);
+    } else if (pb.K <= 32) {
+      cfg.blockDim = dim3(merge_threads<2>());
+      e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<2>, prm);
+    } else {
+      cfg.blockDim = dim3(merge_threads<4>());
+      e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<4>, prm);
+    }
     if (e != cudaSuccess) return e;
     count_launch();
     return cudaGetLastError();

@@ -69,6 +69,8 @@ struct DecodeProblem {
   const float* s;
   void* o;
   int32_t* sel_out;
+  const int32_t* page_table = nullptr;   // [B][max_pages]; null: contiguous cache
+  int max_pages = 0, num_pages = 0;
 };
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int K);
 cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st);

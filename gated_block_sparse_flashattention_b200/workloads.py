@@ -65,12 +65,15 @@ WORKLOADS = {
     "qwen3_14b_t64k": Workload("qwen3_14b_t64k", "bf16", 1, 40, 8, 128, 65536, 16),
     # Memory-bound decode: 16 sequences, one new token each over a 32768-token cache.
     "decode_b16_l32k": Workload("decode_b16_l32k", "bf16", 16, 32, 8, 128, 32768, 16, decode=True),
+    # Long-context decode over a paged cache: 8 sequences, one new token each at 512K
+    # context, budget 2048 tokens (32 blocks, the current one included).
+    "decode_b8_l512k_paged": Workload("decode_b8_l512k_paged", "bf16", 8, 32, 8, 128, 524288, 32, decode=True),
 }
 
 
 def _selector_scores(gen, shape, dist: str, block: int):
     if dist == "normal":
-        return torch.randn(shape, generator=gen)
+        return torch.randn(shape, generator=gen, device=gen.device)
     if dist == "normal2_planted3":
         s = 2.0 * torch.randn(shape, generator=gen)
         B, Hkv, T, NB = shape
@@ -132,3 +135,48 @@ def make_decode_inputs(w: Workload, seed: int = 0, seqlen=None):
 def custom(name="custom", dtype="bf16", B=1, Hq=4, Hkv=1, d=64, T=256, K=3, block=64, s_dist="normal", decode=False):
     """A workload of arbitrary shape (tests and smoke use these)."""
     return Workload(name, dtype, B, Hq, Hkv, d, T, K, block, s_dist, decode)
+
+
+def make_paged_decode_inputs(w: Workload, seed: int = 0, seqlen=None, pool_pages=None, device="cpu"):
+    """Tensors for one decode step over a paged KV cache of one-block pages.
+
+    q [B,Hq,d], Kp/Vp [num_pages,Hkv,block,d] in the workload's dtype,
+    page_table [B,NB] int32, seqlen [B] int32, s [B,Hkv,NB] float32, all on
+    ``device`` (drawn there from one generator seeded once, in the order q, s,
+    page table, Kp, Vp). Without ``pool_pages`` every block a sequence reaches
+    gets a page of its own, the pages in a seeded random order among a few unused
+    ones; with ``pool_pages = P`` the pool holds P pages and each block names a
+    seeded random one of them (pages shared, as under prefix sharing), which keeps
+    long contexts small. Blocks past a sequence's end hold -1.
+    """
+    gen = torch.Generator(device=device).manual_seed(seed)
+    dt = w.torch_dtype
+    q = torch.randn(w.B, w.Hq, w.d, generator=gen, device=device).to(dt)
+    s = _selector_scores(gen, (w.B, w.Hkv, 1, w.NB), w.s_dist, w.block).reshape(w.B, w.Hkv, w.NB).float()
+    if seqlen is None:
+        seqlen = [w.T] * w.B
+    seqlen = torch.as_tensor(seqlen, dtype=torch.int32)
+    n_blocks = [(int(L) + w.block - 1) // w.block for L in seqlen]
+    table = torch.full((w.B, w.NB), -1, dtype=torch.int32)
+    if pool_pages is None:
+        used = sum(n_blocks)
+        num_pages = used + max(4, used // 16)
+        perm = torch.randperm(num_pages, generator=gen, device=device).to(torch.int32).cpu()
+        off = 0
+        for b, n in enumerate(n_blocks):
+            table[b, :n] = perm[off:off + n]
+            off += n
+    else:
+        num_pages = pool_pages
+        pages = torch.randint(0, pool_pages, (w.B, w.NB), generator=gen, device=device).to(torch.int32).cpu()
+        for b, n in enumerate(n_blocks):
+            table[b, :n] = pages[b, :n]
+    pools = []
+    for _ in range(2):
+        pool = torch.empty(num_pages, w.Hkv, w.block, w.d, dtype=dt, device=device)
+        for p0 in range(0, num_pages, 4096):   # bounded fp32 temporaries
+            p1 = min(num_pages, p0 + 4096)
+            pool[p0:p1] = torch.randn(p1 - p0, w.Hkv, w.block, w.d, generator=gen, device=device).to(dt)
+        pools.append(pool)
+    return {"q": q, "Kp": pools[0], "Vp": pools[1], "page_table": table.to(device), "seqlen": seqlen.to(device),
+            "s": s}

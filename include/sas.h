@@ -198,6 +198,27 @@ SAS_API int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dt
                    int d, int block, float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * sas_decode_fwd_paged - sas_decode_fwd over a paged KV cache (SAS paper §5.1
+ * "Inference implementation": a paged cache, only the selected KV blocks
+ * gathered). The computation is that of sas_decode_fwd on the logical cache in
+ * which token p of sequence b is row p % 64 of page page_table[b, p / 64].
+ * Kp/Vp [num_pages, Hkv, 64, d] bf16: one page holds one 64-token block of every
+ * KV head (the head's 64 rows contiguous). page_table [B, max_pages] int32
+ * DEVICE; entries of blocks 0..(seqlen[b]-1)/64 must lie in 0..num_pages-1 (an
+ * entry outside is reported as a device-side bounds error and its block is
+ * skipped); entries past a sequence's last block are never read. Pages may be
+ * shared between sequences. seqlen [B] int32 DEVICE, 1 <= L <= max_pages * 64.
+ * s [B,Hkv,NBmax] fp32 with NBmax >= max_pages. Other arguments, the workspace
+ * (sas_decode_workspace_size with Lmax = max_pages * 64) and errors as for
+ * sas_decode_fwd; dtype must be SAS_DT_BF16 (fp32 returns SAS_ERR_UNSUPPORTED).
+ * Captures into a CUDA graph (no allocation, no host synchronisation).
+ */
+SAS_API int sas_decode_fwd_paged(const void* q, const void* Kp, const void* Vp, int dtype, const int32_t* page_table,
+                                 int max_pages, int num_pages, const int32_t* seqlen, const float* s, int K,
+                                 int apply_log_gate, void* o, int32_t* sel_out, int B, int Hq, int Hkv, int NBmax,
+                                 int d, int block, float sm_scale, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * sas_decode_fwd_static - sas_decode_fwd without a workspace argument. It has no
  * counterpart in the SAS paper; it exists for callers that cannot allocate device
  * memory themselves: a plugin whose host framework owns every device buffer and

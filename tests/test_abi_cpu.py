@@ -88,6 +88,13 @@ def test_invalid_calls_return_errors_without_launching(lib):
     assert lib.sas_gate_grad(fake, fake + 64, fake + 64, 1, 1, 128, 2, 64, None) == -1   # ds aliases dLogG
     assert lib.sas_gate_grad(fake, fake + 64, fake + 132, 1, 1, 128, 2, 64, None) == -1  # misaligned ds
     assert lib.sas_gate_grad(fake, fake + 64, fake + 128, 1, 1, 128, 2, 32, None) == -1  # block != 64
+    # paged decode: fp32 storage is not implemented; NBmax below max_pages is invalid
+    paged = [fake] * 3 + [binding.SAS_DT_F32, fake, 4, 8, fake, fake, 4, 0, fake, None, 1, 4, 1, 4, 128, 64,
+                          ctypes.c_float(0.1), fake, 1 << 20, None]
+    assert lib.sas_decode_fwd_paged(*paged) == -2
+    paged[3] = binding.SAS_DT_BF16
+    paged[16] = 3                 # NBmax < max_pages
+    assert lib.sas_decode_fwd_paged(*paged) == -1
     # sas_fwd: missing workspace / bad sizes
     args = [fake] * 3 + [binding.SAS_DT_BF16] + [fake] * 5 + [1, 4, 1, 128, 128, 64, ctypes.c_float(0.1), None, 0, None]
     assert lib.sas_fwd(*args) == -5
