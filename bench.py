@@ -41,7 +41,8 @@ from gated_block_sparse_flashattention_b200 import workloads  # noqa: E402
 # (sha256 prefixes); after any change they read as unmeasured (null).
 MEASURED_TRAFFIC = {
     "sas_bwd": (2478358784, {"sas_bwd_gather.cu": "f87675f7247ad878", "sas_common.cuh": "d3c29d493fc4dfcf"}),
-    "decode": (67342848, {"sas_decode.cu": "e1bfb301fe1a96f5", "sas_common.cuh": "d3c29d493fc4dfcf"}),
+    "decode": (67355136, {"sas_decode.cu": "4ebaf9cb8b725287", "sas_common.cuh": "d3c29d493fc4dfcf"}),
+    "decode_paged": (68085760, {"sas_decode.cu": "4ebaf9cb8b725287", "sas_common.cuh": "d3c29d493fc4dfcf"}),
 }
 
 
@@ -568,7 +569,7 @@ def run_decode_paged(args, device, stream, binding, peaks, clk=None):
                         f"each, {pool_gb:.1f} GB K/V pool), Hq=32 Hkv=8 d=128 K=32",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": nbytes, "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
-            "traffic": None, "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
+            "traffic": measured_traffic("decode_paged"), "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
             "launches_per_step": per_call, "device_status": binding.sas_device_status(ws),
             "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
 
