@@ -168,6 +168,44 @@ def selection_mask(logG, tau, tau_idx, block: int):
 
 
 # --------------------------------------------------------------------------------------
+# The "full*" training scope of SAS paper §4.1 (Table 1, row 11): noise is added to the
+# selector scores before Top-K, so the attended set is the Top-K of the noisy scores
+# while the gates of the attended blocks stay those of the clean scores.
+# --------------------------------------------------------------------------------------
+def select_noisy(logG32, noise32, K: int, block: int):
+    """Top-(K-1) of the noisy keys ``logG + noise`` and the gate tensor restricted to it.
+
+    logG32, noise32: float32 [B, Hkv, T, NB]. The keys are formed in float32 (the
+    sum decides an index, so it is taken in the kernel's precision); adding noise
+    to s or to logG = s - LSE(s) ranks the blocks of a row alike. Returns
+    ``logG_sel`` (float64: logG on the chosen blocks, -inf elsewhere), ``tau`` and
+    ``tau_idx`` (the threshold of ``logG_sel``, which the attention calls use to
+    find the chosen blocks again) and ``sel`` (ascending chosen blocks, -1 padded).
+    """
+    lg = np.asarray(logG32, dtype=np.float32)
+    keys = (lg + np.asarray(noise32, dtype=np.float32)).astype(np.float32)
+    B, Hkv, T, NB = lg.shape
+    H = K - 1
+    logG_sel = np.full((B, Hkv, T, NB), -np.inf)
+    tau = np.zeros((B, Hkv, T))
+    tidx = np.zeros((B, Hkv, T), dtype=np.int32)
+    sel = np.full((B, Hkv, T, max(H, 0)), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(T):
+                c = min(t // block, NB)
+                _, _, chosen = topk_threshold_row(keys[b, g, t].astype(np.float64), c, H)
+                for m in chosen:
+                    logG_sel[b, g, t, m] = float(lg[b, g, t, m])
+                tv, ti, again = topk_threshold_row(logG_sel[b, g, t], c, H)
+                assert again == chosen
+                tau[b, g, t] = tv
+                tidx[b, g, t] = ti
+                sel[b, g, t, : len(chosen)] = chosen
+    return logG_sel, tau, tidx, sel
+
+
+# --------------------------------------------------------------------------------------
 # The biased logit matrix of SAS paper §4.3 eq. 9:
 #   softmax(q K_S^T + log g_S) V_S,  S = B_0 ∪ (selected historical blocks),
 # written as a dense [rows, T] bias: 0 on the causal part of the current block,

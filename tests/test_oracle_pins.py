@@ -556,3 +556,67 @@ def test_paged_pin_catches_planted_mistake(monkeypatch):
     monkeypatch.setattr(orc, "paged_cache", _bad_paged_cache)
     with pytest.raises(AssertionError):
         test_paged_decode_equals_contiguous_decode_under_a_page_shuffle()
+
+
+# ---------------------------------------------------------------- noisy (full*) selection
+def test_select_noisy_without_noise_is_the_plain_selection():
+    rng = np.random.default_rng(31)
+    B, Hkv, T, NB, block, K = 1, 2, 320, 5, 64, 3
+    logG32 = orc.gate_normalize(rng.standard_normal((B, Hkv, T, NB)), block).astype(np.float32)
+    logG_sel, tau, tidx, sel = orc.select_noisy(logG32, np.zeros_like(logG32), K, block)
+    t2, i2, s2 = orc.select_threshold(logG32.astype(np.float64), K, block)
+    assert np.array_equal(tau, t2) and np.array_equal(tidx, i2) and np.array_equal(sel, s2)
+    mask = orc.selection_mask(logG32, t2, i2, block)
+    assert np.array_equal(logG_sel, np.where(mask, logG32.astype(np.float64), -np.inf))
+
+
+def test_select_noisy_brute_force_and_predicate():
+    """Tiny rows with integer-valued keys (many ties): the chosen set is the first H blocks under
+    (key descending, block ascending) by brute force over all subsets, and the threshold of logG_sel
+    picks exactly that set again."""
+    rng = np.random.default_rng(32)
+    B, Hkv, T, NB, block, K = 1, 1, 8 * 4, 7, 4, 4
+    logG32 = rng.integers(-3, 3, size=(B, Hkv, T, NB)).astype(np.float32)
+    noise32 = rng.integers(-2, 3, size=(B, Hkv, T, NB)).astype(np.float32)
+    logG_sel, tau, tidx, sel = orc.select_noisy(logG32, noise32, K, block)
+    keys = logG32 + noise32
+    mask = orc.selection_mask(logG_sel, tau, tidx, block)
+    for t in range(T):
+        c = min(t // block, NB)
+        want = _brute_force_topk(keys[0, 0, t].astype(np.float64), c, K - 1)
+        assert [m for m in sel[0, 0, t] if m >= 0] == want
+        assert sorted(np.nonzero(mask[0, 0, t])[0].tolist()) == want
+        for m in range(NB):
+            expect = float(logG32[0, 0, t, m]) if m in want else -np.inf
+            assert logG_sel[0, 0, t, m] == expect
+
+
+def test_select_noisy_planted_noise_wins_and_keys_are_fp32():
+    B, Hkv, NB, block, K = 1, 1, 6, 2, 4
+    T = block * (NB + 1)
+    logG32 = np.tile(np.linspace(0.0, -5.0, NB, dtype=np.float32), (B, Hkv, T, 1))
+    noise32 = np.zeros_like(logG32)
+    noise32[..., [1, 3, 5]] = 100.0            # the three lowest gates but the largest keys
+    _, _, _, sel = orc.select_noisy(logG32, noise32, K, block)
+    assert sel[0, 0, T - 1].tolist() == [1, 3, 5]
+    # keys formed in float32: 1 + 2^-24 rounds to 1, a tie that goes to the lower block
+    lg = np.ones((1, 1, 3 * block, 2), np.float32)     # last row: c = 2 historical blocks, H = 1
+    nz = np.zeros_like(lg)
+    nz[..., 1] = 2.0 ** -24
+    assert np.float64(1.0) + 2.0 ** -24 > 1.0          # in float64 block 1 would win
+    _, _, _, sel = orc.select_noisy(lg, nz, 2, block)
+    assert sel[0, 0, 3 * block - 1, 0] == 0
+
+
+def _bad_select_noisy(logG32, noise32, K, block):
+    """Mistake: the noise ignored (the clean Top-K)."""
+    return _real_select_noisy(logG32, np.zeros_like(np.asarray(logG32, np.float32)), K, block)
+
+
+_real_select_noisy = orc.select_noisy
+
+
+def test_select_noisy_pin_catches_planted_mistake(monkeypatch):
+    monkeypatch.setattr(orc, "select_noisy", _bad_select_noisy)
+    with pytest.raises(AssertionError):
+        test_select_noisy_planted_noise_wins_and_keys_are_fp32()
