@@ -128,6 +128,35 @@ def gate_grad_bytes(w) -> float:
     return rows * (4.0 * c.sum() * 2 + 4.0 * w.NB * w.T)
 
 
+def noisy_select_bytes(w) -> float:
+    """HBM bytes of the noisy (full*) selection: the causal parts of logG and of the noise read, the full
+    logG_sel row written, tau and tau_idx written."""
+    c = np.minimum(np.arange(w.T) // w.block, w.NB).astype(np.float64)
+    rows = w.B * w.Hkv
+    return rows * (4.0 * c.sum() * 2 + 4.0 * w.NB * w.T + 8.0 * w.T)
+
+
+def time_noisy_select(w, logG, flush, stream, binding, device, reps=10):
+    """Mean device time (ms) of sas_select_noisy on the step's gates with seeded N(0, 1) noise, L2 flushed
+    before each call (outside the events). Not part of the step: the full* scope replaces the plain
+    selection with it."""
+    gen = torch.Generator(device=device).manual_seed(7)
+    noise = torch.randn(logG.shape, generator=gen, device=device)
+    lsel = torch.empty_like(logG)
+    tau = torch.empty(logG.shape[:3], device=device)
+    tidx = torch.empty(logG.shape[:3], dtype=torch.int32, device=device)
+    times = []
+    for i in range(reps + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        binding.sas_select_noisy(logG, noise, lsel, tau, tidx, None, w.K, stream=stream)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize(device)
+    return statistics.mean(a.elapsed_time(b) for a, b in times[3:])
+
+
 def decode_bytes(w) -> float:
     """Algorithmic bytes of one decode step: selected K/V blocks, q, o and the score rows."""
     el = 2 if w.dtype == "bf16" else 4
@@ -378,6 +407,7 @@ def run_gpu(args):
         torch.cuda.synchronize(device)
         ex_fwd, ex_bwd = executed_flops(w, sel)
         del sel
+        noisy_ms = time_noisy_select(w, logG, flush, stream, binding, device)
         gate_avg = statistics.mean(gate_ms)
         grad_avg = statistics.mean(grad_ms)
         roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
@@ -394,7 +424,9 @@ def run_gpu(args):
                     "gate_select_ms": round(gate_avg, 4),
                     "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1),
                     "gate_grad_ms": round(grad_avg, 4),
-                    "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1)}
+                    "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1),
+                    "noisy_select_ms": round(noisy_ms, 4),
+                    "noisy_select_gbs": round(noisy_select_bytes(w) / (noisy_ms * 1e-3) / 1e9, 1)}
     else:
         value, ms_per_step, launches, roofline = None, None, 0, None
 

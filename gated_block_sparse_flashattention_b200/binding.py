@@ -33,6 +33,7 @@ _SIGNATURES = {
     "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_normalize_select": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _vp]),
+    "sas_select_noisy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_grad": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_fwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
     "sas_bwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
@@ -128,6 +129,13 @@ def sas_gate_normalize_select(s, logG, tau, tau_idx, sel, K, block=BLOCK, stream
     B, Hkv, T, NB = s.shape
     _check("sas_gate_normalize_select", lib().sas_gate_normalize_select(
         _ptr(s), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
+
+
+def sas_select_noisy(logG, noise, logG_sel, tau, tau_idx, sel, K, block=BLOCK, stream=None):
+    B, Hkv, T, NB = logG.shape
+    _check("sas_select_noisy", lib().sas_select_noisy(
+        _ptr(logG), _ptr(noise), _ptr(logG_sel), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K,
+        _stream(stream)))
 
 
 def sas_gate_grad(logG, dLogG, ds, block=BLOCK, stream=None):

@@ -110,6 +110,20 @@ int sas_gate_normalize_select(const float* s, float* logG, float* tau, int32_t* 
       launch_normalize_select(s, logG, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB, K - 1, as_stream(stream)));
 }
 
+int sas_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
+                     int32_t* sel, int B, int Hkv, int T, int NB, int block, int K, void* stream) {
+  if (!logG || !noise || !logG_sel || !tau || !tau_idx) return SAS_ERR_INVALID_ARG;
+  if (logG_sel == logG || logG_sel == noise) return SAS_ERR_INVALID_ARG;
+  if (!aligned16(logG) || !aligned16(noise) || !aligned16(logG_sel) || !aligned16(tau) || !aligned16(tau_idx))
+    return SAS_ERR_INVALID_ARG;
+  if (sel && !aligned16(sel)) return SAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || T <= 0 || NB <= 0 || block != 64 || K < 1) return SAS_ERR_INVALID_ARG;
+  if ((long long)NB * 64 < T) return SAS_ERR_INVALID_ARG;
+  if (NB > 1024) return SAS_ERR_UNSUPPORTED;   // rows are held in registers
+  return cuda_status(launch_select_noisy(logG, noise, logG_sel, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB,
+                                         K - 1, as_stream(stream)));
+}
+
 int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int B, int Hkv, int T, int NB, int block,
                   void* stream) {
   if (!logG || !dLogG || !ds || ds == logG || ds == dLogG) return SAS_ERR_INVALID_ARG;

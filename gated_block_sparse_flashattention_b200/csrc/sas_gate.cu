@@ -215,6 +215,97 @@ __global__ void __launch_bounds__(256) normalize_select_kernel(const float* __re
 }
 
 // ---------------------------------------------------------------------------
+// Noisy selection for the "full*" training scope (SAS paper §4.1, Table 1 row
+// 11: noise added to the scores before Top-K). One warp per row, the row in
+// registers: the keys logG + noise (an fp32 add) give the Top-(K-1) set; logG_sel
+// keeps logG on that set and -inf elsewhere, and (tau, tau_idx) is the threshold
+// of logG_sel (the least kept gate and the last kept block holding it), so that
+// the attention calls, which find the selected blocks by thresholding their gate
+// tensor, find exactly this set in logG_sel.
+// ---------------------------------------------------------------------------
+template <int KREG>
+__global__ void __launch_bounds__(256) select_noisy_kernel(const float* __restrict__ logG,
+                                                           const float* __restrict__ noise,
+                                                           float* __restrict__ logG_sel, float* __restrict__ tau,
+                                                           int32_t* __restrict__ tau_idx, int32_t* __restrict__ sel,
+                                                           long long rows, int T, int NB, int H) {
+  __shared__ __align__(16) uint32_t hist_all[8][256];   // per-warp scratch of the select
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * 8 + wid;
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  const float* lrow = logG + row * (long long)NB;
+  const float* nrow = noise + row * (long long)NB;
+  float* dst = logG_sel + row * (long long)NB;
+  int32_t* out = sel ? sel + row * (long long)H : nullptr;
+  float lg[KREG];
+  uint32_t keys[KREG];
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    const int m = lane + 32 * i;
+    lg[i] = (m < c) ? __ldg(lrow + m) : -INFINITY;
+    keys[i] = (m < c) ? float_key(__fadd_rn(lg[i], __ldg(nrow + m))) : 0u;
+  }
+  bool take[KREG];
+  if (min(c, H) == 0 || c <= H) {   // nothing or every historical block
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) take[i] = (H > 0) && (lane + 32 * i < c);
+  } else {
+    uint32_t tk = 0u;
+    int ti = -1;
+    threshold_keys(keys, c, H, reinterpret_cast<uint2*>(hist_all[wid]), &tk, &ti);
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) {
+      const int m = lane + 32 * i;
+      take[i] = m < c && (keys[i] > tk || (keys[i] == tk && m <= ti));
+    }
+  }
+  // Threshold of logG_sel: the least kept gate and the last kept block holding it.
+  float tmin = INFINITY;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i)
+    if (take[i]) tmin = fminf(tmin, lg[i]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) tmin = fminf(tmin, __shfl_xor_sync(0xffffffffu, tmin, o));
+  int tix = -1;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i)
+    if (take[i] && lg[i] == tmin) tix = lane + 32 * i;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) tix = max(tix, __shfl_xor_sync(0xffffffffu, tix, o));
+  if (lane == 0) {
+    if (min(c, H) == 0) {
+      tau[row] = INFINITY;
+      tau_idx[row] = -1;
+    } else if (c <= H) {
+      tau[row] = -INFINITY;
+      tau_idx[row] = c - 1;
+    } else {
+      tau[row] = (tmin == 0.f) ? 0.f : tmin;   // -0 and +0 are one threshold
+      tau_idx[row] = tix;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    const int m = lane + 32 * i;
+    if (m < NB) dst[m] = take[i] ? lg[i] : -INFINITY;
+  }
+  for (int m = lane + 32 * KREG; m < NB; m += 32) dst[m] = -INFINITY;
+  if (out) {
+    int pos = 0;
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, take[i]);
+      if (take[i]) out[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * i;
+      pos += __popc(bal);
+    }
+    for (int k = pos + lane; k < H; k += 32) out[k] = -1;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Selector-score gradient (SAS paper Appendix D.3, the softmax backward, with the
 // gate gradient in log form): ds[m] = dLogG[m] - exp(logG[m]) * sum_{l<c} dLogG[l]
 // for m < c_t, 0 otherwise. One warp per row; HBM-bound.
@@ -312,6 +403,23 @@ cudaError_t launch_normalize_select(const float* s, float* logG, float* tau, int
     normalize_select_kernel<16><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
   else
     normalize_select_kernel<kSelectReg><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
+                                int32_t* sel, long long rows, int T, int NB, int H, cudaStream_t st) {
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (NB <= 128)
+    select_noisy_kernel<4><<<grid, 256, 0, st>>>(logG, noise, logG_sel, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 256)
+    select_noisy_kernel<8><<<grid, 256, 0, st>>>(logG, noise, logG_sel, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 512)
+    select_noisy_kernel<16><<<grid, 256, 0, st>>>(logG, noise, logG_sel, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 32 * kSelectReg)
+    select_noisy_kernel<kSelectReg><<<grid, 256, 0, st>>>(logG, noise, logG_sel, tau, tau_idx, sel, rows, T, NB, H);
+  else
+    return cudaErrorInvalidValue;
   count_launch();
   return cudaGetLastError();
 }

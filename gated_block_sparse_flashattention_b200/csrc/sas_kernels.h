@@ -16,6 +16,8 @@ cudaError_t launch_select_threshold(const float* logG, float* tau, int32_t* tau_
                                     int T, int NB, int H, cudaStream_t st);
 cudaError_t launch_normalize_select(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel,
                                     long long rows, int T, int NB, int H, cudaStream_t st);
+cudaError_t launch_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
+                                int32_t* sel, long long rows, int T, int NB, int H, cudaStream_t st);
 cudaError_t launch_gate_grad(const float* logG, const float* dLogG, float* ds, long long rows, int T, int NB,
                              cudaStream_t st);
 cudaError_t launch_tile_union(const float* logG, const float* tau, const int32_t* tau_idx, uint32_t* masks,

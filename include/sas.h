@@ -118,6 +118,27 @@ SAS_API int sas_gate_normalize_select(const float* s, float* logG, float* tau, i
                                       int Hkv, int T, int NB, int block, int K, void* stream);
 
 /*
+ * sas_select_noisy - selection for the "full*" training scope (SAS paper §4.1,
+ * Table 1 row 11: noise added to the selector scores before Top-K). Per (b, g, t)
+ * with c = min(t / 64, NB) historical blocks:
+ *   chosen = the K-1 largest of key[m] = logG[m] + noise[m] (an fp32 add) over
+ *            m < c, ties to the lower block (every historical block when c <= K-1);
+ *   logG_sel[m] = logG[m] for m in chosen, -inf otherwise;
+ *   (tau, tau_idx) = the threshold of logG_sel, as sas_select_threshold would give
+ *            it: the least kept gate (-0 written as +0) and the largest kept block
+ *            holding it; (-inf, c-1) when c <= K-1; (+inf, -1) when nothing is kept.
+ * sas_fwd / sas_bwd given (logG_sel, tau, tau_idx) attend exactly the chosen blocks
+ * with the clean gates logG on them; the gradient they return for logG_sel is the
+ * gradient for logG (zero off the chosen blocks), for sas_gate_grad with logG.
+ * logG, noise, logG_sel: [B,Hkv,T,NB] fp32 (logG_sel may alias neither input);
+ * tau [B,Hkv,T] fp32; tau_idx [B,Hkv,T] int32; sel (nullable) [B,Hkv,T,K-1] int32,
+ * the chosen blocks ascending, -1 padded. The caller draws the noise.
+ * NB >= ceil(T / 64), NB <= 1024 (else SAS_ERR_UNSUPPORTED), block == 64, K >= 1.
+ */
+SAS_API int sas_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
+                             int32_t* sel, int B, int Hkv, int T, int NB, int block, int K, void* stream);
+
+/*
  * sas_gate_grad - gradient with respect to the selector scores s through the
  * gate normalisation (SAS paper Appendix D.3, the softmax backward
  * ds_m = g_m (dg_m - sum_l g_l dg_l), with the gate gradient given in log form

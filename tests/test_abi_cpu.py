@@ -85,6 +85,10 @@ def test_invalid_calls_return_errors_without_launching(lib):
                                          None) == -1                                # s aliases logG
     assert lib.sas_gate_normalize_select(fake, fake + 64, fake + 128, fake + 192, None, 1, 1, 192, 2, 64, 4,
                                          None) == -1                                # NB * 64 < T
+    assert lib.sas_select_noisy(fake, fake + 64, fake, fake + 128, fake + 192, None, 1, 1, 128, 2, 64, 4,
+                                None) == -1                                          # logG_sel aliases logG
+    assert lib.sas_select_noisy(fake, fake + 64, fake + 256, fake + 128, fake + 192, None, 1, 1, 128 * 64, 2048,
+                                64, 4, None) == -2                                   # rows over 1024 blocks
     assert lib.sas_gate_grad(fake, fake + 64, fake + 64, 1, 1, 128, 2, 64, None) == -1   # ds aliases dLogG
     assert lib.sas_gate_grad(fake, fake + 64, fake + 132, 1, 1, 128, 2, 64, None) == -1  # misaligned ds
     assert lib.sas_gate_grad(fake, fake + 64, fake + 128, 1, 1, 128, 2, 32, None) == -1  # block != 64
