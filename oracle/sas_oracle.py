@@ -315,6 +315,59 @@ def forward_backward(Q, K, V, dO, logG, tau, tau_idx, block: int, sm_scale: floa
 
 
 # --------------------------------------------------------------------------------------
+# Variable-length packing (SAS paper §5.1 training on packed sequences, and the
+# packing used for the long-context selector training in its appendix): several
+# documents share one sequence axis. A document never sees another: it is its own
+# causal sequence whose blocks start at its first token (every document starts on a
+# block boundary), so the packed problem is the independent problems of its
+# documents. In the packed score and gate tensors, document i's rows are its token
+# range and its blocks are the columns of its own block range.
+# --------------------------------------------------------------------------------------
+def doc_slices(cu_seqlens, block: int):
+    """(token slice, block slice) per document; cu_seqlens: ascending multiples of block from 0 to T."""
+    cu = [int(x) for x in cu_seqlens]
+    assert cu[0] == 0 and all(b > a for a, b in zip(cu, cu[1:])) and all(x % block == 0 for x in cu)
+    return [(slice(a, b), slice(a // block, b // block)) for a, b in zip(cu, cu[1:])]
+
+
+def gate_normalize_varlen(s, cu_seqlens, block: int):
+    """Packed logG: each document's gate_normalize on its own rows and block columns, -inf elsewhere."""
+    s = _f64(s)
+    out = np.full(s.shape, -np.inf)
+    for ts, bs in doc_slices(cu_seqlens, block):
+        out[:, :, ts, bs] = gate_normalize(s[:, :, ts, bs], block)
+    return out
+
+
+def selection_mask_varlen(logG, K: int, cu_seqlens, block: int):
+    """Packed boolean [B,Hkv,T,NB]: each document's Top-(K-1) selection (select_threshold on its own gates)."""
+    lg = _f64(logG)
+    mask = np.zeros(lg.shape, dtype=bool)
+    for ts, bs in doc_slices(cu_seqlens, block):
+        part = lg[:, :, ts, bs]
+        tau, tidx, _ = select_threshold(part, K, block)
+        mask[:, :, ts, bs] = selection_mask(part, tau, tidx, block)
+    return mask
+
+
+def forward_backward_varlen(Q, K, V, dO, logG, Kbudget: int, cu_seqlens, block: int, sm_scale: float):
+    """forward_backward of every document on its own (its gates, its Top-(K-1)), assembled on the packed axis."""
+    Q, K, V, dO, lg = _f64(Q), _f64(K), _f64(V), _f64(dO), _f64(logG)
+    B, Hq, T, d = Q.shape
+    Hkv, NB = K.shape[1], lg.shape[-1]
+    out = {"O": np.zeros((B, Hq, T, d)), "LSE": np.zeros((B, Hq, T)), "dQ": np.zeros((B, Hq, T, d)),
+           "dK": np.zeros((B, Hkv, T, d)), "dV": np.zeros((B, Hkv, T, d)), "dLogG": np.zeros((B, Hkv, T, NB))}
+    for ts, bs in doc_slices(cu_seqlens, block):
+        part = lg[:, :, ts, bs]
+        tau, tidx, _ = select_threshold(part, Kbudget, block)
+        r = forward_backward(Q[:, :, ts], K[:, :, ts], V[:, :, ts], dO[:, :, ts], part, tau, tidx, block, sm_scale)
+        for k in ("O", "LSE", "dQ", "dK", "dV"):
+            out[k][:, :, ts] = r[k]
+        out["dLogG"][:, :, ts, bs] = r["dLogG"]
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # The same eq. 9 evaluated the gathered way: per query row, collect the attended
 # token set S = B_0 ∪ selected blocks and run softmax(q K_S^T + log g_S) V_S on
 # that subset only.  Used for sampled checks at full size, where the dense

@@ -620,3 +620,85 @@ def test_select_noisy_pin_catches_planted_mistake(monkeypatch):
     monkeypatch.setattr(orc, "select_noisy", _bad_select_noisy)
     with pytest.raises(AssertionError):
         test_select_noisy_planted_noise_wins_and_keys_are_fp32()
+
+
+# ---------------------------------------------------------------- variable-length packing
+def _packed_from_docs(docs, block, rng, NB_extra=0):
+    """Pack per-document inputs (each its own problem) along T; score columns of other documents get noise."""
+    B, Hq, Hkv, d = 1, 4, 2, 8
+    cu = np.cumsum([0] + [L for L in docs])
+    T = int(cu[-1])
+    NB = T // block + NB_extra
+    per = []
+    Q = rng.standard_normal((B, Hq, T, d))
+    Kt, Vt, dO = rng.standard_normal((B, Hkv, T, d)), rng.standard_normal((B, Hkv, T, d)), rng.standard_normal((B, Hq, T, d))
+    s = rng.standard_normal((B, Hkv, T, NB)) * 5.0 + 50.0       # leaked columns would dominate
+    for i, L in enumerate(docs):
+        a = int(cu[i])
+        sd = rng.standard_normal((B, Hkv, L, L // block))
+        s[:, :, a:a + L, a // block:a // block + L // block] = sd
+        per.append((slice(a, a + L), sd))
+    return Q, Kt, Vt, dO, s, cu, per
+
+
+def test_varlen_equals_each_document_alone():
+    rng = np.random.default_rng(41)
+    block, Kb, sm = 16, 3, 0.3
+    docs = [48, 16, 80]
+    Q, Kt, Vt, dO, s, cu, per = _packed_from_docs(docs, block, rng, NB_extra=2)
+    logG = orc.gate_normalize_varlen(s, cu, block)
+    out = orc.forward_backward_varlen(Q, Kt, Vt, dO, logG, Kb, cu, block, sm)
+    mask = orc.selection_mask_varlen(logG, Kb, cu, block)
+    for ts, sd in per:
+        lg = orc.gate_normalize(sd, block)
+        tau, tidx, _ = orc.select_threshold(lg, Kb, block)
+        ref = orc.forward_backward(Q[:, :, ts], Kt[:, :, ts], Vt[:, :, ts], dO[:, :, ts], lg, tau, tidx, block, sm)
+        b0 = ts.start // block
+        nb = lg.shape[-1]
+        np.testing.assert_array_equal(logG[:, :, ts, b0:b0 + nb], lg)
+        assert np.all(np.isneginf(np.delete(logG[:, :, ts], np.s_[b0:b0 + nb], axis=-1)))
+        np.testing.assert_array_equal(mask[:, :, ts, b0:b0 + nb], orc.selection_mask(lg, tau, tidx, block))
+        for k in ("O", "LSE", "dQ", "dK", "dV"):
+            np.testing.assert_allclose(out[k][:, :, ts], ref[k], atol=1e-12)
+        np.testing.assert_allclose(out["dLogG"][:, :, ts, b0:b0 + nb], ref["dLogG"], atol=1e-12)
+    assert not mask[..., sum(docs) // block:].any()
+
+
+def test_varlen_uniform_scores_full_budget_is_block_diagonal_sdpa():
+    """Uniform scores and a budget covering every block: each document is causal attention with a
+    -log(historical blocks of its own) bias on its earlier blocks, and nothing across documents."""
+    B, Hq, Hkv, d, block = 1, 2, 1, 8, 16
+    docs = [32, 64, 48]
+    T = sum(docs)
+    rng = np.random.default_rng(42)
+    Q, K, V = rng.standard_normal((B, Hq, T, d)), rng.standard_normal((B, Hkv, T, d)), rng.standard_normal((B, Hkv, T, d))
+    dO = rng.standard_normal((B, Hq, T, d))
+    cu = np.cumsum([0] + docs)
+    s = np.full((B, Hkv, T, T // block), 0.4)
+    logG = orc.gate_normalize_varlen(s, cu, block)
+    out = orc.forward_backward_varlen(Q, K, V, dO, logG, T // block, cu, block, 0.5)
+    i = np.arange(T)
+    doc = np.searchsorted(cu, i, side="right") - 1
+    start_blk = cu[doc] // block
+    c = i // block
+    same = doc[:, None] == doc[None, :]
+    hist = (i[None, :] // block < c[:, None]) & same
+    bias = np.where(hist, -np.log(np.maximum(c - start_blk, 1))[:, None], 0.0)
+    bias = np.where((i[None, :] <= i[:, None]) & same, bias, -np.inf)
+    np.testing.assert_allclose(out["O"], _sdpa(Q, K, V, torch.from_numpy(bias), 0.5, Hq), atol=1e-12)
+
+
+def _bad_gate_normalize_varlen(s, cu_seqlens, block):
+    """Mistake: each document's gates read from the first block columns instead of its own."""
+    s = np.asarray(s, float)
+    out = np.full(s.shape, -np.inf)
+    for ts, bs in orc.doc_slices(cu_seqlens, block):
+        nb = bs.stop - bs.start
+        out[:, :, ts, bs] = orc.gate_normalize(s[:, :, ts, :nb], block)
+    return out
+
+
+def test_varlen_pin_catches_planted_mistake(monkeypatch):
+    monkeypatch.setattr(orc, "gate_normalize_varlen", _bad_gate_normalize_varlen)
+    with pytest.raises(AssertionError):
+        test_varlen_equals_each_document_alone()
