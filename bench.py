@@ -61,6 +61,7 @@ def measured_traffic(name: str):
 BENCH_WORKLOAD = "qwen3_4b_t8k"
 DECODE_WORKLOAD = "decode_b16_l32k"
 PAGED_DECODE_WORKLOAD = "decode_b8_l512k_paged"
+VARLEN_DOCS = [512, 1536, 1024, 2048, 3072]   # documents packed into the bench layer's 8192 positions
 METRIC = "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd+gate-grad step)"
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2, written between timed steps
 
@@ -70,6 +71,13 @@ def attended_keys_per_row(T: int, K: int, block: int = 64) -> np.ndarray:
     """n_t for every position t: causal part of the current block plus min(K-1, c_t) full blocks."""
     t = np.arange(T)
     return (t % block) + 1 + block * np.minimum(K - 1, t // block)
+
+
+def attended_flops_varlen(w, docs) -> tuple[float, float]:
+    """(forward, backward) algorithmic FLOPs of one packed step: every document a sequence of its own."""
+    n = sum(attended_keys_per_row(L, w.K, w.block).sum(dtype=np.float64) for L in docs)
+    fwd = 4.0 * w.d * n * w.B * w.Hq
+    return fwd, 2.5 * fwd
 
 
 def attended_flops(w) -> tuple[float, float]:
@@ -435,6 +443,7 @@ def run_gpu(args):
     e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
     dec = run_decode(args, device, stream, binding, peaks, clk) if "decode" in legs else None
     dec_paged = run_decode_paged(args, device, stream, binding, peaks, clk) if "paged" in legs else None
+    varlen = run_varlen(args, w, host, device, stream, binding, flush) if "varlen" in legs else None
     clk.active = False
     clk.__exit__(None, None, None)
 
@@ -454,6 +463,7 @@ def run_gpu(args):
         "gpu_launches": launches,
         "decode": dec,
         "decode_paged": dec_paged,
+        "varlen": varlen,
     }
     if rank == 0 and world == 1 and "cpu" in legs:
         tf, threads, desc = oracle_sample(w, args.cpu_seconds)
@@ -465,6 +475,50 @@ def run_gpu(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_varlen(args, w, host, device, stream, binding, flush):
+    """The training step on a packed sequence: the bench layer's 8192 positions as five documents of
+    512, 1536, 1024, 2048 and 3072 tokens (varlen gates and selection, then the unchanged forward, backward
+    and selector gradient), device-resident inputs, L2 flushed between steps outside the events."""
+    docs = VARLEN_DOCS
+    cu = np.cumsum([0] + docs).tolist()
+    Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
+    logG = torch.empty_like(s)
+    tau = torch.empty(w.B, w.Hkv, w.T, device=device)
+    tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
+    O, LSE = torch.empty_like(Q), torch.empty(w.B, w.Hq, w.T, device=device)
+    dQ, dK, dV, dLogG, ds = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s),
+                             torch.empty_like(s))
+    ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
+    ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
+
+    def step():
+        binding.sas_gate_normalize_select_varlen(s, logG, tau, tidx, None, w.K, cu, stream=stream)
+        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.sm_scale, ws_f, stream=stream)
+        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
+                        stream=stream)
+        binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize(device)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in times)
+    fwd, bwd = attended_flops_varlen(w, docs)
+    status = binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b)
+    return {"workload": f"qwen3_4b_t8k packed as documents of {docs} tokens", "ms_per_step": round(ms, 4),
+            "value": round((fwd + bwd) / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "attended_gflop_per_step": round((fwd + bwd) / 1e9, 2), "device_status": status}
 
 
 def run_e2e(args, w, host, device, stream, binding, step_flops, world):
@@ -641,10 +695,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--legs", default="step,e2e,decode,paged,cpu",
+    ap.add_argument("--legs", default="step,e2e,decode,paged,varlen,cpu",
                     help="comma list of what to measure and report: step (device-resident timed steps), e2e "
-                         "(host buffers through the C ABI), decode, paged (long-context paged decode), cpu (oracle "
-                         "baseline)")
+                         "(host buffers through the C ABI), decode, paged (long-context paged decode), varlen (packed "
+                         "documents), cpu (oracle baseline)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3

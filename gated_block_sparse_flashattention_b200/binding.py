@@ -33,6 +33,7 @@ _SIGNATURES = {
     "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_normalize_select": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _vp]),
+    "sas_gate_normalize_select_varlen": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_vp, _c_int, _vp]),
     "sas_select_noisy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_grad": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_fwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
@@ -129,6 +130,15 @@ def sas_gate_normalize_select(s, logG, tau, tau_idx, sel, K, block=BLOCK, stream
     B, Hkv, T, NB = s.shape
     _check("sas_gate_normalize_select", lib().sas_gate_normalize_select(
         _ptr(s), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
+
+
+def sas_gate_normalize_select_varlen(s, logG, tau, tau_idx, sel, K, cu_seqlens, block=BLOCK, stream=None):
+    """cu_seqlens: host sequence of n_docs + 1 token offsets (multiples of 64, from 0 to T)."""
+    B, Hkv, T, NB = s.shape
+    cu = (ctypes.c_int32 * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+    _check("sas_gate_normalize_select_varlen", lib().sas_gate_normalize_select_varlen(
+        _ptr(s), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K,
+        ctypes.cast(cu, ctypes.c_void_p), len(cu_seqlens) - 1, _stream(stream)))
 
 
 def sas_select_noisy(logG, noise, logG_sel, tau, tau_idx, sel, K, block=BLOCK, stream=None):

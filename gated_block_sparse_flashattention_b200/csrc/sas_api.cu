@@ -110,6 +110,27 @@ int sas_gate_normalize_select(const float* s, float* logG, float* tau, int32_t* 
       launch_normalize_select(s, logG, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB, K - 1, as_stream(stream)));
 }
 
+int sas_gate_normalize_select_varlen(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel, int B,
+                                     int Hkv, int T, int NB, int block, int K, const int32_t* cu_seqlens,
+                                     int n_docs, void* stream) {
+  if (!s || !logG || !tau || !tau_idx || !cu_seqlens || s == logG) return SAS_ERR_INVALID_ARG;
+  if (!aligned16(s) || !aligned16(logG) || !aligned16(tau) || !aligned16(tau_idx)) return SAS_ERR_INVALID_ARG;
+  if (sel && !aligned16(sel)) return SAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || T <= 0 || NB <= 0 || block != 64 || K < 1) return SAS_ERR_INVALID_ARG;
+  if ((long long)NB * 64 < T) return SAS_ERR_INVALID_ARG;
+  if (n_docs < 1 || n_docs > kMaxDocs) return n_docs < 1 ? SAS_ERR_INVALID_ARG : SAS_ERR_UNSUPPORTED;
+  if (NB > 1024) return SAS_ERR_UNSUPPORTED;   // rows are held in registers
+  DocTable docs{};
+  docs.n = n_docs;
+  if (cu_seqlens[0] != 0 || cu_seqlens[n_docs] != T) return SAS_ERR_INVALID_ARG;
+  for (int i = 0; i < n_docs; ++i) {
+    if (cu_seqlens[i + 1] <= cu_seqlens[i] || cu_seqlens[i] % 64 != 0) return SAS_ERR_INVALID_ARG;
+    docs.start_blk[i] = cu_seqlens[i] / 64;
+  }
+  return cuda_status(launch_normalize_select_varlen(s, logG, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB, K - 1,
+                                                    docs, as_stream(stream)));
+}
+
 int sas_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
                      int32_t* sel, int B, int Hkv, int T, int NB, int block, int K, void* stream) {
   if (!logG || !noise || !logG_sel || !tau || !tau_idx) return SAS_ERR_INVALID_ARG;

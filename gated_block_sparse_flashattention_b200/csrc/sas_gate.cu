@@ -37,18 +37,19 @@ __global__ void __launch_bounds__(256) gate_normalize_kernel(const float* __rest
 
 // Threshold (tau, tau_idx) and optional ascending index list of one row whose
 // keys are in KREG registers per lane (key of block m = lane + 32 i in keys[i]).
+// Block indices written (tau_idx, the list) are base + the key's position.
 template <int KREG>
 __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], int c, int H, uint32_t* hist,
-                                                 float* tau_out, int32_t* tidx_out, int32_t* out) {
+                                                 float* tau_out, int32_t* tidx_out, int32_t* out, int base = 0) {
   const int lane = threadIdx.x & 31;
   uint32_t tkey = 0u, asc = 0u;
   int tidx = -1;
   if (H <= 32 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, &asc)) {
     if (lane == 0) {
       *tau_out = key_float(tkey);
-      *tidx_out = tidx;
+      *tidx_out = base + tidx;
     }
-    if (out && lane < H) out[lane] = (int32_t)asc;   // exactly H blocks, ascending
+    if (out && lane < H) out[lane] = base + (int32_t)asc;   // exactly H blocks, ascending
     return;
   }
   int take_eq = 0;
@@ -56,7 +57,7 @@ __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], i
   tidx = tie_index_keys(keys, c, tkey, take_eq);
   if (lane == 0) {
     *tau_out = key_float(tkey);
-    *tidx_out = tidx;
+    *tidx_out = base + tidx;
   }
   if (out) {
     int pos = 0;
@@ -66,7 +67,7 @@ __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], i
       const int m = lane + 32 * i;
       const bool take = m < c && (keys[i] > tkey || (keys[i] == tkey && m <= tidx));
       const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      if (take) out[pos + __popc(bal & ((1u << lane) - 1u))] = m;
+      if (take) out[pos + __popc(bal & ((1u << lane) - 1u))] = base + m;
       pos += __popc(bal);
     }
     for (int k = pos + lane; k < H; k += 32) out[k] = -1;
@@ -164,13 +165,15 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
 // 32 * kSelectReg blocks use the two kernels.
 // ---------------------------------------------------------------------------
 template <int KREG>
-__device__ __forceinline__ void normalize_select_row(const float* __restrict__ src, float* __restrict__ dst, int c,
-                                                     int NB, int H, uint32_t* hist, float* tau_out,
+__device__ __forceinline__ void normalize_select_row(const float* __restrict__ src, float* __restrict__ dst, int c_lo,
+                                                     int c, int NB, int H, uint32_t* hist, float* tau_out,
                                                      int32_t* tidx_out, int32_t* out) {
+  // The row's historical blocks are c_lo .. c-1 (c_lo > 0 only for a later document of a packed sequence).
   const int lane = threadIdx.x & 31;
+  const int n = c - c_lo;
   float v[KREG];
 #pragma unroll
-  for (int i = 0; i < KREG; ++i) v[i] = (lane + 32 * i < c) ? __ldg(src + lane + 32 * i) : -INFINITY;
+  for (int i = 0; i < KREG; ++i) v[i] = (lane + 32 * i < n) ? __ldg(src + c_lo + lane + 32 * i) : -INFINITY;
   float mx = -INFINITY;
 #pragma unroll
   for (int i = 0; i < KREG; ++i) mx = fmaxf(mx, v[i]);
@@ -179,21 +182,49 @@ __device__ __forceinline__ void normalize_select_row(const float* __restrict__ s
   float sum = 0.f;
 #pragma unroll
   for (int i = 0; i < KREG; ++i)
-    if (lane + 32 * i < c) sum += expf(v[i] - mx);
+    if (lane + 32 * i < n) sum += expf(v[i] - mx);
 #pragma unroll
   for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float lse = mx + logf(sum);
   uint32_t keys[KREG];
 #pragma unroll
   for (int i = 0; i < KREG; ++i) {
-    const int m = lane + 32 * i;
-    const float lg = (m < c) ? v[i] - lse : -INFINITY;
-    if (m < NB) dst[m] = lg;
-    keys[i] = (m < c) ? float_key(lg) : 0u;
+    const int q = lane + 32 * i;
+    const float lg = (q < n) ? v[i] - lse : -INFINITY;
+    if (c_lo + q < NB) dst[c_lo + q] = lg;
+    keys[i] = (q < n) ? float_key(lg) : 0u;
+    v[i] = lg;
   }
-  for (int m = lane + 32 * KREG; m < NB; m += 32) dst[m] = -INFINITY;
-  if (select_trivial_row(c, H, tau_out, tidx_out, out)) return;
-  select_keys_regs(keys, c, H, hist, tau_out, tidx_out, out);
+  for (int m = lane; m < c_lo; m += 32) dst[m] = -INFINITY;
+  for (int m = c_lo + lane + 32 * KREG; m < NB; m += 32) dst[m] = -INFINITY;
+  if (c_lo == 0) {
+    if (select_trivial_row(c, H, tau_out, tidx_out, out)) return;
+  } else if (min(n, H) == 0 || n <= H) {
+    // Nothing, or every block of the row's own document: the threshold is its
+    // least gate (and the last block holding it), which keeps no block of an
+    // earlier document (their gates are -inf).
+    float tmin = INFINITY;
+#pragma unroll
+    for (int i = 0; i < KREG; ++i)
+      if (lane + 32 * i < n) tmin = fminf(tmin, v[i]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) tmin = fminf(tmin, __shfl_xor_sync(0xffffffffu, tmin, o));
+    int tix = -1;
+#pragma unroll
+    for (int i = 0; i < KREG; ++i)
+      if (lane + 32 * i < n && v[i] == tmin) tix = lane + 32 * i;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) tix = max(tix, __shfl_xor_sync(0xffffffffu, tix, o));
+    const bool none = min(n, H) == 0;
+    if (lane == 0) {
+      *tau_out = none ? INFINITY : ((tmin == 0.f) ? 0.f : tmin);
+      *tidx_out = none ? -1 : c_lo + tix;
+    }
+    if (out)
+      for (int k = lane; k < H; k += 32) out[k] = (!none && k < n) ? c_lo + k : -1;
+    return;
+  }
+  select_keys_regs(keys, n, H, hist, tau_out, tidx_out, out, c_lo);
 }
 
 // KREG from the row length NB on the host, so short rows run with few registers
@@ -210,7 +241,35 @@ __global__ void __launch_bounds__(256) normalize_select_kernel(const float* __re
   const int t = (int)(row % T);
   const int c = min(t / kBlock, NB);
   int32_t* out = sel ? sel + row * (long long)H : nullptr;
-  normalize_select_row<KREG>(s + row * (long long)NB, logG + row * (long long)NB, c, NB, H, hist_all[wid],
+  normalize_select_row<KREG>(s + row * (long long)NB, logG + row * (long long)NB, 0, c, NB, H, hist_all[wid],
+                             tau + row, tau_idx + row, out);
+}
+
+// Packed sequences: the same per row, over the blocks of the row's own document
+// (its first block from the document table, by binary search; documents start
+// on block boundaries).
+template <int KREG>
+__global__ void __launch_bounds__(256) normalize_select_varlen_kernel(
+    const float* __restrict__ s, float* __restrict__ logG, float* __restrict__ tau, int32_t* __restrict__ tau_idx,
+    int32_t* __restrict__ sel, long long rows, int T, int NB, int H, const DocTable docs) {
+  __shared__ __align__(16) uint32_t hist_all[8][256];   // per-warp scratch of the select
+  const int wid = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * 8 + wid;
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int cur = t / kBlock;
+  int lo = 0, hi = docs.n - 1;   // the last document starting at or before block cur
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (docs.start_blk[mid] <= cur)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int c = min(cur, NB);
+  const int c_lo = min(docs.start_blk[lo], c);
+  int32_t* out = sel ? sel + row * (long long)H : nullptr;
+  normalize_select_row<KREG>(s + row * (long long)NB, logG + row * (long long)NB, c_lo, c, NB, H, hist_all[wid],
                              tau + row, tau_idx + row, out);
 }
 
@@ -403,6 +462,25 @@ cudaError_t launch_normalize_select(const float* s, float* logG, float* tau, int
     normalize_select_kernel<16><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
   else
     normalize_select_kernel<kSelectReg><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_normalize_select_varlen(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel,
+                                           long long rows, int T, int NB, int H, const DocTable& docs,
+                                           cudaStream_t st) {
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (NB <= 128)
+    normalize_select_varlen_kernel<4><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H, docs);
+  else if (NB <= 256)
+    normalize_select_varlen_kernel<8><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H, docs);
+  else if (NB <= 512)
+    normalize_select_varlen_kernel<16><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H, docs);
+  else if (NB <= 32 * kSelectReg)
+    normalize_select_varlen_kernel<kSelectReg><<<grid, 256, 0, st>>>(s, logG, tau, tau_idx, sel, rows, T, NB, H,
+                                                                      docs);
+  else
+    return cudaErrorInvalidValue;
   count_launch();
   return cudaGetLastError();
 }

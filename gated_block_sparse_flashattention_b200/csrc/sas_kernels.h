@@ -16,6 +16,15 @@ cudaError_t launch_select_threshold(const float* logG, float* tau, int32_t* tau_
                                     int T, int NB, int H, cudaStream_t st);
 cudaError_t launch_normalize_select(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel,
                                     long long rows, int T, int NB, int H, cudaStream_t st);
+// Document table of a packed sequence: the first block of each document.
+constexpr int kMaxDocs = 256;
+struct DocTable {
+  int n;
+  int start_blk[kMaxDocs];
+};
+cudaError_t launch_normalize_select_varlen(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel,
+                                           long long rows, int T, int NB, int H, const DocTable& docs,
+                                           cudaStream_t st);
 cudaError_t launch_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
                                 int32_t* sel, long long rows, int T, int NB, int H, cudaStream_t st);
 cudaError_t launch_gate_grad(const float* logG, const float* dLogG, float* ds, long long rows, int T, int NB,

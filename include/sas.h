@@ -118,6 +118,29 @@ SAS_API int sas_gate_normalize_select(const float* s, float* logG, float* tau, i
                                       int Hkv, int T, int NB, int block, int K, void* stream);
 
 /*
+ * sas_gate_normalize_select_varlen - sas_gate_normalize_select for a packed
+ * sequence of documents (SAS paper §5.1: training on packed sequences). Document
+ * i covers tokens cu_seqlens[i] .. cu_seqlens[i+1]-1 and blocks
+ * cu_seqlens[i]/64 .. cu_seqlens[i+1]/64-1; it never sees another document. For
+ * a row t of document i (c = t/64, c_i = cu_seqlens[i]/64) the gates are the
+ * softmax of s over its own earlier blocks c_i .. c-1 (logG = -inf on every other
+ * column) and the Top-(K-1) is taken among them (ties to the lower block); block
+ * indices in tau_idx and sel are those of the packed sequence. A row keeping every
+ * block of its document (c - c_i <= K-1) gets (-inf, c-1) in the first document
+ * and, in later ones, (the least of its gates, the last block holding it), so that
+ * the threshold keeps no block of an earlier document; a row keeping nothing gets
+ * (+inf, -1). sas_fwd, sas_bwd and sas_gate_grad take these outputs as they are:
+ * the attended set of every row lies inside its own document.
+ * cu_seqlens: HOST int32 [n_docs + 1], 0 = cu[0] < cu[1] < ... < cu[n_docs] = T,
+ * every entry a multiple of 64; 1 <= n_docs <= 256 (more: SAS_ERR_UNSUPPORTED).
+ * Other arguments as for sas_gate_normalize_select; NB <= 1024 (else
+ * SAS_ERR_UNSUPPORTED). The same packing applies to every (b, g).
+ */
+SAS_API int sas_gate_normalize_select_varlen(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel,
+                                             int B, int Hkv, int T, int NB, int block, int K,
+                                             const int32_t* cu_seqlens, int n_docs, void* stream);
+
+/*
  * sas_select_noisy - selection for the "full*" training scope (SAS paper §4.1,
  * Table 1 row 11: noise added to the selector scores before Top-K). Per (b, g, t)
  * with c = min(t / 64, NB) historical blocks:

@@ -89,6 +89,15 @@ def test_invalid_calls_return_errors_without_launching(lib):
                                 None) == -1                                          # logG_sel aliases logG
     assert lib.sas_select_noisy(fake, fake + 64, fake + 256, fake + 128, fake + 192, None, 1, 1, 128 * 64, 2048,
                                 64, 4, None) == -2                                   # rows over 1024 blocks
+    def cu(*v):
+        return ctypes.cast((ctypes.c_int32 * len(v))(*v), ctypes.c_void_p)
+    vl = lambda c, n, T=256: lib.sas_gate_normalize_select_varlen(fake, fake + 64, fake + 128, fake + 192, None, 1,  # noqa: E731
+                                                                  1, T, T // 64, 64, 4, c, n, None)
+    assert vl(cu(0, 100, 256), 2) == -1          # a document not on a block boundary
+    assert vl(cu(0, 128, 192), 2) == -1          # offsets end before T
+    assert vl(cu(0, 128, 128, 256), 3) == -1     # an empty document
+    assert vl(cu(0, 256), 0) == -1               # no document
+    assert vl(cu(*range(0, 64 * 258, 64)), 257, T=64 * 257) == -2   # more than 256 documents
     assert lib.sas_gate_grad(fake, fake + 64, fake + 64, 1, 1, 128, 2, 64, None) == -1   # ds aliases dLogG
     assert lib.sas_gate_grad(fake, fake + 64, fake + 132, 1, 1, 128, 2, 64, None) == -1  # misaligned ds
     assert lib.sas_gate_grad(fake, fake + 64, fake + 128, 1, 1, 128, 2, 32, None) == -1  # block != 64
