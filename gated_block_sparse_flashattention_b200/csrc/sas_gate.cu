@@ -44,7 +44,8 @@ __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], i
   const int lane = threadIdx.x & 31;
   uint32_t tkey = 0u, asc = 0u;
   int tidx = -1;
-  if (H <= 32 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, &asc)) {
+  // The ascending list (a second warp sort) only when it is requested.
+  if (H <= 32 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, out ? &asc : nullptr)) {
     if (lane == 0) {
       *tau_out = key_float(tkey);
       *tidx_out = base + tidx;

@@ -145,3 +145,29 @@ def test_paged_page_out_of_range_is_reported():
     assert binding.sas_device_status(ws) == SAS_DEV_ERR_BOUNDS
     binding.sas_device_status_clear(ws)
     assert binding.sas_device_status(ws) == 0
+
+
+def test_paged_full_size_bench_workload_sampled():
+    """The bench's long-context workload as bench.py runs it (8 sequences at 524288 tokens, 69632 shuffled
+    pages in an 18 GB pool, K=32): every selection list against the oracle, and the outputs of sampled
+    (sequence, group) pairs against the oracle on that pair's own logical cache."""
+    w = workloads.WORKLOADS["decode_b8_l512k_paged"]
+    d = workloads.make_paged_decode_inputs(w, seed=0, device="cuda")
+    o, sel, ws = run_paged(d, w)
+    assert binding.sas_device_status(ws) == 0
+    s64 = d["s"].cpu().numpy().astype(np.float64)
+    got_sel = sel.cpu().numpy()
+    c = (w.T - 1) // w.block
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            _, _, chosen = orc.topk_threshold_row(s64[b, g], c, w.K - 1)
+            assert got_sel[b, g].tolist() == chosen
+    G = w.G
+    for b, g in [(0, 0), (5, 3), (7, 7)]:
+        pages = d["page_table"][b].long()
+        Kc = d["Kp"][pages, g].reshape(1, 1, -1, w.d)           # this group's logical cache, on the device
+        Vc = d["Vp"][pages, g].reshape(1, 1, -1, w.d)
+        ref, _ = orc.decode(to_np(d["q"][b:b + 1, g * G:(g + 1) * G]), to_np(Kc), to_np(Vc),
+                            d["seqlen"][b:b + 1].cpu().numpy(), s64[b:b + 1, g:g + 1], w.K, w.block, w.sm_scale)
+        del Kc, Vc
+        assert max_abs(to_np(o[b:b + 1, g * G:(g + 1) * G]), ref) <= 2e-2

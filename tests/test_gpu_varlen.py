@@ -113,3 +113,11 @@ def test_varlen_forward_backward_and_gate_grad(w, docs):
         other = np.ones(got.shape[-1], bool)
         other[bs] = False
         assert np.all(got[:, :, ts][..., other] == 0.0)
+
+
+def test_varlen_full_size_qwen3_4b_layer_gates():
+    """The bench's packed step (the qwen3_4b_t8k layer as documents of 512, 1536, 1024, 2048 and 3072
+    tokens): gates and selection of every row at full size."""
+    w = workloads.WORKLOADS["qwen3_4b_t8k"]
+    s = workloads.make_training_inputs(w)["s"]
+    check_gates(s, w.K, np.cumsum([0, 512, 1536, 1024, 2048, 3072]).tolist())
