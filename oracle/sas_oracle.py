@@ -181,6 +181,10 @@ def select_noisy(logG32, noise32, K: int, block: int):
     ``logG_sel`` (float64: logG on the chosen blocks, -inf elsewhere), ``tau`` and
     ``tau_idx`` (the threshold of ``logG_sel``, which the attention calls use to
     find the chosen blocks again) and ``sel`` (ascending chosen blocks, -1 padded).
+    Blocks whose gate is -inf (other documents of a packed sequence, see
+    gate_normalize_varlen) are never chosen; a row with fewer finite gates than
+    K-1 chooses them all and gets the threshold (least chosen gate, last chosen
+    block holding it) so that no -inf block passes it.
     """
     lg = np.asarray(logG32, dtype=np.float32)
     keys = (lg + np.asarray(noise32, dtype=np.float32)).astype(np.float32)
@@ -194,11 +198,23 @@ def select_noisy(logG32, noise32, K: int, block: int):
         for g in range(Hkv):
             for t in range(T):
                 c = min(t // block, NB)
-                _, _, chosen = topk_threshold_row(keys[b, g, t].astype(np.float64), c, H)
+                # A block whose gate is -inf (another document of a packed sequence) is never chosen.
+                n_fin = int(np.isfinite(lg[b, g, t, :c]).sum())
+                k = min(H, n_fin)
+                _, _, chosen = topk_threshold_row(keys[b, g, t].astype(np.float64), c, k)
                 for m in chosen:
                     logG_sel[b, g, t, m] = float(lg[b, g, t, m])
-                tv, ti, again = topk_threshold_row(logG_sel[b, g, t], c, H)
-                assert again == chosen
+                if k == H or n_fin == c:
+                    tv, ti, again = topk_threshold_row(logG_sel[b, g, t], c, H)
+                    assert again == chosen
+                elif k == 0:
+                    tv, ti = math.inf, -1
+                else:
+                    # Every finite block chosen but fewer than H: the least chosen gate and the
+                    # last chosen block holding it, so that no -inf block passes the threshold.
+                    tv = min(float(lg[b, g, t, m]) for m in chosen)
+                    ti = max(m for m in chosen if float(lg[b, g, t, m]) == tv)
+                    tv = 0.0 if tv == 0.0 else tv
                 tau[b, g, t] = tv
                 tidx[b, g, t] = ti
                 sel[b, g, t, : len(chosen)] = chosen

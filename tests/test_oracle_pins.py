@@ -702,3 +702,26 @@ def test_varlen_pin_catches_planted_mistake(monkeypatch):
     monkeypatch.setattr(orc, "gate_normalize_varlen", _bad_gate_normalize_varlen)
     with pytest.raises(AssertionError):
         test_varlen_equals_each_document_alone()
+
+
+def test_select_noisy_on_packed_gates_stays_in_each_document():
+    """Packed gates carry -inf on other documents' blocks: the noisy choice of every row is its own
+    document's (the per-document choice shifted by the document's first block), and the threshold of
+    logG_sel passes exactly the chosen blocks, also on rows whose document has fewer blocks than K-1."""
+    rng = np.random.default_rng(43)
+    block, K = 16, 4
+    docs = [32, 96, 64]
+    cu = np.cumsum([0] + docs)
+    T = int(cu[-1])
+    s = rng.standard_normal((1, 2, T, T // block))
+    lg = orc.gate_normalize_varlen(s, cu, block).astype(np.float32)
+    noise = rng.gumbel(size=lg.shape).astype(np.float32)
+    logG_sel, tau, tidx, sel = orc.select_noisy(lg, noise, K, block)
+    mask = orc.selection_mask(logG_sel, tau, tidx, block)
+    for ts, bs in orc.doc_slices(cu, block):
+        _, _, _, sd = orc.select_noisy(lg[:, :, ts, bs], noise[:, :, ts, bs], K, block)
+        want = np.where(sd >= 0, sd + bs.start, -1)
+        assert np.array_equal(sel[:, :, ts], want)
+    for b, g, t in np.ndindex(*sel.shape[:3]):
+        chosen = [m for m in sel[b, g, t] if m >= 0]
+        assert sorted(np.nonzero(mask[b, g, t])[0].tolist()) == chosen
