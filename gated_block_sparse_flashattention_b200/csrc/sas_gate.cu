@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(256) normalize_select_varlen_kernel(
 // keeps logG on that set and -inf elsewhere, and (tau, tau_idx) is the threshold
 // of logG_sel (the least kept gate and the last kept block holding it), so that
 // the attention calls, which find the selected blocks by thresholding their gate
-// tensor, find exactly this set in logG_sel.
+// tensor, find exactly this set in logG_sel. Blocks with a -inf gate (other
+// documents of a packed sequence) are never chosen.
 // ---------------------------------------------------------------------------
 template <int KREG>
 __global__ void __launch_bounds__(256) select_noisy_kernel(const float* __restrict__ logG,
@@ -300,18 +301,24 @@ __global__ void __launch_bounds__(256) select_noisy_kernel(const float* __restri
   const float* nrow = noise + row * (long long)NB;
   float* dst = logG_sel + row * (long long)NB;
   int32_t* out = sel ? sel + row * (long long)H : nullptr;
+  // A block whose gate is -inf (another document of a packed sequence) is never a
+  // candidate: its key is 0, below every real key.
   float lg[KREG];
   uint32_t keys[KREG];
+  int n_fin = 0;
 #pragma unroll
   for (int i = 0; i < KREG; ++i) {
     const int m = lane + 32 * i;
     lg[i] = (m < c) ? __ldg(lrow + m) : -INFINITY;
-    keys[i] = (m < c) ? float_key(__fadd_rn(lg[i], __ldg(nrow + m))) : 0u;
+    const bool fin = lg[i] != -INFINITY;
+    keys[i] = fin ? float_key(__fadd_rn(lg[i], __ldg(nrow + m))) : 0u;
+    n_fin += fin ? 1 : 0;
   }
+  n_fin = __reduce_add_sync(0xffffffffu, n_fin);
   bool take[KREG];
-  if (min(c, H) == 0 || c <= H) {   // nothing or every historical block
+  if (min(n_fin, H) == 0 || n_fin <= H) {   // nothing, or every block with a gate
 #pragma unroll
-    for (int i = 0; i < KREG; ++i) take[i] = (H > 0) && (lane + 32 * i < c);
+    for (int i = 0; i < KREG; ++i) take[i] = (H > 0) && lg[i] != -INFINITY;
   } else {
     uint32_t tk = 0u;
     int ti = -1;
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(256) select_noisy_kernel(const float* __restri
 #pragma unroll
     for (int i = 0; i < KREG; ++i) {
       const int m = lane + 32 * i;
-      take[i] = m < c && (keys[i] > tk || (keys[i] == tk && m <= ti));
+      take[i] = m < c && keys[i] != 0u && (keys[i] > tk || (keys[i] == tk && m <= ti));
     }
   }
   // Threshold of logG_sel: the least kept gate and the last kept block holding it.
@@ -336,13 +343,13 @@ __global__ void __launch_bounds__(256) select_noisy_kernel(const float* __restri
 #pragma unroll
   for (int o = 16; o; o >>= 1) tix = max(tix, __shfl_xor_sync(0xffffffffu, tix, o));
   if (lane == 0) {
-    if (min(c, H) == 0) {
+    if (min(n_fin, H) == 0) {
       tau[row] = INFINITY;
       tau_idx[row] = -1;
-    } else if (c <= H) {
+    } else if (n_fin == c && c <= H) {   // every historical block
       tau[row] = -INFINITY;
       tau_idx[row] = c - 1;
-    } else {
+    } else {   // the least kept gate and the last kept block holding it
       tau[row] = (tmin == 0.f) ? 0.f : tmin;   // -0 and +0 are one threshold
       tau_idx[row] = tix;
     }

@@ -153,6 +153,10 @@ SAS_API int sas_gate_normalize_select_varlen(const float* s, float* logG, float*
  * sas_fwd / sas_bwd given (logG_sel, tau, tau_idx) attend exactly the chosen blocks
  * with the clean gates logG on them; the gradient they return for logG_sel is the
  * gradient for logG (zero off the chosen blocks), for sas_gate_grad with logG.
+ * Blocks whose gate is -inf (other documents of a packed sequence, from
+ * sas_gate_normalize_select_varlen) are never chosen; a row with fewer gated
+ * blocks than K-1 keeps all of them, with (the least kept gate, the last block
+ * holding it) as its threshold unless they are all its historical blocks.
  * logG, noise, logG_sel: [B,Hkv,T,NB] fp32 (logG_sel may alias neither input);
  * tau [B,Hkv,T] fp32; tau_idx [B,Hkv,T] int32; sel (nullable) [B,Hkv,T,K-1] int32,
  * the chosen blocks ascending, -1 padded. The caller draws the noise.

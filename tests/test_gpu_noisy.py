@@ -28,7 +28,7 @@ def gpu_noisy(logG32, noise32, K):
     return out, tau, tidx, sel
 
 
-def check_noisy(logG32, noise32, K):
+def check_noisy(logG32, noise32, K, same_threshold=True):
     out, tau, tidx, sel = gpu_noisy(logG32, noise32, K)
     r_lg, r_tau, r_tidx, r_sel = orc.select_noisy(logG32, noise32, K, 64)
     assert np.array_equal(out.cpu().numpy().astype(np.float64), r_lg)
@@ -36,6 +36,8 @@ def check_noisy(logG32, noise32, K):
     assert np.array_equal(tidx.cpu().numpy(), r_tidx)
     if K > 1:
         assert np.array_equal(sel.cpu().numpy(), r_sel)
+    if not same_threshold:
+        return out, tau, tidx
     # the threshold of logG_sel is what sas_select_threshold itself finds in it
     t2 = torch.empty_like(tau)
     i2 = torch.empty_like(tidx)
@@ -90,3 +92,28 @@ def test_full_star_forward_backward(w):
                                                                                w.block)[:2], w.block)
     noisy = orc.selection_mask(lg_sel.astype(np.float64), tau.cpu().numpy(), tidx.cpu().numpy(), w.block)
     assert (clean != noisy).any()
+
+
+def test_full_star_on_a_packed_sequence():
+    """Noisy selection on packed gates: each row chooses inside its own document, and the attention calls
+    on the result match the oracle's (on the packed tensors, the chosen set held fixed)."""
+    w = workloads.custom("noisy_packed", "bf16", B=1, Hq=8, Hkv=2, d=128, T=2048, K=8)
+    cu = [0, 512, 576, 1600, 2048]
+    inp = workloads.make_training_inputs(w, seed=6)
+    s = dev(inp["s"])
+    logG = torch.empty_like(s)
+    t0 = torch.empty(1, 2, 2048, device="cuda")
+    i0 = torch.empty(1, 2, 2048, dtype=torch.int32, device="cuda")
+    binding.sas_gate_normalize_select_varlen(s, logG, t0, i0, None, w.K, cu)
+    torch.cuda.synchronize()
+    lg32 = logG.cpu().numpy()
+    noise32 = np.random.default_rng(11).gumbel(0.0, 1.0, lg32.shape).astype(np.float32)
+    out, tau, tidx = check_noisy(lg32, noise32, w.K, same_threshold=False)
+    lg_sel = out.cpu().numpy()
+    mask = orc.selection_mask(lg_sel.astype(np.float64), tau.cpu().numpy(), tidx.cpu().numpy(), w.block)
+    for ts, bs in orc.doc_slices(cu, w.block):
+        inside = np.zeros(mask.shape[-1], bool)
+        inside[bs] = True
+        assert not mask[:, :, ts][..., ~inside].any()
+    assert mask.sum(-1).max() <= w.K - 1
+    check_full(w, inp, lg_sel, tau.cpu().numpy(), tidx.cpu().numpy())

@@ -4,7 +4,8 @@ The packed gates and selection come from sas_gate_normalize_select_varlen; the
 attention calls and the selector gradient run unchanged on them. Gates within
 2e-5 of the oracle; the selection (as the set the threshold keeps) bit-exact
 against the oracle's per-document Top-K on the GPU's own fp32 gates; forward and
-backward within the bf16 tolerances of the other parity tests."""
+backward within the tolerances of the other parity tests (bf16: 2e-2 max-abs on
+O, 1e-2 relative L2 on the gradients; fp32: 1e-4)."""
 
 import numpy as np
 import pytest
@@ -82,6 +83,7 @@ def test_varlen_one_document_is_the_plain_fused_call():
 @pytest.mark.parametrize("w,docs", [
     (workloads.custom("varlen_g4", "bf16", B=1, Hq=8, Hkv=2, d=128, T=2048, K=4), [512, 64, 1024, 448]),
     (workloads.custom("varlen_g8_k8", "bf16", B=2, Hq=8, Hkv=1, d=128, T=1536, K=8), [768, 192, 576]),
+    (workloads.custom("varlen_f32", "f32", B=1, Hq=4, Hkv=1, d=64, T=768, K=3), [128, 448, 192]),
 ], ids=lambda x: getattr(x, "name", "docs"))
 def test_varlen_forward_backward_and_gate_grad(w, docs):
     cu = np.cumsum([0] + docs).tolist()
@@ -95,10 +97,11 @@ def test_varlen_forward_backward_and_gate_grad(w, docs):
     lg64 = logG.cpu().numpy().astype(np.float64)
     ref = orc.forward_backward_varlen(*(to_np(inp[k]) for k in ("Q", "K", "V", "dO")), lg64, w.K, cu, w.block,
                                       w.sm_scale)
-    assert max_abs(to_np(O), ref["O"]) <= 2e-2
-    assert max_abs(to_np(LSE), ref["LSE"]) <= 1e-2
+    tol = {"bf16": (2e-2, 1e-2, 1e-2), "f32": (1e-4, 1e-4, 1e-4)}[w.dtype]
+    assert max_abs(to_np(O), ref["O"]) <= tol[0]
+    assert max_abs(to_np(LSE), ref["LSE"]) <= tol[1]
     for name, got in (("dQ", dQ), ("dK", dK), ("dV", dV), ("dLogG", dLogG)):
-        assert rel_l2(to_np(got), ref[name]) <= 1e-2, (name, rel_l2(to_np(got), ref[name]))
+        assert rel_l2(to_np(got), ref[name]) <= tol[2], (name, rel_l2(to_np(got), ref[name]))
     mask = orc.selection_mask_varlen(lg64, w.K, cu, w.block)
     assert np.all(to_np(dLogG)[~mask] == 0.0)
     # selector-score gradient, document by document, against the oracle's Jacobian product
