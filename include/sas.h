@@ -16,7 +16,16 @@
  *     backward pass (Appendix E "Backward pass"; Appendix D.1 eq. 5);
  *   * decoding selects Top-(K-1) historical blocks by score and runs ungated
  *     attention over them and the current block (§4.3 Algorithm 2; §5.1
- *     "Inference implementation").
+ *     "Inference implementation"), from a contiguous or a paged KV cache;
+ *   * around the path: the gradient with respect to the selector scores
+ *     (Appendix D.3), the noisy "full*" selection (§4.1, Table 1), and packed
+ *     sequences of documents (§5.1).
+ *
+ * Entry points: sas_gate_normalize, sas_select_threshold and their fused form
+ * sas_gate_normalize_select (and _varlen for packed documents), sas_select_noisy,
+ * sas_fwd, sas_bwd, sas_gate_grad, sas_decode_fwd (and _paged, _static), the
+ * workspace sizes, the device status word, sas_status_string, sas_version and
+ * sas_launch_count.
  *
  * Conventions shared by every call
  * --------------------------------
