@@ -41,8 +41,8 @@ from gated_block_sparse_flashattention_b200 import workloads  # noqa: E402
 # (sha256 prefixes); after any change they read as unmeasured (null).
 MEASURED_TRAFFIC = {
     "sas_bwd": (2507901696, {"sas_bwd_gather.cu": "f87675f7247ad878", "sas_common.cuh": "d3c29d493fc4dfcf"}),
-    "decode": (67355136, {"sas_decode.cu": "4ebaf9cb8b725287", "sas_common.cuh": "d3c29d493fc4dfcf"}),
-    "decode_paged": (68085760, {"sas_decode.cu": "4ebaf9cb8b725287", "sas_common.cuh": "d3c29d493fc4dfcf"}),
+    "decode": (67355136, {"sas_decode.cu": "fe0147b988941a3e", "sas_common.cuh": "d3c29d493fc4dfcf"}),
+    "decode_paged": (68085760, {"sas_decode.cu": "fe0147b988941a3e", "sas_common.cuh": "d3c29d493fc4dfcf"}),
 }
 
 

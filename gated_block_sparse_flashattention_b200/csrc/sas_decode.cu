@@ -8,13 +8,15 @@
 // bf16 storage, three kernels:
 //   decode_select_kernel    one warp (one CTA) per (b, g): Top-(K-1) of the score
 //                           row; the attended list [c, selected blocks] goes to
-//                           the workspace.
+//                           the workspace (rows over 1024 blocks:
+//                           decode_select_radix_kernel, one 512-thread CTA per
+//                           (b, g)); for a paged cache also each block's page.
 //   decode_fused_mma_kernel persistent, two 4-warp CTAs per SM, each walking a
 //                           contiguous run of items (b, g, attended block) with a
 //                           3-stage TMA ring; the G heads' scores and P V run as
 //                           m16n8k16 MMAs (fp32 accumulation); the items of one
 //                           (b, g) are folded online and leave one fp32 partial.
-//   decode_merge_kernel     one CTA per (b, g): merges the partials into o.
+//   decode_merge_kernel<S>  one CTA per (b, g): merges the partials into o.
 // The second and third are programmatic dependents of the one before them.
 // fp32 storage: decode_select_kernel, then decode_attn_kernel<float> (one
 // 128-thread CTA per item on the CUDA cores, one bulk copy each for K and V),
