@@ -513,14 +513,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 constexpr int kChunkRows = 256;
 
 // Calls f(t, m) for every selected historical block m of every position t of the
-// chunk. One warp per group of 4 positions (blocks strided over the lanes): the
-// loads of the 4 rows are issued together, so a warp pays one round trip per
-// group instead of one per row.
+// chunk. One warp per group of 4 positions (blocks strided over the lanes, 128
+// blocks per pass): the loads of the 4 rows' 128-block spans are issued together,
+// so a warp pays one round trip per group and pass instead of one per row and
+// 32 blocks.
 template <typename F>
 __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, const float* __restrict__ tau,
                                               const int32_t* __restrict__ tau_idx, long long bg, int t0, int T,
                                               int NB, F&& f) {
-  constexpr int R = 4;
+  constexpr int R = 4, U = 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
   const int t_end = min(T, t0 + kChunkRows);
   for (int tb = t0 + warp * R; tb < t_end; tb += n_warps * R) {
@@ -534,14 +535,21 @@ __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, co
       ti[r] = c[r] ? tau_idx[bg * T + t] : 0;
     }
     const int cmax = max(max(c[0], c[1]), max(c[2], c[3]));
-    for (int m0 = 0; m0 < cmax; m0 += 32) {
-      const int m = m0 + lane;
-      float x[R];
+    for (int m0 = 0; m0 < cmax; m0 += 32 * U) {
+      float x[U][R];
 #pragma unroll
-      for (int r = 0; r < R; ++r) x[r] = (m < c[r]) ? logG[(bg * T + tb + r) * (long long)NB + m] : 0.f;
+      for (int u = 0; u < U; ++u) {
+        const int m = m0 + 32 * u + lane;
 #pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (m < c[r] && (x[r] > tv[r] || (x[r] == tv[r] && m <= ti[r]))) f(tb + r, m);
+        for (int r = 0; r < R; ++r) x[u][r] = (m < c[r]) ? logG[(bg * T + tb + r) * (long long)NB + m] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int m = m0 + 32 * u + lane;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (m < c[r] && (x[u][r] > tv[r] || (x[u][r] == tv[r] && m <= ti[r]))) f(tb + r, m);
+      }
     }
   }
 }
