@@ -421,15 +421,20 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const float* __restrict
     const float tv = tau[row];
     const int ti = tau_idx[row];
     const float* v = logG + row * (long long)NB;
-    for (int base = 0; base < c; base += 32) {
-      const int m = base + lane;
-      bool sel = false;
-      if (m < c) {
-        const float x = v[m];
-        sel = (x > tv) || (x == tv && m <= ti);
+    for (int base = 0; base < c; base += 128) {   // four 32-block spans per round trip
+      float x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = base + 32 * u + lane;
+        x[u] = (m < c) ? v[m] : 0.f;
       }
-      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0 && bal) atomicOr(&words[base >> 5], bal);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = base + 32 * u + lane;
+        const bool sel = m < c && ((x[u] > tv) || (x[u] == tv && m <= ti));
+        const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0 && bal) atomicOr(&words[(base >> 5) + u], bal);
+      }
     }
   }
   __syncthreads();
