@@ -1,18 +1,21 @@
 """Benchmark of the SAS hot path on B200.
 
 One step = one pass of the whole training-side path over one batch of the
-Qwen3-4B-like layer (B=1, Hq=32, Hkv=8, d=128, T=8192, block 64, K=16 blocks):
-gate normalisation fused with Top-K threshold selection, forward, backward
-(dQ/dK/dV/dLogG) and the selector-score gradient ds. The metric is attended-block TFLOP/s: 4*d*sum_rows(n_t) for
-the forward and 2.5x that for the backward, n_t = (t mod 64) + 1 + 64*min(K-1, c_t)
-attended keys of row t. The memory-bound decode step (16 sequences over a
-32768-token cache) is reported beside it in GB/s.
+Qwen3-8B-like layer (B=2, Hq=32, Hkv=8, d=128, T=32768, block 64, K=32 blocks,
+Student-t selector scores): gate normalisation fused with Top-K threshold
+selection, forward, backward (dQ/dK/dV/dLogG) and the selector-score gradient
+ds. The metric is attended-block TFLOP/s: 4*d*sum_rows(n_t) for the forward and
+2.5x that for the backward, n_t = (t mod 64) + 1 + 64*min(K-1, c_t) attended keys
+of row t. The same step on the Qwen3-4B-like layer (T=8192, K=16) and the
+Qwen3-14B-like layer (T=65536, K=16) is reported in "legs", and the
+memory-bound decode step (16 sequences over a 32768-token cache) in GB/s.
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-Multi-GPU: launched by torchrun, one process per GPU; each rank runs its own
-batch of the same shape (no collective on the data path: the work splits into
-independent (batch, KV-group) units), timings are reduced with max over ranks.
+Multi-GPU: launched by torchrun, one process per GPU; each rank runs a replica
+of the step on its own batch (inputs seeded by the rank; no collective on the
+data path: the work splits into independent (batch, KV-group) units), and the
+timed region is reduced with max over ranks.
 """
 
 from __future__ import annotations
@@ -58,10 +61,12 @@ def measured_traffic(name: str):
     return nbytes
 
 
-BENCH_WORKLOAD = "qwen3_4b_t8k"
+BENCH_WORKLOAD = "qwen3_8b_t32k"
+LEG_WORKLOADS = ("qwen3_4b_t8k", "qwen3_14b_t64k")
+VARLEN_WORKLOAD = "qwen3_4b_t8k"
 DECODE_WORKLOAD = "decode_b16_l32k"
 PAGED_DECODE_WORKLOAD = "decode_b8_l512k_paged"
-VARLEN_DOCS = [512, 1536, 1024, 2048, 3072]   # documents packed into the bench layer's 8192 positions
+VARLEN_DOCS = [512, 1536, 1024, 2048, 3072]   # documents packed into the Qwen3-4B-like layer's 8192 positions
 METRIC = "fwd+bwd attended-block TFLOP/s (normalise+select+fwd+bwd+gate-grad step)"
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2, written between timed steps
 
@@ -87,13 +92,25 @@ def attended_flops(w) -> tuple[float, float]:
     return fwd, 2.5 * fwd
 
 
+SLOT_BUDGET = 8 << 30   # bytes of forward partials per batch of (b, g) groups
+
+
+def fwd_uses_gather(w) -> bool:
+    """Whether sas_fwd runs the KV-block-outer forward (per-pair partials of one (b, g) within the slot budget:
+    T * min(K, NB+1) slots of G x (128 bf16 + one fp32)) or the q-tile union forward."""
+    slots = 1 + max(0, min(w.K - 1, w.NB))
+    return w.T * slots * w.G * (128 * 2 + 4) <= SLOT_BUDGET
+
+
 def executed_flops(w, sel):
     """(forward, backward) FLOPs the tensor cores execute for one step, from the selection sel [B,Hkv,T,K-1].
 
-    Forward: every q-tile (P positions x G heads = 128 rows) runs S = Q K^T and O += P V (128 x 64 x 128 MACs
-    each) over its block list: the current block(s) plus the union of its rows' selected blocks. Backward: the
-    CTA of block j runs 5 MMAs of 128 x 64 x 128 MACs per tile of P positions over the positions that attend j
-    (its own 64 and those that selected it). The ratio to the attended FLOPs is the waste of the tiling.
+    KV-block-outer kernels (the backward, and the forward when its partials fit the slot budget): the CTA of
+    block j runs its MMAs per tile of P positions x G heads (up to 128 rows) over the positions that attend j
+    (its own 64 and those that selected it): 2 MMAs of 128 x 64 x 128 MACs per tile for the forward (S and P V),
+    5 for the backward. The q-tile union forward: every q-tile (P positions x G heads) runs S = Q K^T and
+    O += P V over its block list, the current block(s) plus the union of its rows' selected blocks. The ratio
+    to the attended FLOPs is the waste of the tiling.
     """
     G = w.G
     P = (128 // G) & ~7
@@ -110,13 +127,15 @@ def executed_flops(w, sel):
     t0 = torch.arange(n_pt, device=sel.device) * P
     t1 = torch.clamp(t0 + P, max=T) - 1
     n_cur = (t1 // w.block - t0 // w.block + 1).to(torch.float64)
-    fwd = float((hit[:, :, 1:].sum(-1).to(torch.float64) + n_cur).sum()) * 2 * mma
+    fwd_union = float((hit[:, :, 1:].sum(-1).to(torch.float64) + n_cur).sum()) * 2 * mma
+    del hit
     counts = torch.zeros(nbg, w.NB + 1, dtype=torch.float64, device=sel.device)
     counts.scatter_add_(1, sel.reshape(nbg, T * H).long() + 1, torch.ones(nbg, T * H, dtype=torch.float64,
                                                                         device=sel.device))
     own = torch.clamp(T - torch.arange(w.NB, device=sel.device) * w.block, max=w.block).to(torch.float64)
-    tiles = torch.ceil((counts[:, 1:] + own) / P)
-    bwd = float(tiles.sum()) * 5 * mma
+    tiles = float(torch.ceil((counts[:, 1:] + own) / P).sum())
+    fwd = tiles * 2 * mma if fwd_uses_gather(w) else fwd_union
+    bwd = tiles * 5 * mma
     return fwd, bwd
 
 
@@ -182,9 +201,15 @@ def dist_env():
     return world, rank, local
 
 
-def shard_units(n_units: int, rank: int, world: int) -> list[int]:
-    """Round-robin assignment of independent (batch, KV-group) units to ranks."""
-    return list(range(rank, n_units, world))
+def rank_inputs(w, rank: int):
+    """The batch one rank works on: the workload's seeded inputs with the rank as the seed (every rank a
+    replica of the step on its own data)."""
+    return workloads.make_training_inputs(w, seed=rank)
+
+
+def job_throughput(flops_per_step: float, steps: int, max_total_ms: float, world: int) -> float:
+    """Whole-job TFLOP/s: every rank's steps, over the slowest rank's timed region."""
+    return world * flops_per_step * steps / (max_total_ms * 1e-3) / 1e12
 
 
 def reduce_max(value: float, device=None) -> float:
@@ -325,6 +350,116 @@ def oracle_sample(w, seconds: float, seed: int = 0):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def workload_desc(w) -> str:
+    dist = {"normal": "s~N(0,1)", "normal2_planted3": "s~N(0,2) + 3 planted blocks per query",
+            "student_t3": "s~Student-t(nu=3)"}[w.s_dist]
+    return (f"{w.name} layer fwd+bwd: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} T={w.T} block={w.block} K={w.K} "
+            f"({w.K * w.block}-token budget), {dist}")
+
+
+def run_training(w, args, device, stream, binding, peaks, rank, world, host=None, noisy=False):
+    """Times the training step (fused normalise+select, fwd, bwd, selector gradient) of workload w with inputs
+    resident in HBM, a 512 MiB L2 flush between steps outside the events. Returns (result dict, host inputs)."""
+    fwd_flops, bwd_flops = attended_flops(w)
+    step_flops = fwd_flops + bwd_flops
+    if host is None:
+        host = rank_inputs(w, rank)
+    Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
+    logG = torch.empty_like(s)
+    tau = torch.empty(w.B, w.Hkv, w.T, device=device)
+    tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(w.B, w.Hq, w.T, device=device)
+    dQ, dK, dV, dLogG = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s)
+    ds = torch.empty_like(s)
+    ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
+    ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        binding.sas_gate_normalize_select(s, logG, tau, tidx, None, w.K, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream)
+        if ev:
+            ev[2].record(stream)
+        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
+                        stream=stream)
+        if ev:
+            ev[3].record(stream)
+        binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    if binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b):
+        raise RuntimeError(f"kernel-side error during warm-up of {w.name}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    launches0 = binding.launch_count()
+    for i in range(args.steps):
+        flush.zero_()      # L2 flush between timed steps (outside the events)
+        step(evs[i])
+    torch.cuda.synchronize(device)
+    launches = binding.launch_count() - launches0
+    barrier(device)
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    gate_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    grad_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    total_ms = reduce_max(sum(step_ms), device)
+    status = binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b)
+
+    # Dominant call against the tensor-core roofline.
+    bwd_avg = statistics.mean(bwd_ms)
+    fwd_avg = statistics.mean(fwd_ms)
+    dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
+        ("sas_fwd", fwd_avg, fwd_flops)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    sel = torch.empty(w.B, w.Hkv, w.T, w.K - 1, dtype=torch.int32, device=device)
+    binding.sas_select_threshold(logG, tau, tidx, sel, w.K, stream=stream)
+    torch.cuda.synchronize(device)
+    ex_fwd, ex_bwd = executed_flops(w, sel)
+    del sel
+    gate_avg = statistics.mean(gate_ms)
+    grad_avg = statistics.mean(grad_ms)
+    traffic_key = f"{dom_name}:{w.name}"
+    roofline = {"bound": "tensor", "kernel": f"{dom_name} call", "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": measured_traffic(traffic_key) if traffic_key in MEASURED_TRAFFIC else None,
+                "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
+                "fwd_path": "kv-block outer, per-pair partials + merge" if fwd_uses_gather(w) else "q-tile union",
+                "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
+                "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
+                "fwd_executed_tflops": round(ex_fwd / (fwd_avg * 1e-3) / 1e12, 2),
+                "fwd_inflation": round(ex_fwd / fwd_flops, 3),
+                "bwd_tflops": round(bwd_flops / (bwd_avg * 1e-3) / 1e12, 2),
+                "bwd_executed_tflops": round(ex_bwd / (bwd_avg * 1e-3) / 1e12, 2),
+                "bwd_inflation": round(ex_bwd / bwd_flops, 3),
+                "gate_select_ms": round(gate_avg, 4),
+                "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1),
+                "gate_grad_ms": round(grad_avg, 4),
+                "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1)}
+    if noisy:
+        noisy_ms = time_noisy_select(w, logG, flush, stream, binding, device)
+        roofline["noisy_select_ms"] = round(noisy_ms, 4)
+        roofline["noisy_select_gbs"] = round(noisy_select_bytes(w) / (noisy_ms * 1e-3) / 1e9, 1)
+    res = {"workload": workload_desc(w), "value": round(job_throughput(step_flops, args.steps, total_ms, world), 3),
+           "unit": "TFLOP/s", "ms_per_step": round(total_ms / args.steps, 4),
+           "attended_gflop_per_step": round(step_flops / 1e9, 2), "gpu_launches": launches,
+           "device_status": status, "roofline": roofline}
+    return res, host
+
+
 def run_gpu(args):
     from gated_block_sparse_flashattention_b200 import binding
 
@@ -340,127 +475,50 @@ def run_gpu(args):
     fwd_flops, bwd_flops = attended_flops(w)
     step_flops = fwd_flops + bwd_flops
     peaks = measured_peaks()
-
-    # Inputs: this rank's own batch (seeded by rank), resident in HBM before timing.
-    host = workloads.make_training_inputs(w, seed=rank)
-    Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
-    logG = torch.empty_like(s)
-    tau = torch.empty(w.B, w.Hkv, w.T, device=device)
-    tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
-    O = torch.empty_like(Q)
-    LSE = torch.empty(w.B, w.Hq, w.T, device=device)
-    dQ, dK, dV, dLogG = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s)
-    ds = torch.empty_like(s)
-    ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
-    ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        binding.sas_gate_normalize_select(s, logG, tau, tidx, None, w.K, stream=stream)
-        if ev:
-            ev[1].record(stream)
-        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.sm_scale, ws_f, stream=stream)
-        if ev:
-            ev[2].record(stream)
-        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
-                        stream=stream)
-        if ev:
-            ev[3].record(stream)
-        binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
-        if ev:
-            ev[4].record(stream)
-
     legs = set(args.legs.split(","))
     clk = ClockSampler(local).__enter__()   # running through every leg; samples kept while active
     time.sleep(0.3)
+    clk.active = True
+
+    head, host = None, None
     if "step" in legs:
-        clk.active = True
-        for _ in range(args.warmup):
-            flush.zero_()
-            step()
-        torch.cuda.synchronize(device)
-        if binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b):
-            raise RuntimeError("kernel-side timeout during warm-up")
-
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-        barrier(device)
-        torch.cuda.synchronize(device)
-        launches0 = binding.launch_count()
-        for i in range(args.steps):
-            flush.zero_()      # L2 flush between timed steps (outside the events)
-            step(evs[i])
-        torch.cuda.synchronize(device)
-        launches = binding.launch_count() - launches0
-        barrier(device)
-        step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-        fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-        bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
-        gate_ms = [e[0].elapsed_time(e[1]) for e in evs]
-        grad_ms = [e[3].elapsed_time(e[4]) for e in evs]
-        total_ms = reduce_max(sum(step_ms), device)
-        ms_per_step = total_ms / args.steps
-        value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
-
-        # Dominant call (the backward) against the tensor-core roofline.
-        bwd_avg = statistics.mean(bwd_ms)
-        fwd_avg = statistics.mean(fwd_ms)
-        dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
-            ("sas_fwd", fwd_avg, fwd_flops)
-        achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-        sel = torch.empty(w.B, w.Hkv, w.T, w.K - 1, dtype=torch.int32, device=device)
-        binding.sas_select_threshold(logG, tau, tidx, sel, w.K, stream=stream)
-        torch.cuda.synchronize(device)
-        ex_fwd, ex_bwd = executed_flops(w, sel)
-        del sel
-        noisy_ms = time_noisy_select(w, logG, flush, stream, binding, device)
-        gate_avg = statistics.mean(gate_ms)
-        grad_avg = statistics.mean(grad_ms)
-        roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 2),
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": round(achieved / peaks["bf16_tflops"], 4),
-                    "traffic": measured_traffic(dom_name) if dom_name == "sas_bwd" else None,
-                    "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
-                    "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
-                    "fwd_tflops": round(fwd_flops / (fwd_avg * 1e-3) / 1e12, 2),
-                    "fwd_executed_tflops": round(ex_fwd / (fwd_avg * 1e-3) / 1e12, 2),
-                    "fwd_inflation": round(ex_fwd / fwd_flops, 3),
-                    "bwd_executed_tflops": round(ex_bwd / (bwd_avg * 1e-3) / 1e12, 2),
-                    "bwd_inflation": round(ex_bwd / bwd_flops, 3),
-                    "gate_select_ms": round(gate_avg, 4),
-                    "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1),
-                    "gate_grad_ms": round(grad_avg, 4),
-                    "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1),
-                    "noisy_select_ms": round(noisy_ms, 4),
-                    "noisy_select_gbs": round(noisy_select_bytes(w) / (noisy_ms * 1e-3) / 1e9, 1)}
-    else:
-        value, ms_per_step, launches, roofline = None, None, 0, None
+        head, host = run_training(w, args, device, stream, binding, peaks, rank, world, noisy=True)
+        torch.cuda.empty_cache()
+    other = {}
+    if "legs" in legs:
+        for name in LEG_WORKLOADS:
+            other[name], _ = run_training(workloads.WORKLOADS[name], args, device, stream, binding, peaks, rank,
+                                          world)
+            torch.cuda.empty_cache()
 
     # End to end through the C ABI from pinned host buffers, results copied back.
-    clk.active = True
+    if "e2e" in legs and host is None:
+        host = rank_inputs(w, rank)
     e2e = run_e2e(args, w, host, device, stream, binding, step_flops, world) if "e2e" in legs else None
+    host = None
+    torch.cuda.empty_cache()
     dec = run_decode(args, device, stream, binding, peaks, clk) if "decode" in legs else None
     dec_paged = run_decode_paged(args, device, stream, binding, peaks, clk) if "paged" in legs else None
-    varlen = run_varlen(args, w, host, device, stream, binding, flush) if "varlen" in legs else None
+    varlen = run_varlen(args, device, stream, binding, rank) if "varlen" in legs else None
     clk.active = False
     clk.__exit__(None, None, None)
 
     result = {
         "metric": METRIC,
-        "value": round(value, 3) if value is not None else None, "unit": "TFLOP/s", "n_gpus": world,
+        "value": head["value"] if head else None, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 4) if ms_per_step is not None else None, "higher_is_better": True,
+        "ms_per_step": head["ms_per_step"] if head else None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "qwen3_4b_t8k layer fwd+bwd: B=1 Hq=32 Hkv=8 d=128 T=8192 block=64 K=16 "
-                               "(1024-token budget), s~N(0,2) + 3 planted blocks per query",
-                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world} (independent batches)",
+        "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"dp{world} (replicas on independent batches)",
                    "l2": "flushed between timed steps (512 MiB write, outside the timed events)",
                    "attended_gflop_per_step": round(step_flops / 1e9, 2)},
-        "roofline": roofline,
+        "roofline": head["roofline"] if head else None,
         "e2e": e2e,
-        "gpu_launches": launches,
+        "gpu_launches": head["gpu_launches"] if head else 0,
+        "device_status": head["device_status"] if head else None,
+        "legs": other,
         "decode": dec,
         "decode_paged": dec_paged,
         "varlen": varlen,
@@ -477,10 +535,12 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_varlen(args, w, host, device, stream, binding, flush):
-    """The training step on a packed sequence: the bench layer's 8192 positions as five documents of
+def run_varlen(args, device, stream, binding, rank):
+    """The training step on a packed sequence: the Qwen3-4B-like layer's 8192 positions as five documents of
     512, 1536, 1024, 2048 and 3072 tokens (varlen gates and selection, then the unchanged forward, backward
     and selector gradient), device-resident inputs, L2 flushed between steps outside the events."""
+    w = workloads.WORKLOADS[VARLEN_WORKLOAD]
+    host = rank_inputs(w, rank)
     docs = VARLEN_DOCS
     cu = np.cumsum([0] + docs).tolist()
     Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
@@ -490,12 +550,13 @@ def run_varlen(args, w, host, device, stream, binding, flush):
     O, LSE = torch.empty_like(Q), torch.empty(w.B, w.Hq, w.T, device=device)
     dQ, dK, dV, dLogG, ds = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s),
                              torch.empty_like(s))
-    ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, 1), device)
+    ws_f = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
     ws_b = binding.workspace(binding.sas_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1), device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     def step():
         binding.sas_gate_normalize_select_varlen(s, logG, tau, tidx, None, w.K, cu, stream=stream)
-        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.sm_scale, ws_f, stream=stream)
+        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream)
         binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
                         stream=stream)
         binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
@@ -516,7 +577,7 @@ def run_varlen(args, w, host, device, stream, binding, flush):
     ms = statistics.mean(a.elapsed_time(b) for a, b in times)
     fwd, bwd = attended_flops_varlen(w, docs)
     status = binding.sas_device_status(ws_f) or binding.sas_device_status(ws_b)
-    return {"workload": f"qwen3_4b_t8k packed as documents of {docs} tokens", "ms_per_step": round(ms, 4),
+    return {"workload": f"{w.name} packed as documents of {docs} tokens", "ms_per_step": round(ms, 4),
             "value": round((fwd + bwd) / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "attended_gflop_per_step": round((fwd + bwd) / 1e9, 2), "device_status": status}
 
@@ -537,8 +598,8 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
         for k, v in pinned.items():
             dev_in[k].copy_(v, non_blocking=True)
         logG, tau, tidx, _ = binding.gate_and_select(dev_in["s"], w.K, stream=stream)
-        O, LSE = binding.forward(dev_in["Q"], dev_in["K"], dev_in["V"], logG, tau, tidx, w.sm_scale, stream=stream,
-                                 check=False)
+        O, LSE = binding.forward(dev_in["Q"], dev_in["K"], dev_in["V"], logG, tau, tidx, w.K, w.sm_scale,
+                                 stream=stream, check=False)
         dQ, dK, dV, dLogG = binding.backward(dev_in["Q"], dev_in["K"], dev_in["V"], O, dev_in["dO"], logG, tau,
                                              tidx, LSE, w.K, w.sm_scale, stream=stream, check=False)
         ds = binding.gate_grad(logG, dLogG, stream=stream)
@@ -558,7 +619,7 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
         b.synchronize()
         times.append(a.elapsed_time(b))
     total = reduce_max(sum(times), device)
-    return {"value": round(world * step_flops * args.steps / (total * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    return {"value": round(job_throughput(step_flops, args.steps, total, world), 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(total / args.steps, 4)}
 
 
@@ -681,7 +742,7 @@ def run_reference(args):
         "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "qwen3_4b_t8k layer fwd+bwd: B=1 Hq=32 Hkv=8 d=128 T=8192 block=64 K=16"},
+        "config": {"workload": workload_desc(w)},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -695,10 +756,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--legs", default="step,e2e,decode,paged,varlen,cpu",
-                    help="comma list of what to measure and report: step (device-resident timed steps), e2e "
-                         "(host buffers through the C ABI), decode, paged (long-context paged decode), varlen (packed "
-                         "documents), cpu (oracle baseline)")
+    ap.add_argument("--legs", default="step,legs,e2e,decode,paged,varlen,cpu",
+                    help="comma list of what to measure and report: step (device-resident timed steps of the "
+                         "headline layer), legs (the same step on the 8K and 64K layers), e2e (host buffers through "
+                         "the C ABI), decode, paged (long-context paged decode), varlen (packed documents), cpu "
+                         "(oracle baseline)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3

@@ -29,6 +29,7 @@ _SIGNATURES = {
     "sas_status_string": (ctypes.c_char_p, [_c_int]),
     "sas_version": (_c_int, []),
     "sas_launch_count": (ctypes.c_uint64, []),
+    "sas_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "sas_gate_normalize": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_normalize_select": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -36,10 +37,10 @@ _SIGNATURES = {
     "sas_gate_normalize_select_varlen": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_vp, _c_int, _vp]),
     "sas_select_noisy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_grad": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
-    "sas_fwd_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
+    "sas_fwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_bwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_decode_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
-    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_f, _vp, _sz, _vp]),
+    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_f, _vp, _sz, _vp]),
     "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7
                 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
@@ -48,6 +49,7 @@ _SIGNATURES = {
                                       _vp] + [_c_int] * 6 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd_static": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                               + [_c_f, _vp]),
+    "sas_decode_static_status": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int32)]),
     "sas_device_status": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "sas_device_status_clear": (_c_int, [_vp, _vp]),
 }
@@ -111,6 +113,11 @@ def launch_count() -> int:
     return int(lib().sas_launch_count())
 
 
+def set_wait_limit_ns(ns: int) -> int:
+    """Limit of each bounded wait in the fwd/bwd tensor-core kernels (0: the 1 s default); returns the old one."""
+    return int(lib().sas_set_wait_limit_ns(int(ns)))
+
+
 def status_string(status: int) -> str:
     return lib().sas_status_string(status).decode()
 
@@ -160,8 +167,8 @@ def _ws_size(name, *args) -> int:
     return out.value
 
 
-def sas_fwd_workspace_size(B, Hq, Hkv, T, d, dtype_code, block=BLOCK) -> int:
-    return _ws_size("sas_fwd_workspace_size", B, Hq, Hkv, T, d, block, dtype_code)
+def sas_fwd_workspace_size(B, Hq, Hkv, T, d, K, dtype_code, block=BLOCK) -> int:
+    return _ws_size("sas_fwd_workspace_size", B, Hq, Hkv, T, d, block, K, dtype_code)
 
 
 def sas_bwd_workspace_size(B, Hq, Hkv, T, d, K, dtype_code, block=BLOCK) -> int:
@@ -177,12 +184,13 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, sm_scale, ws, block=BLOCK, stream=None):
+def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block=BLOCK, stream=None):
     B, Hq, T, d = Q.shape
     Hkv = K.shape[1]
     _check("sas_fwd", lib().sas_fwd(
         _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(O), _ptr(LSE),
-        B, Hq, Hkv, T, d, block, float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+        B, Hq, Hkv, T, d, block, int(Kbudget), float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block=BLOCK,
@@ -230,6 +238,13 @@ def sas_decode_fwd_static(q, Kc, Vc, seqlen, s, K, o, sm_scale, sel_out=None, ap
         _ptr(o), _ptr(sel_out), B, Hq, Hkv, Lmax, NBmax, d, block, float(sm_scale), _stream(stream)))
 
 
+def sas_decode_static_status(stream=None) -> int:
+    """Status word of the last sas_decode_fwd_static call on the current device (0: no kernel-side error)."""
+    out = ctypes.c_int32(0)
+    lib().sas_decode_static_status(_stream(stream), ctypes.byref(out))
+    return out.value
+
+
 def sas_device_status(ws, stream=None) -> int:
     out = ctypes.c_int32(0)
     lib().sas_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
@@ -267,15 +282,15 @@ def _check_device_status(fn, ws, stream):
         raise SasError(fn, -4)
 
 
-def forward(Q, K, V, logG, tau, tau_idx, sm_scale, block=BLOCK, stream=None, ws=None, check=True):
+def forward(Q, K, V, logG, tau, tau_idx, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None, check=True):
     """O, LSE of ``sas_fwd``. With ``check`` the stream is synchronised and the
-    kernel status word is read (raises ``SasError`` on a kernel-side timeout)."""
+    kernel status word is read (raises ``SasError`` on a kernel-side error)."""
     B, Hq, T, d = Q.shape
     O = torch.empty_like(Q)
     LSE = torch.empty(B, Hq, T, dtype=torch.float32, device=Q.device)
     if ws is None:
-        ws = workspace(sas_fwd_workspace_size(B, Hq, K.shape[1], T, d, _dtype_code(Q), block), Q.device)
-    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, sm_scale, ws, block, stream)
+        ws = workspace(sas_fwd_workspace_size(B, Hq, K.shape[1], T, d, Kbudget, _dtype_code(Q), block), Q.device)
+    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block, stream)
     if check:
         _check_device_status("sas_fwd", ws, stream)
     return O, LSE

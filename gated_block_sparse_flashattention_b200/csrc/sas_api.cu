@@ -12,6 +12,10 @@ namespace sas {
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// 1 s unless sas_set_wait_limit_ns() changed it.
+static std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 QTileShape qtile_shape(int G, int T, int NB) {
   QTileShape s;
   s.P = (128 / G) & ~7;
@@ -80,6 +84,11 @@ const char* sas_status_string(int status) {
 int sas_version(void) { return 100; }
 
 uint64_t sas_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+uint64_t sas_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t v = ns == 0 ? 1000000000ull : ns;
+  return g_wait_limit_ns.exchange(v, std::memory_order_relaxed);
+}
 
 int sas_gate_normalize(const float* s, float* logG, int B, int Hkv, int T, int NB, int block, void* stream) {
   if (!s || !logG || !aligned16(s) || !aligned16(logG) || s == logG) return SAS_ERR_INVALID_ARG;
@@ -154,11 +163,15 @@ int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int B, int H
   return cuda_status(launch_gate_grad(logG, dLogG, ds, (long long)B * Hkv * T, T, NB, as_stream(stream)));
 }
 
-int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes) {
-  if (!bytes) return SAS_ERR_INVALID_ARG;
+int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int K, int dtype, size_t* bytes) {
+  if (!bytes || K < 1) return SAS_ERR_INVALID_ARG;
   const int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
-  *bytes = kStatusBytes + (dtype == SAS_DT_BF16 ? masks_bytes(B, Hkv, T, Hq / Hkv) : 0);
+  size_t n = kStatusBytes;
+  if (dtype == SAS_DT_BF16)
+    n += fwd_gather_applies(B, Hq, Hkv, T, K) ? fwd_gather_workspace_bytes(B, Hq, Hkv, T, K)
+                                              : masks_bytes(B, Hkv, T, Hq / Hkv);
+  *bytes = n;
   return SAS_OK;
 }
 
@@ -182,15 +195,15 @@ int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int block
 
 int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* tau,
             const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d, int block,
-            float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+            int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
   const void* ptrs[] = {Q, K, V, logG, tau, tau_idx, O, LSE};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
   int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
-  if (!(sm_scale > 0.f)) return SAS_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || Kbudget < 1) return SAS_ERR_INVALID_ARG;
   size_t need = 0;
-  sas_fwd_workspace_size(B, Hq, Hkv, T, d, block, dtype, &need);
+  sas_fwd_workspace_size(B, Hq, Hkv, T, d, block, Kbudget, dtype, &need);
   if (!ws || !aligned256(ws) || ws_bytes < need) return SAS_ERR_WORKSPACE;
   TcProblem pb{};
   pb.B = B;
@@ -210,6 +223,8 @@ int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float*
   cudaStream_t s = as_stream(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
   if (dtype == SAS_DT_F32) return cuda_status(launch_fwd_simt(pb, static_cast<float*>(O), LSE, s));
+  if (fwd_gather_applies(B, Hq, Hkv, T, Kbudget))
+    return cuda_status(launch_fwd_gather(pb, Kbudget, O, LSE, reinterpret_cast<int32_t*>(w), w + kStatusBytes, s));
   return cuda_status(launch_fwd_tc(pb, O, LSE, reinterpret_cast<int32_t*>(w),
                                    reinterpret_cast<uint32_t*>(w + kStatusBytes), s));
 }
@@ -365,6 +380,14 @@ int sas_decode_fwd_static(const void* q, const void* Kc, const void* Vc, int dty
   pb.o = o;
   pb.sel_out = sel_out;
   return cuda_status(launch_decode_static(pb, as_stream(stream)));
+}
+
+int sas_decode_static_status(void* stream, int32_t* status_out) {
+  if (!status_out) return SAS_ERR_INVALID_ARG;
+  int32_t v = 0;
+  if (decode_static_status(as_stream(stream), &v) != cudaSuccess) return SAS_ERR_CUDA;
+  *status_out = v;
+  return v == 0 ? SAS_OK : SAS_ERR_TIMEOUT;
 }
 
 int sas_device_status(const void* ws, void* stream, int32_t* status_out) {

@@ -26,13 +26,15 @@
 // that is exactly Delta_h - Delta_stored_h, because P sums to one) and stores
 // P_h(B_m); a finishing kernel subtracts sum_h P_h(B_m) eps[t, h] from dLogG.
 //
-// Pre-pass (three small kernels): per-block counts of selecting rows, their
-// offsets, and the position lists.
-#include <algorithm>
+// Pre-pass: the per-block position lists of sas_lists.cu, and a pack kernel
+// that gathers each position's Q and dO rows of the G heads with LSE and Delta
+// into one contiguous chunk.
 
 #include "sas_common.cuh"
 #include "sas_kernels.h"
 #include "sas_tmap.h"
+
+#include <algorithm>
 
 namespace sas {
 namespace gbwd {
@@ -77,7 +79,7 @@ struct Params {
   const float* LSE;
   const int32_t* cnt;        // [B*Hkv*NB] selecting rows per block
   const int32_t* off;        // [B*Hkv*NB] start of each block's list
-  const int32_t* list;       // positions
+  const int32_t* list;       // entries: position | slot << kEntrySlotShift
   const int32_t* list_cap;   // [B*Hkv*NB] entries of each list that fit its region
   // Packed rows, one chunk of `chunk` bytes per (b, g, position): Q [G][D] bf16,
   // dO [G][D] bf16, then LSE[G] and Delta[G] fp32 (padded to 16 bytes).
@@ -94,6 +96,7 @@ struct Params {
   int B, Hq, Hkv, T, NB, G, P;
   float scale_log2;
   float sm_scale;
+  uint64_t wait_ns;          // limit of one bounded wait
 };
 
 struct Bars {
@@ -104,7 +107,7 @@ struct Bars {
 // Position of list entry `idx` of block j: the block's own positions first, then the selecting rows.
 __device__ __forceinline__ int tile_position(const int32_t* lst, int own_n, int total, int j, int idx) {
   if (idx >= total) return -1;
-  return idx < own_n ? j * kBlock + idx : lst[idx - own_n];
+  return idx < own_n ? j * kBlock + idx : (lst[idx - own_n] & kEntryPosMask);
 }
 
 __device__ __forceinline__ void flush_dq(const Params& p, uint32_t taddr, int qrow) {
@@ -134,14 +137,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Block-major order: block j is attended by its own positions and by the later
-  // positions that select it, so small j carry the longest row lists. Launching
-  // them first (all groups' block 0, then block 1, ...) leaves the short lists to
-  // fill the SMs at the end. (Measured: group-major and pairs-of-groups orders,
-  // which keep fewer groups' rows in L2, were 17% and 11% slower.)
-  const int n_bg = p.B * p.Hkv;
-  const int bg = blockIdx.x % n_bg;
-  const int j = blockIdx.x / n_bg;
+  // Group-major order: the CTAs of one (b, g) run together, so the packed rows
+  // they gather (2 KB per position) and the dQ accumulator rows they reduce into
+  // stay in L2 while the group is processed. Within a group, block j is attended
+  // by its own positions and by the later positions that select it, so small j
+  // carry the longest row lists and start first.
+  const int bg = blockIdx.x / p.NB;
+  const int j = blockIdx.x % p.NB;
+  const uint64_t wait_ns = p.wait_ns;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int PP = p.P, G = p.G;
   const int rows_used = G * PP;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST;
       bool ok = true;
-      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status);
+      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       int* pos = reinterpret_cast<int*>(smem + OFF_META + st * META_STAGE);
@@ -231,11 +234,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------------ loaders: Q / dO row gathers
     const int lt = tid - LOADER_WARP0 * 32;
     constexpr int NL = N_LOADER_WARPS * 32;
+    int issued = 0;
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST;
       bool ok = true;
-      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status);
-      if (ok) ok = mbar_wait(&bars->pos_ready[st], (i / NST) & 1, status);
+      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status, wait_ns);
+      if (ok) ok = mbar_wait(&bars->pos_ready[st], (i / NST) & 1, status, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
@@ -272,11 +276,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           ++pp;
         }
       }
-      cp_async_commit_wait_all();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->qd_full[st]);
+      cp_async_commit();
+      issued = i + 1;
+      // Tile i-1 is signalled once it has landed, while tile i is in flight: two
+      // tiles of row gathers overlap (the loads of one tile take several
+      // microseconds from issue to landing).
+      if (i >= 1) {
+        cp_async_wait_group<1>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->qd_full[(i - 1) % NST]);
+      }
     }
+    cp_async_wait_all();   // also on the way out after a failed wait: no copy may outlive the CTA
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (issued > 0 && lane == 0) mbar_arrive(&bars->qd_full[(issued - 1) % NST]);
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     // A polling state machine: S/dP of the next tile and dV/dK/dQ of the oldest
@@ -285,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idesc_s = make_idesc_bf16(128, 64, 0, 0);    // rows x keys, K = features
       const uint32_t idesc_t = make_idesc_bf16(128, 64, 1, 1);    // features x keys, K = rows
       const uint32_t idesc_q = make_idesc_bf16(128, D, 0, 1);     // rows x features, K = keys
-      bool ok = mbar_wait(&bars->kv_full, 0, status);
+      bool ok = mbar_wait(&bars->kv_full, 0, status, wait_ns);
       int ns = 0, nb = 0;
       uint64_t t_last = global_ns();
       uint32_t spins = 0;
@@ -345,7 +360,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           spins = 0;
         } else if ((++spins & 255u) == 0u) {
           if (*reinterpret_cast<volatile int32_t*>(status) != 0) break;
-          if (global_ns() - t_last > kWaitLimitNs) {
+          if (global_ns() - t_last > wait_ns) {
             set_status(status, SAS_DEV_ERR_TIMEOUT);
             break;
           }
@@ -361,8 +376,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     for (int i = 0; i < n_tiles; ++i) {
       const int qb = i & 1;
-      if (!warp_wait(&bars->qrow_full[qb], (i >> 1) & 1, status)) break;
-      if (!warp_wait(&bars->dq_done[qb], (i >> 1) & 1, status)) break;
+      if (!warp_wait(&bars->qrow_full[qb], (i >> 1) & 1, status, wait_ns)) break;
+      if (!warp_wait(&bars->dq_done[qb], (i >> 1) & 1, status, wait_ns)) break;
       tc_fence_after();
       flush_dq(p, tmem + lane_base + COL_DQ0 + 128 * qb, qrow_s[qb * 128 + row]);
       tc_fence_before();
@@ -378,7 +393,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST, qb = i & 1;
-      bool step_ok = warp_wait(&bars->qd_full[st], (i / NST) & 1, status);
+      bool step_ok = warp_wait(&bars->qd_full[st], (i / NST) & 1, status, wait_ns);
       int t = -1;
       float lse2 = 0.f, dlt = 0.f, bias2 = 0.f;
       if (step_ok && r < rows_used) {
@@ -395,12 +410,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool valid = step_ok && t >= 0;
       const bool own = valid && (t / kBlock == j);
       const int lim = own ? t - j * kBlock : 63;
-      if (step_ok) step_ok = warp_wait(&bars->s_full, i & 1, status);
+      if (step_ok) step_ok = warp_wait(&bars->s_full, i & 1, status, wait_ns);
       // Two passes of 32 key columns: S, dP -> P, dS (bf16) into shared memory.
       if (step_ok) tc_fence_after();
       if (step_ok && i >= 1) {
         // P / dS shared tiles are free once tile i-1's MMAs completed.
-        step_ok = warp_wait(&bars->pd_free, (i - 1) & 1, status);
+        step_ok = warp_wait(&bars->pd_free, (i - 1) & 1, status, wait_ns);
       }
       float rs = 0.f, pm = 0.f;
       if (step_ok) {
@@ -442,7 +457,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_proxy_async_smem();
       }
       // The dQ row map of buffer qb is reusable once tile i-2 was flushed.
-      if (step_ok && i >= 2) step_ok = warp_wait(&bars->dq_free[qb], ((i - 2) >> 1) & 1, status);
+      if (step_ok && i >= 2) step_ok = warp_wait(&bars->dq_free[qb], ((i - 2) >> 1) & 1, status, wait_ns);
       if (step_ok) {
         qrow_s[qb * 128 + r] = valid ? (int)(((long long)b * p.Hq + h) * p.T + t) : -1;
         tc_fence_before();
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         p.dLogG[((long long)bg * p.T + t) * p.NB + j] = acc;
       }
     }
-    if (ok && n_tiles > 0) ok = warp_wait(&bars->pd_free, (n_tiles - 1) & 1, status);
+    if (ok && n_tiles > 0) ok = warp_wait(&bars->pd_free, (n_tiles - 1) & 1, status, wait_ns);
     if (ok) {
       tc_fence_after();
       const int dd = r;   // TMEM lane = feature
@@ -506,147 +521,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------- pre-pass
-// The pre-pass works on chunks of kChunkRows positions of one (b, g): each CTA
-// counts its chunk's (position, selected block) pairs per block in shared memory
-// and touches the global counters once per (chunk, block), so the global atomics
-// do not pile up on the few thousand block counters.
-constexpr int kChunkRows = 256;
-
-// Calls f(t, m) for every selected historical block m of every position t of the
-// chunk. One warp per group of 4 positions (blocks strided over the lanes, 128
-// blocks per pass): the loads of the 4 rows' 128-block spans are issued together,
-// so a warp pays one round trip per group and pass instead of one per row and
-// 32 blocks.
-template <typename F>
-__device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, const float* __restrict__ tau,
-                                              const int32_t* __restrict__ tau_idx, long long bg, int t0, int T,
-                                              int NB, F&& f) {
-  constexpr int R = 4, U = 4;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
-  const int t_end = min(T, t0 + kChunkRows);
-  for (int tb = t0 + warp * R; tb < t_end; tb += n_warps * R) {
-    float tv[R];
-    int ti[R], c[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int t = tb + r;
-      c[r] = (t < t_end) ? min(t / kBlock, NB) : 0;
-      tv[r] = c[r] ? tau[bg * T + t] : 0.f;
-      ti[r] = c[r] ? tau_idx[bg * T + t] : 0;
-    }
-    const int cmax = max(max(c[0], c[1]), max(c[2], c[3]));
-    for (int m0 = 0; m0 < cmax; m0 += 32 * U) {
-      float x[U][R];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int m = m0 + 32 * u + lane;
-#pragma unroll
-        for (int r = 0; r < R; ++r) x[u][r] = (m < c[r]) ? logG[(bg * T + tb + r) * (long long)NB + m] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int m = m0 + 32 * u + lane;
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-          if (m < c[r] && (x[u][r] > tv[r] || (x[u][r] == tv[r] && m <= ti[r]))) f(tb + r, m);
-      }
-    }
-  }
-}
-
-// Count, per (b, g, block), the positions whose selection contains the block.
-// Grid: (chunks of T, B * Hkv); dynamic shared memory: NB ints.
-__global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
-                                                    const int32_t* __restrict__ tau_idx, int32_t* __restrict__ cnt,
-                                                    int T, int NB) {
-  extern __shared__ int32_t hist[];
-  const long long bg = blockIdx.y;
-  const int t0 = blockIdx.x * kChunkRows;
-  for (int m = threadIdx.x; m < NB; m += blockDim.x) hist[m] = 0;
-  __syncthreads();
-  for_each_pair(logG, tau, tau_idx, bg, t0, T, NB, [&](int, int m) { atomicAdd(hist + m, 1); });
-  __syncthreads();
-  for (int m = threadIdx.x; m < NB; m += blockDim.x)
-    if (hist[m]) atomicAdd(cnt + bg * NB + m, hist[m]);
-}
-
-// Offsets: each (b, g) owns a region of T * min(H, NB) entries; off = region + prefix of counts.
-__global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ cnt, int32_t* __restrict__ off,
-                                                       int32_t* __restrict__ cursor, int32_t* __restrict__ cap,
-                                                       int32_t* __restrict__ total, int32_t* status, int NB,
-                                                       long long region) {
-  __shared__ int32_t warp_sums[32];
-  const long long bg = blockIdx.x;
-  int base = 0;
-  for (int j0 = 0; j0 < NB; j0 += 1024) {
-    const int j = j0 + threadIdx.x;
-    const int v = j < NB ? cnt[bg * NB + j] : 0;
-    int incl = v;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
-    }
-    if (lane == 31) warp_sums[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-      int ws = warp_sums[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, ws, o);
-        if (lane >= o) ws += u;
-      }
-      warp_sums[lane] = ws;
-    }
-    __syncthreads();
-    const int excl = incl - v + (w > 0 ? warp_sums[w - 1] : 0);
-    if (j < NB) {
-      // Lists beyond the (b, g) region (only possible if the threshold kept more
-      // than K-1 blocks for some row) are cut and flagged.
-      const long long start = base + excl;
-      const long long room = region - start;
-      off[bg * NB + j] = (int32_t)(bg * region + (start < region ? start : region));
-      cap[bg * NB + j] = (int32_t)(room <= 0 ? 0 : (room < v ? room : v));
-      if (room < v) set_status(status, SAS_DEV_ERR_BOUNDS);
-      cursor[bg * NB + j] = 0;
-    }
-    base += warp_sums[31];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) total[bg] = (int32_t)(base < region ? base : region);   // entries in use
-}
-
-// Writes the position lists: the chunk's pairs are counted per block in shared
-// memory, each (chunk, block) reserves its range of the block's list with one
-// global atomic, and the positions are placed in that range.
-// Grid: (chunks of T, B * Hkv); dynamic shared memory: 2 * NB ints.
-__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
-                                                   const int32_t* __restrict__ tau_idx,
-                                                   const int32_t* __restrict__ off, const int32_t* __restrict__ cap,
-                                                   int32_t* __restrict__ cursor, int32_t* __restrict__ list, int T,
-                                                   int NB) {
-  extern __shared__ int32_t sm[];
-  int32_t* lcnt = sm;        // pairs of the chunk per block, then the running slot
-  int32_t* lbase = sm + NB;  // the chunk's first slot in each block's list
-  const long long bg = blockIdx.y;
-  const int t0 = blockIdx.x * kChunkRows;
-  for (int m = threadIdx.x; m < NB; m += blockDim.x) lcnt[m] = 0;
-  __syncthreads();
-  for_each_pair(logG, tau, tau_idx, bg, t0, T, NB, [&](int, int m) { atomicAdd(lcnt + m, 1); });
-  __syncthreads();
-  for (int m = threadIdx.x; m < NB; m += blockDim.x) {
-    const int n = lcnt[m];
-    lbase[m] = n ? atomicAdd(cursor + bg * NB + m, n) : 0;
-    lcnt[m] = 0;
-  }
-  __syncthreads();
-  for_each_pair(logG, tau, tau_idx, bg, t0, T, NB, [&](int t, int m) {
-    const int slot = lbase[m] + atomicAdd(lcnt + m, 1);
-    if (slot < cap[bg * NB + m]) list[off[bg * NB + m] + slot] = t;
-  });
-}
-
 // Packs the rows of each (b, g, position) into one chunk: Q [G][D], dO [G][D]
 // (bf16), LSE [G] and Delta [G] = rowsum(O * dO) (fp32). One warp per (b, g, t, head).
 __global__ void __launch_bounds__(256) pack_kernel(const __nv_bfloat16* __restrict__ Q,
@@ -731,37 +605,28 @@ size_t bwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K) {
   auto a256 = [](size_t x) { return (x + 255) / 256 * 256; };
   size_t n = 0;
   n += a256((size_t)B * Hq * T * 128 * sizeof(float));     // dQ accumulator
-  n += 4 * a256((size_t)nbg * NB * sizeof(int32_t));       // counts, offsets, caps, cursors
-  n += a256((size_t)nbg * region * sizeof(int32_t));       // position lists
+  n += block_lists_bytes(nbg, T, NB, K);                   // per-block position lists
   n += a256((size_t)B * Hkv * T * packed_chunk_bytes(Hq / Hkv));   // packed rows
   n += a256((size_t)B * Hq * T * sizeof(float));           // eps [B*Hkv*T][G]
   n += a256((size_t)nbg * region * (Hq / Hkv) * sizeof(float));    // pmass, one per list entry and head
   n += a256((size_t)nbg * region * sizeof(int32_t));       // dLogG element of each list entry
-  n += a256((size_t)nbg * sizeof(int32_t));                // entries in use per (b, g)
   return n;
 }
 
 cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, void* dV, float* dLogG, int32_t* status,
                               float* delta, uint8_t* scratch, cudaStream_t st) {
   using namespace gbwd;
+  (void)delta;
   const int NB = pb.NB;
   const long long nbg = (long long)pb.B * pb.Hkv;
   const long long rows = nbg * pb.T;
   const long long qrows = (long long)pb.B * pb.Hq * pb.T;
-  const long long region = (long long)pb.T * std::max(1, std::min(K - 1, NB));
   auto a256 = [](size_t x) { return (x + 255) / 256 * 256; };
   float* dQacc = reinterpret_cast<float*>(scratch);
   size_t o = a256((size_t)qrows * D * sizeof(float));
-  int32_t* cnt = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * NB * sizeof(int32_t));
-  int32_t* off = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * NB * sizeof(int32_t));
-  int32_t* cursor = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * NB * sizeof(int32_t));
-  int32_t* cap = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * NB * sizeof(int32_t));
-  int32_t* list = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * region * sizeof(int32_t));
+  const BlockLists L = carve_block_lists(scratch + o, nbg, pb.T, NB, K);
+  o += block_lists_bytes(nbg, pb.T, NB, K);
+  const long long region = L.region;
   uint8_t* packed = scratch + o;
   const int chunk = (int)packed_chunk_bytes(pb.G);
   o += a256((size_t)rows * chunk);
@@ -770,22 +635,13 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   float* pmass = reinterpret_cast<float*>(scratch + o);
   o += a256((size_t)nbg * region * pb.G * sizeof(float));
   int32_t* dl_idx = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * region * sizeof(int32_t));
-  int32_t* total = reinterpret_cast<int32_t*>(scratch + o);
 
   cudaError_t e;
   if ((e = cudaMemsetAsync(dLogG, 0, (size_t)rows * NB * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dQacc, 0, (size_t)qrows * D * sizeof(float), st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(eps, 0, (size_t)qrows * sizeof(float), st)) != cudaSuccess) return e;
-  const dim3 chunks((unsigned)((pb.T + kChunkRows - 1) / kChunkRows), (unsigned)nbg);
-  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(pb.logG, pb.tau, pb.tau_idx, cnt, pb.T, NB);
-  count_launch();
-  offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(cnt, off, cursor, cap, total, status, NB, region);
-  count_launch();
-  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(pb.logG, pb.tau, pb.tau_idx, off, cap, cursor, list,
-                                                              pb.T, NB);
-  count_launch();
+  if ((e = launch_block_lists(pb.logG, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, false, status, st)) != cudaSuccess)
+    return e;
   pack_kernel<<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(pb.Q), reinterpret_cast<const __nv_bfloat16*>(pb.dO),
       reinterpret_cast<const __nv_bfloat16*>(pb.O), pb.LSE, packed, qrows, pb.T, pb.G, pb.Hq, pb.Hkv, chunk);
@@ -802,10 +658,10 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   prm.tau = pb.tau;
   prm.tau_idx = pb.tau_idx;
   prm.LSE = pb.LSE;
-  prm.cnt = cnt;
-  prm.off = off;
-  prm.list = list;
-  prm.list_cap = cap;
+  prm.cnt = L.cnt;
+  prm.off = L.off;
+  prm.list = L.list;
+  prm.list_cap = L.cap;
   prm.dQacc = dQacc;
   prm.packed = packed;
   prm.chunk = chunk;
@@ -825,13 +681,14 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   prm.P = qs.P;
   prm.scale_log2 = pb.sm_scale * kLog2e;
   prm.sm_scale = pb.sm_scale;
+  prm.wait_ns = wait_limit_ns();
   if ((e = cudaFuncSetAttribute(sas_bwd_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
       cudaSuccess)
     return e;
   sas_bwd_gather_kernel<<<(unsigned)(nbg * NB), THREADS, SMEM_BYTES, st>>>(tk, tv, prm);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dlogg_fix_kernel<<<(unsigned)((nbg * region + 255) / 256), 256, 0, st>>>(total, dl_idx, pmass, eps, dLogG,
+  dlogg_fix_kernel<<<(unsigned)((nbg * region + 255) / 256), 256, 0, st>>>(L.total, dl_idx, pmass, eps, dLogG,
                                                                           nbg * region, region, pb.T, NB, pb.G);
   count_launch();
   const long long n4 = qrows * D / 4;

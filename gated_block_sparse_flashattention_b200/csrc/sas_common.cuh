@@ -21,8 +21,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Device status codes, written to the status word in the caller's workspace.
 enum DeviceStatus : int32_t { SAS_DEV_OK = 0, SAS_DEV_ERR_TIMEOUT = 1, SAS_DEV_ERR_BOUNDS = 2 };
 
-// Wall-clock limit for one mbarrier wait (nanoseconds). Legitimate waits inside
-// these kernels last microseconds; one second means something is broken.
+// Default wall-clock limit for one mbarrier wait (nanoseconds). Legitimate waits
+// inside these kernels last microseconds; one second means something is broken.
+// Kernels that take a limit as a parameter get it from sas_set_wait_limit_ns().
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // Limit for waits while winding down: copies and MMAs already issued finish in
 // microseconds, so a few milliseconds bound a kernel that is aborting.
@@ -78,16 +79,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Returns false (and
-// records a timeout) when the wait exceeds kWaitLimitNs or another thread of the
+// records a timeout) when the wait exceeds limit_ns or another thread of the
 // launch has already recorded an error.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
+    if (it == 1u || (it & 255u) == 0u) {   // the first check early: a tiny test limit trips at once
       if (*reinterpret_cast<volatile int32_t*>(status) != 0) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         set_status(status, SAS_DEV_ERR_TIMEOUT);
         return false;
       }
@@ -97,8 +99,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
 
 // mbar_wait taken by a whole warp: true only if every lane's wait succeeded,
 // so warp-collective tcgen05 instructions that follow stay convergent.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status));
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int32_t* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, limit_ns));
 }
 
 // Wait used only while winding down (copies or MMAs still in flight): ignores
@@ -156,6 +159,11 @@ __device__ __forceinline__ void cp_async_commit_wait_all() {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Wait until at most N of this thread's most recent cp.async groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

@@ -22,6 +22,8 @@
 // 128-thread CTA per item on the CUDA cores, one bulk copy each for K and V),
 // whose CTA taking the last ticket of a (b, g) merges its partials.
 #include <algorithm>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "sas_common.cuh"
@@ -1531,25 +1533,61 @@ constexpr size_t kScratchBytes = 8u << 20;   // 8 MiB
 static __device__ __align__(256) uint8_t g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-static void* g_scratch_addr[kMaxDevices] = {};
+// Per device: the context the address was looked up in (its process-unique id)
+// and the address. A device reset or a released and re-created primary context
+// reloads the module, so the array may move: a call from a context with another
+// id looks the address up again.
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  void* addr;
+};
+static ScratchSlot g_scratch[kMaxDevices] = {};
 static std::mutex g_scratch_mutex;
 
-// Device address of g_decode_scratch on the current device, looked up once per
-// device. The host-side name is only a stand-in: the kernel must be given this
-// address, never &g_decode_scratch.
+// Id of the calling thread's current context (driver entry points resolved once).
+static cudaError_t current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+  return get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+
+// Device address of g_decode_scratch in the current device's context, looked up
+// once per context. The host-side name is only a stand-in: the kernels must be
+// given this address, never &g_decode_scratch.
 static cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  unsigned long long id = 0;
+  if (current_context_id(&id) != cudaSuccess) {
+    // No current context yet on this thread: cudaSetDevice makes the device's
+    // primary context current (it allocates nothing).
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return e;
+    if ((e = current_context_id(&id)) != cudaSuccess) return e;
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch[dev].addr == nullptr || g_scratch[dev].ctx_id != id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    g_scratch[dev] = ScratchSlot{id, p};
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch[dev].addr;
   return cudaSuccess;
 }
 
@@ -1565,6 +1603,14 @@ cudaError_t launch_decode_static(const DecodeProblem& pb, cudaStream_t st) {
   e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   return launch_decode(pb, ws, st);
+}
+
+cudaError_t decode_static_status(cudaStream_t st, int32_t* out) {
+  void* ws = nullptr;
+  cudaError_t e = decode_static::scratch_address(&ws);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
+  return cudaMemcpy(out, ws, sizeof(int32_t), cudaMemcpyDeviceToHost);
 }
 
 }  // namespace sas

@@ -11,7 +11,7 @@
 //   warps 0-3  softmax: one thread per row; gate bias, threshold mask, online
 //              softmax (exp2 domain), P written back to TMEM as bf16, epilogue;
 //   warp 4     TMA producer: Q tile once, then K/V of each block of the tile's
-//              block list into a 3-stage ring;
+//              block list into a 2-stage ring;
 //   warp 5     MMA issuer (one thread): S = Q K^T (M=128, N=64, K=128) into a
 //              double-buffered TMEM S, O += P V (A = P from TMEM, N=128) into
 //              the TMEM O accumulator. Also owns the TMEM allocation.
@@ -57,6 +57,7 @@ struct Params {
   int32_t* status;
   int B, Hq, Hkv, T, NB, NBW, G, P, n_ptiles;
   float scale_log2;
+  uint64_t wait_ns;
 };
 
 struct Bars {
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % NST;
-        if (j >= NST && !mbar_wait(&bars->kv_empty[st], ((j / NST) - 1) & 1, status)) break;
+        if (j >= NST && !mbar_wait(&bars->kv_empty[st], ((j / NST) - 1) & 1, status, p.wait_ns)) break;
         const int m = list[j];
         uint8_t* kv = smem + OFF_KV + st * STAGE_BYTES;
         mbar_expect_tx(&bars->k_full[st], 2 * KV_HALF);
@@ -197,14 +198,14 @@ __global__ void __launch_bounds__(THREADS, 2)
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc_bf16(128, 64, 0, 0);
       const uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);
-      bool ok = mbar_wait(&bars->q_full, 0, status);
+      bool ok = mbar_wait(&bars->q_full, 0, status, p.wait_ns);
       for (int j = 0; ok && j <= n; ++j) {
         if (j < n) {
           const int st = j % NST;
           const int sb = j & 1;
-          ok = mbar_wait(&bars->k_full[st], (j / NST) & 1, status);
+          ok = mbar_wait(&bars->k_full[st], (j / NST) & 1, status, p.wait_ns);
           // S buffer sb held S and then P of block j-2: free once that P V has completed.
-          if (ok && j >= 2) ok = mbar_wait(&bars->pv_done[sb], ((j - 2) >> 1) & 1, status);
+          if (ok && j >= 2) ok = mbar_wait(&bars->pv_done[sb], ((j - 2) >> 1) & 1, status, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = s_base + OFF_KV + st * STAGE_BYTES;
@@ -221,8 +222,8 @@ __global__ void __launch_bounds__(THREADS, 2)
           const int jj = j - 1;
           const int st = jj % NST;
           const int pb = jj & 1;
-          ok = mbar_wait(&bars->p_full[pb], (jj >> 1) & 1, status);
-          if (ok) ok = mbar_wait(&bars->v_full[st], (jj / NST) & 1, status);
+          ok = mbar_wait(&bars->p_full[pb], (jj >> 1) & 1, status, p.wait_ns);
+          if (ok) ok = mbar_wait(&bars->v_full[st], (jj / NST) & 1, status, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vb = s_base + OFF_KV + st * STAGE_BYTES + 2 * KV_HALF;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           bias2 = gv * kLog2e;
         }
       }
-      ok = warp_wait(&bars->s_full[sb], (j >> 1) & 1, status);
+      ok = warp_wait(&bars->s_full[sb], (j >> 1) & 1, status, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[2][32];
@@ -300,13 +301,13 @@ __global__ void __launch_bounds__(THREADS, 2)
       const float m_new = need ? mx : m_used;
       // P buffer sb is free once the PV of block j-2 has completed.
       if (j >= 2) {
-        ok = warp_wait(&bars->pv_done[sb], ((j - 2) >> 1) & 1, status);
+        ok = warp_wait(&bars->pv_done[sb], ((j - 2) >> 1) & 1, status, p.wait_ns);
         if (!ok) break;
       }
       const bool rescale_o = need && (m_used != -INFINITY) && (j > 0);
       if (__any_sync(0xffffffffu, rescale_o)) {
         // Every PV issued so far (through block j-1) must have landed in O.
-        ok = warp_wait(&bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status);
+        ok = warp_wait(&bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         const float f = rescale_o ? ex2(m_used - m_new) : 1.f;
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (lane == 0) mbar_arrive(&bars->p_full[sb]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) ok = warp_wait(&bars->pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, status);
+    if (ok && n > 0) ok = warp_wait(&bars->pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, status, p.wait_ns);
     if (ok) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
@@ -409,6 +410,7 @@ cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* sta
   prm.P = qs.P;
   prm.n_ptiles = qs.n_ptiles;
   prm.scale_log2 = pb.sm_scale * kLog2e;
+  prm.wait_ns = wait_limit_ns();
   e = cudaFuncSetAttribute(fwd::sas_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // All of L1 as shared memory, so that two CTAs fit on an SM.

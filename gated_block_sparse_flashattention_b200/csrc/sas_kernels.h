@@ -10,6 +10,9 @@ namespace sas {
 
 // Counts one kernel launch (reported by sas_launch_count()).
 void count_launch();
+// Limit of one bounded wait inside the kernels that take it as a parameter
+// (nanoseconds; sas_set_wait_limit_ns).
+uint64_t wait_limit_ns();
 
 cudaError_t launch_gate_normalize(const float* s, float* logG, long long rows, int T, int NB, cudaStream_t st);
 cudaError_t launch_select_threshold(const float* logG, float* tau, int32_t* tau_idx, int32_t* sel, long long rows,
@@ -55,9 +58,40 @@ struct TcProblem {
   const float* LSE;  // bwd only
 };
 
-// bf16 tensor-core forward; ws holds the status word and the tile masks.
+// Per-(b, g, block) position lists of the KV-block-outer kernels (sas_lists.cu).
+// An entry packs the position (bits 0-17) and the pair's slot in its row (bits
+// 18-30): 1 + the block's rank among the row's selected blocks, slot 0 being the
+// row's own block.
+constexpr int kEntrySlotShift = 18;
+constexpr int32_t kEntryPosMask = (1 << kEntrySlotShift) - 1;
+struct BlockLists {
+  int32_t* cnt;      // [nbg * NB] selecting positions per block
+  int32_t* off;      // [nbg * NB] first entry of each block's list
+  int32_t* cursor;   // [nbg * NB]
+  int32_t* cap;      // [nbg * NB] entries of each list that fit its region
+  int32_t* list;     // [nbg * region] entries
+  int32_t* nsel;     // [nbg * T] selected blocks per row (capped at K-1)
+  int32_t* total;    // [nbg] entries in use
+  long long region;  // entries per (b, g): T * min(K-1, NB)
+};
+size_t block_lists_bytes(long long nbg, int T, int NB, int K);
+BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int K);
+cudaError_t launch_block_lists(const float* logG, const float* tau, const int32_t* tau_idx, const BlockLists& L,
+                               long long nbg, int T, int NB, int K, bool want_nsel, int32_t* status,
+                               cudaStream_t st);
+
+// bf16 tensor-core forward over the union of each q-tile's blocks; ws holds the
+// status word and the tile masks.
 cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* status, uint32_t* masks,
                           cudaStream_t st);
+// bf16 tensor-core forward, KV-block outer over gathered query rows with
+// per-(position, block) partials merged per row; `scratch` holds
+// fwd_gather_workspace_bytes bytes. fwd_gather_applies: whether the partials of
+// one (b, g) fit the slot budget (else the union forward runs).
+bool fwd_gather_applies(int B, int Hq, int Hkv, int T, int K);
+size_t fwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K);
+cudaError_t launch_fwd_gather(const TcProblem& pb, int K, void* O, float* LSE, int32_t* status, uint8_t* scratch,
+                              cudaStream_t st);
 // bf16 tensor-core backward (KV-block outer, gathered query rows); `scratch`
 // holds bwd_gather_workspace_bytes bytes.
 size_t bwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K);
@@ -88,5 +122,7 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st);
 // Decode with the library's own static device scratch instead of a workspace.
 size_t decode_static_scratch_limit();
 cudaError_t launch_decode_static(const DecodeProblem& pb, cudaStream_t st);
+// Synchronises st and reads the status word of the static scratch of the current device.
+cudaError_t decode_static_status(cudaStream_t st, int32_t* out);
 
 }  // namespace sas

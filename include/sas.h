@@ -92,6 +92,18 @@ SAS_API int sas_version(void);
 SAS_API uint64_t sas_launch_count(void);
 
 /*
+ * sas_set_wait_limit_ns - limit (nanoseconds) of each bounded wait inside the
+ * sas_fwd and sas_bwd tensor-core kernels launched after this call (process-wide;
+ * 0 restores the default of 1 s). A wait that exceeds it records a timeout in the
+ * workspace status word (sas_device_status) and the kernel winds down: it lets the
+ * copies and MMAs it has issued finish, releases its tensor memory and returns,
+ * leaving its outputs incomplete. Meant for testing the failure path; a limit of a
+ * few microseconds makes the first wait of every CTA expire. Returns the previous
+ * limit. Not synchronised with calls in flight on other host threads.
+ */
+SAS_API uint64_t sas_set_wait_limit_ns(uint64_t ns);
+
+/*
  * sas_gate_normalize - softmax gate activation in log form.
  * SAS paper §4.1 eq. 4 (g = phi(s), g_0 = 1) with phi = softmax, §4.2 eq. 6:
  *   logG[b,g,t,m] = s[b,g,t,m] - log sum_{m' < c_t} exp(s[b,g,t,m'])   for m < c_t,
@@ -193,7 +205,8 @@ SAS_API int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int 
  * and may be reused across calls on the same stream. Its first word is the
  * device status word.
  */
-SAS_API int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int dtype, size_t* bytes);
+SAS_API int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int K, int dtype,
+                                   size_t* bytes);
 SAS_API int sas_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int K, int dtype,
                                size_t* bytes);
 SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int block, int K, size_t* bytes);
@@ -210,11 +223,19 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * produced by the two calls above (any values obeying their contract work).
  * O [B,Hq,T,d] of `dtype`; LSE [B,Hq,T] fp32. T % 64 == 0, NB == T / 64,
  * Hq % Hkv == 0, d in {64, 128} (fp32) or d == 128 (bf16).
- * ws: workspace of sas_fwd_workspace_size bytes.
+ * Kbudget: the budget K given to the selection (the threshold keeps at most K-1
+ * historical blocks per row; a threshold that keeps more is reported as a
+ * device-side bounds error and its extra blocks are not attended). For bf16 the
+ * workspace holds per-block row lists and one partial output per (position,
+ * attended block), about T * K * Hq/Hkv KiB per (b, g), processed in batches of
+ * (b, g) of at most 8 GiB of partials; when one (b, g) alone needs more, the
+ * call runs a q-tile kernel over the union of each tile's blocks instead and the
+ * workspace is small.
+ * ws: workspace of sas_fwd_workspace_size bytes (same K).
  */
 SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* tau,
             const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d, int block,
-            float sm_scale, void* ws, size_t ws_bytes, void* stream);
+            int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * sas_bwd - gradients of a scalar loss through sas_fwd (SAS paper Appendix E
@@ -295,14 +316,26 @@ SAS_API int sas_decode_fwd_paged(const void* q, const void* Kp, const void* Vp, 
  *    GPU (different streams, or different host threads) race on it and give
  *    wrong results: serialise them;
  *  - the first call on each device looks up the array's device address (with that
- *    device current) and caches it; make that first call before any stream capture;
- *  - the array's status word is cleared at the start of every call and is not
- *    readable through this ABI.
+ *    device current) and caches it per CUDA context (a device reset or a re-created
+ *    primary context triggers a new lookup); make that first call before any stream
+ *    capture;
+ *  - the array's status word is cleared at the start of every call; read it after
+ *    a call with sas_decode_static_status().
  */
 SAS_API int sas_decode_fwd_static(const void* q, const void* Kc, const void* Vc, int dtype, const int32_t* seqlen,
                                   const float* s, int K, int apply_log_gate, void* o, int32_t* sel_out, int B,
                                   int Hq, int Hkv, int Lmax, int NBmax, int d, int block, float sm_scale,
                                   void* stream);
+
+/*
+ * sas_decode_static_status - the device status word of the last sas_decode_fwd_static
+ * call on the current device: synchronises `stream`, copies the word of the static
+ * array to *status_out (0 = no kernel-side error; a seqlen outside 1..Lmax is a
+ * bounds error) and returns SAS_ERR_TIMEOUT if it is non-zero, else SAS_OK. Like
+ * the entry point it reads, it has no counterpart in the SAS paper and allocates
+ * nothing.
+ */
+SAS_API int sas_decode_static_status(void* stream, int32_t* status_out);
 
 /*
  * sas_device_status - read the device status word of a workspace used by

@@ -49,12 +49,21 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_sizes(lib):
-    # bf16 Qwen3-4B-like layer: status word + Delta + per-tile block masks
-    fwd = binding.sas_fwd_workspace_size(1, 32, 8, 8192, 128, binding.SAS_DT_BF16)
+    # bf16 Qwen3-4B-like layer, K = 16: the forward keeps one partial per (position, attended block): 16 slots of
+    # 4 heads x (128 bf16 + one fp32 log-sum-exp) per position and (b, g), all 8 groups in one batch
+    fwd = binding.sas_fwd_workspace_size(1, 32, 8, 8192, 128, 16, binding.SAS_DT_BF16)
     bwd = binding.sas_bwd_workspace_size(1, 32, 8, 8192, 128, 16, binding.SAS_DT_BF16)
-    assert fwd >= 256 + 8 * 256 * 4 * 4          # 256 q-tiles x 4 mask words per (b, g)
+    assert fwd >= 256 + 8 * 8192 * 16 * 4 * (256 + 4)
     assert bwd >= 256 + 32 * 8192 * 4 + 32 * 8192 * 128 * 4   # Delta + fp32 dQ accumulator
-    assert binding.sas_fwd_workspace_size(1, 4, 1, 1024, 64, binding.SAS_DT_F32) == 256
+    assert binding.sas_fwd_workspace_size(1, 4, 1, 1024, 64, 4, binding.SAS_DT_F32) == 256
+    # partials of one (b, g) over 8 GiB (T = 256K tokens, K = 64): the q-tile union forward with its small
+    # per-tile block masks (4096 q-tiles x 128 mask words) runs instead
+    big = binding.sas_fwd_workspace_size(1, 4, 1, 262144, 128, 64, binding.SAS_DT_BF16)
+    assert big == 256 + 8192 * 128 * 4
+    # the 32K layer with K = 32 needs 1.09 GB of partials per (b, g): batches of at most 8 GiB
+    c3 = binding.sas_fwd_workspace_size(2, 32, 8, 32768, 128, 32, binding.SAS_DT_BF16)
+    per_group = 32768 * 32 * 4 * (256 + 4)
+    assert 6 * per_group < c3 < 8 * per_group + (1 << 30)
     assert binding.sas_decode_workspace_size(16, 32, 8, 32768, 128, 16) > 0
 
 
@@ -68,7 +77,8 @@ def test_workspace_sizes(lib):
 def test_workspace_size_rejects(lib, args, expect):
     out = ctypes.c_size_t(0)
     B, Hq, Hkv, T, d, dt = args
-    assert lib.sas_fwd_workspace_size(B, Hq, Hkv, T, d, 64, dt, ctypes.byref(out)) == expect
+    assert lib.sas_fwd_workspace_size(B, Hq, Hkv, T, d, 64, 16, dt, ctypes.byref(out)) == expect
+    assert lib.sas_fwd_workspace_size(1, 32, 8, 8192, 128, 64, 0, binding.SAS_DT_BF16, ctypes.byref(out)) == -1
 
 
 def test_invalid_calls_return_errors_without_launching(lib):
@@ -109,10 +119,14 @@ def test_invalid_calls_return_errors_without_launching(lib):
     paged[16] = 3                 # NBmax < max_pages
     assert lib.sas_decode_fwd_paged(*paged) == -1
     # sas_fwd: missing workspace / bad sizes
-    args = [fake] * 3 + [binding.SAS_DT_BF16] + [fake] * 5 + [1, 4, 1, 128, 128, 64, ctypes.c_float(0.1), None, 0, None]
+    args = [fake] * 3 + [binding.SAS_DT_BF16] + [fake] * 5 + [1, 4, 1, 128, 128, 64, 2, ctypes.c_float(0.1), None, 0,
+                                                              None]
     assert lib.sas_fwd(*args) == -5
     args[-3] = fake
     args[-2] = 1 << 30
     args[12] = 100   # T not a multiple of 64
+    assert lib.sas_fwd(*args) == -1
+    args[12] = 128
+    args[15] = 0     # budget K < 1
     assert lib.sas_fwd(*args) == -1
     assert lib.sas_launch_count() == before

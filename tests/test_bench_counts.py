@@ -53,16 +53,46 @@ def test_executed_flops_brute_force():
     fwd, bwd = bench.executed_flops(w, torch.from_numpy(sel))
     mma = 2.0 * 128 * 64 * 128
     P = 32
-    f = b = 0.0
+    f_union = f_kv = b = 0.0
     for g in range(w.Hkv):
         for t0 in range(0, w.T, P):
             rows = range(t0, min(t0 + P, w.T))
             blocks = {t // w.block for t in rows} | {int(m) for t in rows for m in sel[0, g, t] if m >= 0}
-            f += 2 * mma * len(blocks)
+            f_union += 2 * mma * len(blocks)
         for j in range(w.NB):
             attend = min(w.block, w.T - j * w.block) + int((sel[0, g] == j).sum())
+            f_kv += 2 * mma * math.ceil(attend / P)
             b += 5 * mma * math.ceil(attend / P)
-    assert fwd == f and bwd == b
+    assert bench.fwd_uses_gather(w)
+    assert fwd == f_kv and bwd == b
+    # a problem whose per-(b, g) partials exceed the slot budget is counted as the union forward
+    big = workloads.custom("cnt", "bf16", B=1, Hq=8, Hkv=2, d=128, T=448, K=4)
+    orig = bench.SLOT_BUDGET
+    try:
+        bench.SLOT_BUDGET = 1
+        assert not bench.fwd_uses_gather(big)
+        assert bench.executed_flops(big, torch.from_numpy(sel)) == (f_union, b)
+    finally:
+        bench.SLOT_BUDGET = orig
+
+
+def test_forward_path_rule_matches_the_library_workspace():
+    """bench.fwd_uses_gather follows the library's own choice: the union forward's workspace is the status word
+    plus per-q-tile block masks, the gather forward's holds the per-pair partials."""
+    from gated_block_sparse_flashattention_b200 import binding
+    try:
+        binding.lib()
+    except RuntimeError:
+        import pytest
+        pytest.skip("library not built")
+    for (B, Hq, Hkv, T, K) in [(1, 32, 8, 8192, 16), (2, 32, 8, 32768, 32), (1, 40, 8, 65536, 16),
+                               (1, 4, 1, 262144, 64), (1, 8, 1, 131072, 300)]:
+        w = workloads.custom("rule", "bf16", B=B, Hq=Hq, Hkv=Hkv, d=128, T=T, K=K)
+        ws = binding.sas_fwd_workspace_size(B, Hq, Hkv, T, 128, K, binding.SAS_DT_BF16)
+        P = (128 // w.G) & ~7
+        masks = B * Hkv * ((T + P - 1) // P) * ((w.NB + 31) // 32) * 4
+        union_ws = 256 + (masks + 255) // 256 * 256
+        assert bench.fwd_uses_gather(w) == (ws != union_ws), (B, Hq, Hkv, T, K)
 
 
 def test_gate_kernel_byte_counts_brute_force():

@@ -21,7 +21,7 @@ TOL = {"f32": dict(o=1e-4, rel=1e-4, lse=1e-4), "bf16": dict(o=2e-2, rel=1e-2, l
 def run_gpu(inp, logG32, tau, tidx, w):
     Q, K, V, dO = (dev(inp[k]) for k in ("Q", "K", "V", "dO"))
     lg, ta, ti = dev(logG32), dev(tau), dev(tidx)
-    O, LSE = binding.forward(Q, K, V, lg, ta, ti, w.sm_scale)
+    O, LSE = binding.forward(Q, K, V, lg, ta, ti, w.K, w.sm_scale)
     dQ, dK, dV, dLogG = binding.backward(Q, K, V, O, dO, lg, ta, ti, LSE, w.K, w.sm_scale)
     torch.cuda.synchronize()
     return {k: to_np(v) for k, v in dict(O=O, LSE=LSE, dQ=dQ, dK=dK, dV=dV, dLogG=dLogG).items()}
@@ -146,7 +146,7 @@ def _full_size_sampled(w, groups, rows, blocks, seed=0):
         assert np.array_equal(sel[b, g].cpu().numpy(), se[0, 0])
     del sel
     Q, K, V, dO = (dev(inp[k]) for k in ("Q", "K", "V", "dO"))
-    O, LSE = binding.forward(Q, K, V, logG, tau, tidx, w.sm_scale)
+    O, LSE = binding.forward(Q, K, V, logG, tau, tidx, w.K, w.sm_scale)
     dQ, dK, dV, dLogG = binding.backward(Q, K, V, O, dO, logG, tau, tidx, LSE, w.K, w.sm_scale)
     torch.cuda.synchronize()
     tol = TOL[w.dtype]

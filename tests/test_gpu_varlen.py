@@ -90,7 +90,7 @@ def test_varlen_forward_backward_and_gate_grad(w, docs):
     inp = workloads.make_training_inputs(w, seed=4)
     logG, tau, tidx = check_gates(inp["s"], w.K, cu)
     Q, K, V, dO = (dev(inp[k]) for k in ("Q", "K", "V", "dO"))
-    O, LSE = binding.forward(Q, K, V, logG, tau, tidx, w.sm_scale)
+    O, LSE = binding.forward(Q, K, V, logG, tau, tidx, w.K, w.sm_scale)
     dQ, dK, dV, dLogG = binding.backward(Q, K, V, O, dO, logG, tau, tidx, LSE, w.K, w.sm_scale)
     ds = binding.gate_grad(logG, dLogG)
     torch.cuda.synchronize()

@@ -1,7 +1,8 @@
 """Host-side logic of the N>1 bench path on CPU: two gloo ranks.
 
-The work splits into independent (batch, KV-group) units with no data-path
-collective; the only exchange is the max-over-ranks reduction of timings."""
+Every rank runs a replica of the step on its own batch (seeded by the rank),
+with no data-path collective; the only exchange is the max-over-ranks
+reduction of the timed region, from which the whole-job throughput follows."""
 
 import os
 import socket
@@ -22,20 +23,25 @@ def _worker(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
                       LOCAL_RANK=str(rank))
     import bench
+    from gated_block_sparse_flashattention_b200 import workloads
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        w, r, lr = bench.dist_env()
-        units = bench.shard_units(16, r, w)
-        gathered = [None] * world
-        dist.all_gather_object(gathered, units)
-        mx = bench.reduce_max(10.0 + rank)   # per-rank "time"
+        w_, r, lr = bench.dist_env()
+        # Each rank builds its own batch of the step (seeded by its rank), as the bench's replicas do.
+        wl = workloads.custom("gloo", "bf16", B=1, Hq=4, Hkv=1, d=128, T=128, K=2)
+        inp = bench.rank_inputs(wl, r)
+        fp = float(inp["Q"].float().sum()) + float(inp["s"].sum())
+        prints = [None] * world
+        dist.all_gather_object(prints, fp)
+        mx = bench.reduce_max(10.0 + rank)   # per-rank timed region (ms)
+        value = bench.job_throughput(1e12, 4, mx, w_)
         bench.barrier()
-        q.put((rank, w, sorted(sum(gathered, [])), mx))
+        q.put((rank, w_, lr, prints, mx, value))
     finally:
         dist.destroy_process_group()
 
 
-def test_two_rank_sharding_and_max_reduction():
+def test_two_rank_replicas_and_max_reduction():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -46,10 +52,18 @@ def test_two_rank_sharding_and_max_reduction():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, world, all_units, mx in res:
-        assert world == 2
-        assert all_units == list(range(16))      # every unit exactly once across ranks
-        assert mx == 11.0                          # max over ranks
+    from gated_block_sparse_flashattention_b200 import workloads
+    wl = workloads.custom("gloo", "bf16", B=1, Hq=4, Hkv=1, d=128, T=128, K=2)
+    expect = []
+    for seed in range(2):
+        inp = workloads.make_training_inputs(wl, seed=seed)
+        expect.append(float(inp["Q"].float().sum()) + float(inp["s"].sum()))
+    assert expect[0] != expect[1]
+    for rank, world, local, prints, mx, value in res:
+        assert world == 2 and local == rank
+        assert prints == expect                    # rank r works on the batch seeded with r
+        assert mx == 11.0                          # the slowest rank's timed region
+        assert abs(value - 2 * 1e12 * 4 / 11e-3 / 1e12) < 1e-9   # every rank's steps over that time
 
 
 def test_attended_flop_count_matches_closed_form():

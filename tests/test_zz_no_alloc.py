@@ -5,8 +5,9 @@ that owns every device buffer and only hands over inputs and outputs, or a
 decode loop that must not call cudaMalloc between steps. For them the library
 keeps the decode step's scratch in a static device array. This test calls the
 entry point through the C ABI and checks it against sas_decode_fwd (which takes
-a caller workspace) on two calls in a row, within the decode tolerance of the
-other tests. The file name sorts last so that a run stopping at the first
+a caller workspace) and against the CPU oracle, on two calls in a row, within the
+decode tolerance of the other tests, and reads the static array's status word
+after each call. The file name sorts last so that a run stopping at the first
 failure has already run every other test."""
 
 import ctypes
@@ -16,6 +17,7 @@ import pytest
 import torch
 
 from gated_block_sparse_flashattention_b200 import binding, workloads
+from oracle import sas_oracle as orc
 
 pytestmark = pytest.mark.gpu
 
@@ -42,9 +44,16 @@ def test_static_scratch_decode_matches_workspace_decode_twice():
         sel = torch.full_like(sel_ref, -7)
         assert _static_call(lib, q, Kc, Vc, seqlen, s, w.K, o, sel, w) == 0
         torch.cuda.synchronize()
+        assert binding.sas_decode_static_status() == 0, f"call {call}: kernel-side error"
         assert torch.equal(sel, sel_ref), f"call {call}: selected blocks differ"
         err = (o.float() - o_ref.float()).abs().max().item()
         assert err <= 2e-2, f"call {call}: max-abs difference {err}"
+        f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+        ref_o, ref_sel = orc.decode(f64(inp["q"]), f64(inp["Kc"]), f64(inp["Vc"]), inp["seqlen"].numpy(),
+                                    inp["s"].numpy().astype(np.float64), w.K, w.block, w.sm_scale)
+        assert np.array_equal(sel.cpu().numpy(), ref_sel), f"call {call}: selection differs from the oracle"
+        err_o = np.abs(o.float().cpu().numpy() - ref_o).max()
+        assert err_o <= 2e-2, f"call {call}: max-abs difference {err_o} against the oracle"
 
 
 def test_static_scratch_rejects_problems_beyond_its_limit():
