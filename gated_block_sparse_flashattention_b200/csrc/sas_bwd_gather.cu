@@ -41,8 +41,10 @@ namespace gbwd {
 
 constexpr int D = 128;
 // Warps 0-3: softmax / dS (one thread per tile row); warp 4: control (row
-// positions and gates of each tile, K/V load); warp 5: MMA issuer; warps 6-9:
-// dQ flush (TMEM -> fp32 reductions); warps 10-15: Q/dO row gathers. The gather
+// positions of each tile, the next tile's loaded ahead; K/V load); warp 5: MMA
+// issuer; warps 6-9: dQ flush (TMEM -> shared-memory staging -> fp32 reductions
+// of whole row segments); warps 10-15: Q/dO row
+// and gate gathers. The gather
 // bandwidth one SM sustains grows with the number of warps issuing copies, so
 // most warps load; the softmax works on 32 key columns at a time to keep the
 // kernel within 128 registers per thread.
@@ -57,8 +59,8 @@ constexpr uint32_t OFF_V = 2 * KV_HALF;
 constexpr uint32_t OFF_QD = 4 * KV_HALF;                  // stage s: Q at +2s*TILE, dO at +(2s+1)*TILE
 constexpr uint32_t OFF_P = OFF_QD + NST * 2 * TILE;       // P  [128 rows][64 keys] bf16 (16 KiB)
 constexpr uint32_t OFF_DS = OFF_P + 128 * 128;            // dS [128 rows][64 keys] bf16 (16 KiB)
-// Per stage: the tile's positions [128] int, the gate of each position for block j
-// [128] float (log2 units), and the chunk tails (LSE and Delta of the G heads) of
+// Per stage: the tile's positions [128] int, the log gate of each position for
+// block j [128] float, and the chunk tails (LSE and Delta of the G heads) of
 // each position, `tail` bytes apiece (P positions * tail <= 2 KiB for every G).
 constexpr uint32_t CMETA_STAGE = 2048;
 constexpr uint32_t OFF_META = OFF_DS + 128 * 128;
@@ -66,7 +68,13 @@ constexpr uint32_t META_STAGE = 128 * 4 + 128 * 4;
 constexpr uint32_t OFF_CMETA = OFF_META + NST * META_STAGE;
 constexpr uint32_t OFF_QROW = OFF_CMETA + NST * CMETA_STAGE;   // [2][128] global row of each dQ buffer row (-1: none)
 constexpr uint32_t OFF_RED = OFF_QROW + 2 * 128 * 4;      // [2][128] fp32 row sums for dLogG
-constexpr uint32_t OFF_BAR = OFF_RED + 2 * 128 * 4;
+// dQ flush staging: per flush warp one 32-column chunk of its 32 rows (fp32,
+// 16-byte pieces XOR-swizzled by row), so that each reduction instruction adds
+// whole 128-byte row segments (four rows, four full lines) instead of one
+// 16-byte piece of 32 different rows.
+constexpr uint32_t OFF_DQS = OFF_RED + 2 * 128 * 4;
+constexpr uint32_t DQS_WARP_BYTES = 32 * 128;
+constexpr uint32_t OFF_BAR = OFF_DQS + 4 * DQS_WARP_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
 // TMEM columns
@@ -110,19 +118,31 @@ __device__ __forceinline__ int tile_position(const int32_t* lst, int own_n, int 
   return idx < own_n ? j * kBlock + idx : (lst[idx - own_n] & kEntryPosMask);
 }
 
-__device__ __forceinline__ void flush_dq(const Params& p, uint32_t taddr, int qrow) {
+// One flush warp's 32 rows of a dQ partial (TMEM lanes of its quarter) into the
+// fp32 accumulator, 32 columns at a time through the warp's staging area.
+// qrows: this warp's 32 entries of the buffer's row map (-1: no row).
+__device__ __forceinline__ void flush_dq(const Params& p, uint32_t taddr, const int* qrows, uint8_t* stage) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll 1
   for (int ch = 0; ch < D / 32; ++ch) {
     uint32_t v[32];
     tmem_ld32(taddr + 32 * ch, v);
     tmem_wait_ld();
-    if (qrow >= 0) {
-      float* dst = p.dQacc + (long long)qrow * D + 32 * ch;
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        red_add_v4(dst + 4 * k, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), __uint_as_float(v[4 * k + 2]),
-                   __uint_as_float(v[4 * k + 3]));
+    for (int k = 0; k < 8; ++k)
+      *reinterpret_cast<uint4*>(stage + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+          make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {   // rows 4m .. 4m+3, eight lanes per row
+      const int rr = 4 * m + (lane >> 3), k = lane & 7;
+      const int qrow = qrows[rr];
+      if (qrow >= 0) {
+        const float4 x = *reinterpret_cast<const float4*>(stage + rr * 128 + ((k ^ (rr & 7)) << 4));
+        red_add_v4(p.dQacc + (long long)qrow * D + 32 * ch + 4 * k, x.x, x.y, x.z, x.w);
+      }
     }
+    __syncwarp();
   }
 }
 
@@ -137,13 +157,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Group-major order: the CTAs of one (b, g) run together, so the packed rows
-  // they gather (2 KB per position) and the dQ accumulator rows they reduce into
-  // stay in L2 while the group is processed. Within a group, block j is attended
-  // by its own positions and by the later positions that select it, so small j
-  // carry the longest row lists and start first.
-  const int bg = blockIdx.x / p.NB;
-  const int j = blockIdx.x % p.NB;
+  // Block-major order: block j is attended by its own positions and by the later
+  // positions that select it, so small j carry the longest row lists. Launching
+  // them first (all groups' block 0, then block 1, ...) leaves the short lists to
+  // fill the SMs at the end. (Measured: group-major order, which keeps one
+  // group's rows in L2, was 17% slower at 8K tokens and no faster at 32K: its
+  // last group's long lists start late.)
+  const int n_bg = p.B * p.Hkv;
+  const int bg = blockIdx.x % n_bg;
+  const int j = blockIdx.x / n_bg;
   const uint64_t wait_ns = p.wait_ns;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int PP = p.P, G = p.G;
@@ -200,41 +222,39 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_3d(smem + OFF_V, &tmV, &bars->kv_full, 0, j * kBlock, bg);
       tma_load_3d(smem + OFF_V + KV_HALF, &tmV, &bars->kv_full, 64, j * kBlock, bg);
     }
+    // Positions of tile i (own positions first, then the list; -1 past the end).
+    // The next tile's are loaded while the current one is published.
+    auto load_pos = [&](int i, int (&tl)[4]) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        tl[u] = (lane + 32 * u < PP) ? tile_position(lst, own_n, total, j, i * PP + lane + 32 * u) : -1;
+    };
+    int cur[4], nxt[4] = {-1, -1, -1, -1};
+    load_pos(0, cur);
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST;
+      if (i + 1 < n_tiles) load_pos(i + 1, nxt);
       bool ok = true;
       if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       int* pos = reinterpret_cast<int*>(smem + OFF_META + st * META_STAGE);
-      float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
-      int tl[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) tl[u] = (lane + 32 * u < PP) ? tile_position(lst, own_n, total, j, i * PP + lane + 32 * u) : -1;
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (lane + 32 * u < PP) pos[lane + 32 * u] = tl[u];
+        if (lane + 32 * u < PP) pos[lane + 32 * u] = cur[u];
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pos_ready[st]);
-      // Gate of block j for each selecting position (log2 units); own positions get 0.
-      float gv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = tl[u];
-        gv[u] = (t >= 0 && t / kBlock != j) ? __ldg(p.logG + ((long long)bg * p.T + t) * p.NB + j) : 0.f;
+      if (lane == 0) {
+        mbar_arrive(&bars->pos_ready[st]);
+        mbar_arrive(&bars->qd_full[st]);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (lane + 32 * u < PP) gate[lane + 32 * u] = gv[u] * kLog2e;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->qd_full[st]);
+      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
     }
     if (lane == 0) mbar_wait_drain(&bars->kv_full, 0);
   } else if (warp >= LOADER_WARP0) {
     // ------------------------------------------------------------------ loaders: Q / dO row gathers
     const int lt = tid - LOADER_WARP0 * 32;
     constexpr int NL = N_LOADER_WARPS * 32;
-    int issued = 0;
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST;
       bool ok = true;
@@ -243,7 +263,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
+      float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
       const int first = pos[0];
+      // The log gate of block j for each selecting position (0 for own positions
+      // and empty slots), copied in the same group as the rows.
+      for (int pp = lt; pp < PP; pp += NL) {
+        const int t = pos[pp];
+        if (t >= 0 && t / kBlock != j)
+          cp_async4(smem_u32(gate + pp), p.logG + ((long long)bg * p.T + t) * p.NB + j);
+        else
+          gate[pp] = 0.f;
+      }
       const uint32_t qd = s_base + OFF_QD + st * 2 * TILE;
       const uint32_t cm = s_base + OFF_CMETA + st * CMETA_STAGE;
       // Pieces of 16 bytes of each position's chunk: 32*G of Q/dO rows (ordered
@@ -276,22 +306,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           ++pp;
         }
       }
-      cp_async_commit();
-      issued = i + 1;
-      // Tile i-1 is signalled once it has landed, while tile i is in flight: two
-      // tiles of row gathers overlap (the loads of one tile take several
-      // microseconds from issue to landing).
-      if (i >= 1) {
-        cp_async_wait_group<1>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->qd_full[(i - 1) % NST]);
-      }
+      cp_async_commit_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qd_full[st]);
     }
-    cp_async_wait_all();   // also on the way out after a failed wait: no copy may outlive the CTA
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (issued > 0 && lane == 0) mbar_arrive(&bars->qd_full[(issued - 1) % NST]);
+    cp_async_wait_all();   // after a failed wait too: no copy may outlive the CTA
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     // A polling state machine: S/dP of the next tile and dV/dK/dQ of the oldest
@@ -308,8 +328,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool prog = false;
         if (ns < n_tiles) {
           const int st = ns % NST;
-          if (mbar_try_wait(&bars->qd_full[st], (ns / NST) & 1) &&
-              (ns == 0 || mbar_try_wait(&bars->sp_free, (ns - 1) & 1))) {
+          if (mbar_test_wait(&bars->qd_full[st], (ns / NST) & 1) &&
+              (ns == 0 || mbar_test_wait(&bars->sp_free, (ns - 1) & 1))) {
             tc_fence_after();
             const uint32_t qb = s_base + OFF_QD + st * 2 * TILE;
 #pragma unroll
@@ -329,8 +349,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             prog = true;
           }
         }
-        if (nb < ns && mbar_try_wait(&bars->p_full, nb & 1) &&
-            (nb < 2 || mbar_try_wait(&bars->dq_free[nb & 1], ((nb - 2) >> 1) & 1))) {
+        if (nb < ns && mbar_test_wait(&bars->p_full, nb & 1) &&
+            (nb < 2 || mbar_test_wait(&bars->dq_free[nb & 1], ((nb - 2) >> 1) & 1))) {
           tc_fence_after();
           const int st = nb % NST, qb_ = nb & 1;
           const uint32_t qb = s_base + OFF_QD + st * 2 * TILE;
@@ -372,14 +392,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp >= 6) {
     // ------------------------------------------------------------------ dQ flush (warps 6-9)
     const int quarter = warp & 3;                    // TMEM lanes this warp may access
-    const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     for (int i = 0; i < n_tiles; ++i) {
       const int qb = i & 1;
       if (!warp_wait(&bars->qrow_full[qb], (i >> 1) & 1, status, wait_ns)) break;
       if (!warp_wait(&bars->dq_done[qb], (i >> 1) & 1, status, wait_ns)) break;
       tc_fence_after();
-      flush_dq(p, tmem + lane_base + COL_DQ0 + 128 * qb, qrow_s[qb * 128 + row]);
+      flush_dq(p, tmem + lane_base + COL_DQ0 + 128 * qb, qrow_s + qb * 128 + quarter * 32,
+               smem + OFF_DQS + quarter * DQS_WARP_BYTES);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_free[qb]);
@@ -404,7 +424,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               reinterpret_cast<const float*>(smem + OFF_CMETA + st * CMETA_STAGE + pp * (p.chunk - 512 * G));
           lse2 = tail[hh] * kLog2e;
           dlt = tail[G + hh];
-          bias2 = reinterpret_cast<const float*>(smem + OFF_META + st * META_STAGE + 128 * 4)[pp];
+          bias2 = reinterpret_cast<const float*>(smem + OFF_META + st * META_STAGE + 128 * 4)[pp] * kLog2e;
         }
       }
       const bool valid = step_ok && t >= 0;

@@ -78,6 +78,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking check of a phase (never suspends the thread): for polling loops
+// that watch several barriers at once.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed. Returns false (and
 // records a timeout) when the wait exceeds limit_ns or another thread of the
 // launch has already recorded an error.
@@ -148,6 +162,11 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 4-byte global -> shared copy (cp.async through L1).
+__device__ __forceinline__ void cp_async4(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 
 // 16-byte global -> shared copy (cp.async, L2 only), and its group wait.
@@ -487,12 +506,111 @@ __device__ __forceinline__ bool pivot_select_keys(const uint32_t (&keys)[KREG], 
   return true;
 }
 
+// Bitonic sort of 64 values held two per lane (element e = lane + 32 r in v[r]),
+// descending by element index.
+template <typename T>
+__device__ __forceinline__ void warp_sort64_desc(T (&v)[2]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {   // partners in the same lane
+        const bool keep_max = ((lane + 0) & k) == 0;   // element lane keeps the max when ascending block
+        const T hi = v[0] > v[1] ? v[0] : v[1], lo = v[0] > v[1] ? v[1] : v[0];
+        v[0] = keep_max ? hi : lo;
+        v[1] = keep_max ? lo : hi;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int e = lane + 32 * r;
+          const T o = __shfl_xor_sync(0xffffffffu, v[r], j);
+          const bool keep_max = ((e & j) == 0) == ((e & k) == 0);
+          v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] < o ? v[r] : o);
+        }
+      }
+    }
+  }
+}
+
+// Threshold of the H largest keys for 16 < H <= 63 (ties toward the lower index),
+// the pivot select of pivot_select_keys with a tighter bound: each lane's two
+// largest keys give 64 values whose H-th largest is a lower bound of the
+// threshold (H distinct keys reach it); with about H + a few keys at or above it,
+// the candidates are sorted across the warp two per lane by (key descending,
+// index ascending). *asc gets the selected indices in ascending order, element e
+// (lane + 32 r) in asc[r] for e < H (when asc != null). Returns false, with
+// nothing written, when more than 64 keys reach the bound. Requires c > H. `cand`
+// is 64 uint2 of this warp's shared memory.
+template <int KREG>
+__device__ __forceinline__ bool pivot2_select_keys(const uint32_t (&keys)[KREG], int c, int H, uint2* cand,
+                                                   uint32_t* tkey, int* tidx, uint32_t (*asc)[2] = nullptr) {
+  const int lane = threadIdx.x & 31;
+  uint32_t top[2] = {0u, 0u};   // this lane's two largest keys (empty slots hold key 0)
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) {
+    const uint32_t k = keys[i];
+    if (k > top[0]) {
+      top[1] = top[0];
+      top[0] = k;
+    } else if (k > top[1]) {
+      top[1] = k;
+    }
+  }
+  warp_sort64_desc(top);
+  const int hb = H - 1;
+  const uint32_t bound = __shfl_sync(0xffffffffu, top[hb >> 5], hb & 31);
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i) n += (lane + 32 * i < c && keys[i] >= bound) ? 1 : 0;
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total > 64) return false;
+  int pos = incl - n;
+#pragma unroll
+  for (int i = 0; i < KREG; ++i)
+    if (lane + 32 * i < c && keys[i] >= bound) cand[pos++] = make_uint2(keys[i], (uint32_t)(lane + 32 * i));
+  __syncwarp();
+  uint64_t v[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int e = lane + 32 * r;
+    v[r] = 0ull;   // below every candidate
+    if (e < total) {
+      const uint2 x = cand[e];
+      v[r] = ((uint64_t)x.x << 32) | (uint64_t)(0xffffffffu - x.y);
+    }
+  }
+  __syncwarp();
+  warp_sort64_desc(v);
+  const uint64_t th = __shfl_sync(0xffffffffu, v[hb >> 5], hb & 31);
+  *tkey = (uint32_t)(th >> 32);
+  *tidx = (int)(0xffffffffu - (uint32_t)th);
+  if (asc) {
+    // Elements 0..H-1 hold the selection; order it by index (complements sorted
+    // descending), the unselected elements last.
+    uint32_t comp[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) comp[r] = (lane + 32 * r < H) ? (uint32_t)v[r] : 0u;
+    warp_sort64_desc(comp);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) (*asc)[r] = 0xffffffffu - comp[r];
+  }
+  return true;
+}
+
 // Threshold key and tie index of the H largest keys (c > H): the pivot path when
 // it applies, else the bisection and the tie scan.
 template <int KREG>
 __device__ __forceinline__ void threshold_keys(const uint32_t (&keys)[KREG], int c, int H, uint2* cand,
                                                uint32_t* tkey, int* tidx) {
-  if (H <= 32 && pivot_select_keys(keys, c, H, cand, tkey, tidx)) return;
+  if (H <= 16 && pivot_select_keys(keys, c, H, cand, tkey, tidx)) return;
+  if (H > 16 && H <= 63 && pivot2_select_keys(keys, c, H, cand, tkey, tidx)) return;
   int take_eq = 0;
   *tkey = radix_select_keys(keys, c, H, nullptr, &take_eq);
   *tidx = tie_index_keys(keys, c, *tkey, take_eq);

@@ -23,11 +23,13 @@
 //
 // Warp roles (512 threads, one CTA per SM):
 //   warps 0-3   softmax: one thread per tile row (TMEM lane), P -> TMEM as bf16;
-//   warps 4-7   epilogue: O_j rows TMEM -> bf16 partials in global memory;
-//   warp 8      control: K_j/V_j by TMA, then per tile the positions, slots and gates;
+//   warps 4-7   epilogue: O_j rows TMEM -> bf16 -> shared-memory staging ->
+//               whole-row stores of the partials to global memory;
+//   warp 8      control: K_j/V_j by TMA, then per tile the positions and slots
+//               (the next tile's list entries loaded while the current one is published);
 //   warp 9      MMA issuer (one thread);
-//   warps 10-15 loaders: cp.async gathers of the tile's Q rows (4-stage ring,
-//               three tiles in flight per thread).
+//   warps 10-15 loaders: cp.async gathers of the tile's Q rows and of each row's
+//               gate (4-stage ring, three tiles in flight per thread).
 // TMEM: two S/P buffers (64 columns each) and two O buffers (128 each), so the
 // epilogue of tile i overlaps the softmax of tile i+1 and the MMAs of tile i+2.
 #include <algorithm>
@@ -50,7 +52,7 @@ constexpr uint32_t KV_HALF = 64 * 128;           // 64 keys x 64 features, bf16
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = 2 * KV_HALF;
 constexpr uint32_t OFF_Q = 4 * KV_HALF;          // stage s at OFF_Q + s * QTILE
-// Per stage: position [128] int, gate of block j in log2 units [128] float, slot [128] int.
+// Per stage: position [128] int, log gate of block j [128] float, slot [128] int.
 constexpr uint32_t META_STAGE = 3 * 128 * 4;
 constexpr uint32_t OFF_META = OFF_Q + NST * QTILE;
 // Per O buffer and row: partial row index (or -1), 1/l, log2-sum-exp.
@@ -60,7 +62,13 @@ struct RowInfo {
   float lse2;
 };
 constexpr uint32_t OFF_ROW = OFF_META + NST * META_STAGE;
-constexpr uint32_t OFF_BAR = OFF_ROW + 2 * 128 * sizeof(RowInfo);
+// Epilogue staging: per epilogue warp its 32 rows of bf16 partials (256 bytes
+// each, 16-byte chunks XOR-swizzled by row), so that the stores to global
+// memory write whole rows (each warp store: two rows, four full 128-byte lines)
+// instead of one 16-byte piece of 32 different rows.
+constexpr uint32_t OFF_EPI = OFF_ROW + 2 * 128 * sizeof(RowInfo);
+constexpr uint32_t EPI_WARP_BYTES = 32 * 256;
+constexpr uint32_t OFF_BAR = OFF_EPI + 4 * EPI_WARP_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;   // + alignment slack
 constexpr uint32_t COL_S = 0, COL_O = 128, TMEM_COLS = 512;   // S/P buffer b at 64 b, O buffer b at 128 + 128 b
@@ -157,50 +165,40 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_3d(smem + OFF_V, &tmV, &bars->kv_full, 0, j * kBlock, bg);
       tma_load_3d(smem + OFF_V + KV_HALF, &tmV, &bars->kv_full, 64, j * kBlock, bg);
     }
+    // Entries (position | slot << kEntrySlotShift, -1 past the end) of tile i:
+    // own positions first, then the list. The next tile's entries are loaded
+    // while the current one is published, so the list's latency is not paid per tile.
+    auto load_entries = [&](int i, int (&e)[4]) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = i * PP + lane + 32 * u;
+        e[u] = -1;
+        if (lane + 32 * u < PP && idx < total) e[u] = idx < own_n ? j * kBlock + idx : lst[idx - own_n];
+      }
+    };
+    int cur[4], nxt[4] = {-1, -1, -1, -1};
+    load_entries(0, cur);
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST;
+      if (i + 1 < n_tiles) load_entries(i + 1, nxt);
       bool ok = true;
       if (i >= NST) ok = mbar_wait(&bars->st_free[st], ((i / NST) - 1) & 1, status, wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       int* pos = reinterpret_cast<int*>(smem + OFF_META + st * META_STAGE);
-      float* gate = reinterpret_cast<float*>(pos + 128);
       int* slot = pos + 256;
-      int tl[4], sl[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = i * PP + lane + 32 * u;
-        tl[u] = -1;
-        sl[u] = 0;
-        if (lane + 32 * u < PP && idx < total) {
-          if (idx < own_n) {
-            tl[u] = j * kBlock + idx;
-          } else {
-            const int e = lst[idx - own_n];
-            tl[u] = e & kEntryPosMask;
-            sl[u] = e >> kEntrySlotShift;
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (lane + 32 * u < PP) pos[lane + 32 * u] = tl[u];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pos_ready[st]);
-      // Gate of block j for each selecting position (log2 units); own positions get 0.
-      float gv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = tl[u];
-        gv[u] = (t >= 0 && t / kBlock != j) ? __ldg(p.logG + ((long long)bg * p.T + t) * p.NB + j) : 0.f;
-      }
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if (lane + 32 * u < PP) {
-          gate[lane + 32 * u] = gv[u] * kLog2e;
-          slot[lane + 32 * u] = sl[u];
+          pos[lane + 32 * u] = cur[u] >= 0 ? (cur[u] & kEntryPosMask) : -1;
+          slot[lane + 32 * u] = cur[u] >= 0 ? (cur[u] >> kEntrySlotShift) : 0;
         }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->q_full[st]);
+      if (lane == 0) {
+        mbar_arrive(&bars->pos_ready[st]);
+        mbar_arrive(&bars->q_full[st]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
     }
     if (lane == 0) mbar_wait_drain(&bars->kv_full, 0);
   } else if (warp >= LOADER_WARP0) {
@@ -217,7 +215,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) ok = mbar_wait(&bars->pos_ready[st], (i / NST) & 1, status, wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
+      float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE) + 128;
       const uint32_t qd = s_base + OFF_Q + st * QTILE;
+      // The log gate of block j for each selecting position (0 for own positions
+      // and empty slots), copied in the same group as the rows.
+      for (int pp = lt; pp < PP; pp += NL) {
+        const int t = pos[pp];
+        if (t >= 0 && t / kBlock != j)
+          cp_async4(smem_u32(gate + pp), p.logG + ((long long)bg * p.T + t) * p.NB + j);
+        else
+          gate[pp] = 0.f;
+      }
       // Pieces ordered (position, head, 16-byte chunk): consecutive lanes copy
       // consecutive bytes of one 256-byte row.
       for (int piece = lt; piece < PP * per_pos; piece += NL) {
@@ -260,8 +268,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool prog = false;
         if (ns < n_tiles && ns < np + 2) {
           const int st = ns % NST, sb = ns & 1;
-          if (mbar_try_wait(&bars->q_full[st], (ns / NST) & 1) &&
-              (ns < 2 || mbar_try_wait(&bars->s_free[sb], ((ns - 2) >> 1) & 1))) {
+          if (mbar_test_wait(&bars->q_full[st], (ns / NST) & 1) &&
+              (ns < 2 || mbar_test_wait(&bars->s_free[sb], ((ns - 2) >> 1) & 1))) {
             tc_fence_after();
             const uint32_t qb = s_base + OFF_Q + st * QTILE;
 #pragma unroll
@@ -277,8 +285,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (np < ns) {
           const int pb = np & 1;
-          if (mbar_try_wait(&bars->p_full[pb], (np >> 1) & 1) &&
-              (np < 2 || mbar_try_wait(&bars->o_free[pb], ((np - 2) >> 1) & 1))) {
+          if (mbar_test_wait(&bars->p_full[pb], (np >> 1) & 1) &&
+              (np < 2 || mbar_test_wait(&bars->o_free[pb], ((np - 2) >> 1) & 1))) {
             tc_fence_after();
             const uint32_t vb = s_base + OFF_V;
 #pragma unroll
@@ -311,31 +319,54 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp - EPI_WARP0;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    uint8_t* stage = smem + OFF_EPI + quarter * EPI_WARP_BYTES;
     for (int i = 0; i < n_tiles; ++i) {
       const int ob = i & 1;
       if (!warp_wait(&bars->p_full[ob], (i >> 1) & 1, status, wait_ns)) break;   // row info written
       if (!warp_wait(&bars->o_full[ob], (i >> 1) & 1, status, wait_ns)) break;
       tc_fence_after();
       const RowInfo info = rowinfo[ob * 128 + r];
+      // O_j / l of this lane's row as bf16 into its staging row.
 #pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + COL_O + 128 * ob + 32 * ch, v);
+      for (int ch = 0; ch < D / 32; ch += 2) {   // two 32-column chunks per TMEM round trip
+        uint32_t v[2][32];
+        tmem_ld32(tmem + lane_base + COL_O + 128 * ob + 32 * ch, v[0]);
+        tmem_ld32(tmem + lane_base + COL_O + 128 * ob + 32 * ch + 32, v[1]);
         tmem_wait_ld();
-        if (info.dst >= 0) {
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t w[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            w[k] = pack_bf16(__uint_as_float(v[2 * k]) * info.inv_l, __uint_as_float(v[2 * k + 1]) * info.inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(p.oslot + info.dst * D + 32 * ch);
+            w[k] = pack_bf16(__uint_as_float(v[c2][2 * k]) * info.inv_l, __uint_as_float(v[c2][2 * k + 1]) * info.inv_l);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          for (int k = 0; k < 4; ++k) {
+            const int cc = 4 * (ch + c2) + k;   // 16-byte chunk of the 256-byte row
+            *reinterpret_cast<uint4*>(stage + lane * 256 + ((cc ^ (lane & 15)) << 4)) =
+                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
         }
       }
-      if (info.dst >= 0) p.lslot[info.dst] = info.lse2;
+      // The O buffer and its row info are free once TMEM is read: the stores
+      // below use this warp's staging rows and registers only.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->o_free[ob]);
+      // Whole rows out: lanes 0-15 store row 2m, lanes 16-31 row 2m+1 (the
+      // destination of row rr is held by lane rr).
+      const int dlo = (int)(info.dst & 0xffffffffll), dhi = (int)(info.dst >> 32);
+#pragma unroll 4
+      for (int m = 0; m < 16; ++m) {
+        const int rr = 2 * m + (lane >> 4), cc = lane & 15;
+        const long long d = ((long long)__shfl_sync(0xffffffffu, dhi, rr) << 32) |
+                            (uint32_t)__shfl_sync(0xffffffffu, dlo, rr);
+        if (d >= 0) {
+          const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 256 + ((cc ^ (rr & 15)) << 4));
+          *reinterpret_cast<uint4*>(p.oslot + d * D + cc * 8) = val;
+        }
+      }
+      if (info.dst >= 0) p.lslot[info.dst] = info.lse2;
+      __syncwarp();   // the staging rows are rewritten by the next tile
     }
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-3)
@@ -354,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float bias2 = 0.f;
       if (r < rows_used) {
         t = pos[pp];
-        bias2 = reinterpret_cast<const float*>(pos + 128)[pp];
+        bias2 = reinterpret_cast<const float*>(pos + 128)[pp] * kLog2e;
         sl = pos[256 + pp];
       }
       uint32_t sr[2][32];
@@ -403,67 +434,93 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// Combines the slots of each (position, head): one warp per (b, g, t, head),
-// four features per lane. n = 1 + nsel[t] slots: slot 0 (own block) and the
-// selected blocks.
+// Combines the slots of each position: one warp per (b, g, t), all G heads. A
+// slot holds G rows of 128 bf16 (G * 256 contiguous bytes): lane l owns the
+// 16-byte chunks l, l + 32, ... (KC of them, KC = ceil(G / 2)) and folds them
+// over the slots with the weights exp2(lse_s - LSE) of their head. n = 1 +
+// nsel[t] slots: slot 0 (own block) and the selected blocks.
+template <int KC>
 __global__ void __launch_bounds__(256) merge_kernel(const __nv_bfloat16* __restrict__ oslot,
                                                     const float* __restrict__ lslot,
                                                     const int32_t* __restrict__ nsel, __nv_bfloat16* __restrict__ O,
-                                                    float* __restrict__ LSE, int bg0, long long n_warps, int T,
-                                                    int Ks, int G, int Hq, int Hkv) {
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (w >= n_warps) return;
-  const int hh = (int)(w % G);
-  const long long bt = w / G;
-  const int t = (int)(bt % T);
-  const long long bgl = bt / T;
+                                                    float* __restrict__ LSE, int bg0, long long n_rows, int T, int Ks,
+                                                    int G, int Hq, int Hkv) {
+  __shared__ float lse_sh[8][16];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * 8 + wid;
+  if (w >= n_rows) return;
+  const int t = (int)(w % T);
+  const long long bgl = w / T;
   const long long bg = bg0 + bgl;
+  const long long b = bg / Hkv, g = bg % Hkv;
   const int n = 1 + min(nsel[bg * T + t], Ks - 1);
   const long long row0 = (bgl * T + t) * Ks;   // first slot of the row
-  const float* ls = lslot + row0 * G + hh;
-  float M = -INFINITY;
-  for (int s = lane; s < n; s += 32) M = fmaxf(M, ls[(long long)s * G]);
+  const float* ls = lslot + row0 * G;          // [slot][head]
+  for (int hh = 0; hh < G; ++hh) {
+    float M = -INFINITY;
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, ls[(long long)s * G + hh]);
 #pragma unroll
-  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const long long b = bg / Hkv, g = bg % Hkv;
-  const long long orow = ((b * Hq + g * G + hh) * T + t);
-  if (M == -INFINITY) {   // no finite partial (cannot happen for valid inputs: the own block holds key t)
-    *reinterpret_cast<uint2*>(O + orow * 128 + lane * 4) = make_uint2(0u, 0u);
-    if (lane == 0) LSE[orow] = -INFINITY;
-    return;
-  }
-  float L = 0.f;
-  for (int s = lane; s < n; s += 32) L += ex2(ls[(long long)s * G] - M);
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    if (M != -INFINITY)
+      for (int s = lane; s < n; s += 32) L += ex2(ls[(long long)s * G + hh] - M);
 #pragma unroll
-  for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float lse2 = M + __log2f(L);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const __nv_bfloat16* os = oslot + (row0 * G + hh) * 128 + lane * 4;
-  for (int c0 = 0; c0 < n; c0 += 32) {
-    const int s_l = c0 + lane;
-    const float wgt = s_l < n ? ex2(ls[(long long)s_l * G] - lse2) : 0.f;
-    const int cnt = min(32, n - c0);
-    for (int k0 = 0; k0 < cnt; k0 += 8) {
-      uint2 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        v[u] = (k0 + u < cnt) ? *reinterpret_cast<const uint2*>(os + (long long)(c0 + k0 + u) * G * 128)
-                              : make_uint2(0u, 0u);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float wu = __shfl_sync(0xffffffffu, wgt, (k0 + u) & 31);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-        const float2 a = __bfloat1622float2(h2[0]), c = __bfloat1622float2(h2[1]);
-        acc[0] = fmaf(wu, a.x, acc[0]);
-        acc[1] = fmaf(wu, a.y, acc[1]);
-        acc[2] = fmaf(wu, c.x, acc[2]);
-        acc[3] = fmaf(wu, c.y, acc[3]);
-      }
+    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    // No finite partial cannot happen for valid inputs (the own block holds key t).
+    const float lse2 = (M == -INFINITY) ? -INFINITY : M + __log2f(L);
+    if (lane == 0) {
+      lse_sh[wid][hh] = lse2;
+      LSE[(b * Hq + g * G + hh) * T + t] = lse2 * kLn2;
     }
   }
-  *reinterpret_cast<uint2*>(O + orow * 128 + lane * 4) = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
-  if (lane == 0) LSE[orow] = lse2 * kLn2;
+  __syncwarp();
+  const int n_chunks = 16 * G;
+  float acc[KC][8];
+#pragma unroll
+  for (int k = 0; k < KC; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+  const uint4* os = reinterpret_cast<const uint4*>(oslot + row0 * G * 128);   // slot s: G * 16 chunks
+  constexpr int U = KC <= 2 ? 4 : 2;   // slots per batch of loads
+  for (int s0 = 0; s0 < n; s0 += U) {
+    uint4 v[U][KC];
+    float wt[U][KC];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        const int c = lane + 32 * k;
+        const bool on = s0 + u < n && c < n_chunks;
+        v[u][k] = on ? os[(long long)(s0 + u) * n_chunks + c] : make_uint4(0u, 0u, 0u, 0u);
+        wt[u][k] = on ? ls[(long long)(s0 + u) * G + (c >> 4)] : -INFINITY;
+      }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        const int c = lane + 32 * k;
+        if (c >= n_chunks || wt[u][k] == -INFINITY) continue;
+        const float wu = ex2(wt[u][k] - lse_sh[wid][c >> 4]);
+        const uint32_t x[4] = {v[u][k].x, v[u][k].y, v[u][k].z, v[u][k].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[k][2 * e] = fmaf(wu, __uint_as_float(x[e] << 16), acc[k][2 * e]);
+          acc[k][2 * e + 1] = fmaf(wu, __uint_as_float(x[e] & 0xffff0000u), acc[k][2 * e + 1]);
+        }
+      }
+  }
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    const int c = lane + 32 * k;
+    if (c >= n_chunks) continue;
+    const int hh = c >> 4;
+    uint4 o;
+    o.x = pack_bf16(acc[k][0], acc[k][1]);
+    o.y = pack_bf16(acc[k][2], acc[k][3]);
+    o.z = pack_bf16(acc[k][4], acc[k][5]);
+    o.w = pack_bf16(acc[k][6], acc[k][7]);
+    *reinterpret_cast<uint4*>(O + ((b * Hq + g * G + hh) * T + t) * 128 + (c & 15) * 8) = o;
+  }
 }
 
 // Partials of one (b, g) may take at most this many bytes of workspace; larger
@@ -553,10 +610,19 @@ cudaError_t launch_fwd_gather(const TcProblem& pb, int K, void* O, float* LSE, i
     prm.bg0 = (int)bg0;
     sas_fwd_gather_kernel<<<(unsigned)(n_in * NB), THREADS, SMEM_BYTES, st>>>(tk, tv, prm);
     count_launch();
-    const long long n_warps = (long long)n_in * pb.T * pb.G;
-    merge_kernel<<<(unsigned)((n_warps + 7) / 8), 256, 0, st>>>(
-        oslot, lslot, L.nsel, reinterpret_cast<__nv_bfloat16*>(O), LSE, (int)bg0, n_warps, pb.T, Ks, pb.G, pb.Hq,
-        pb.Hkv);
+    const long long n_rows = (long long)n_in * pb.T;
+    const unsigned mgrid = (unsigned)((n_rows + 7) / 8);
+    __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(O);
+    if (pb.G <= 2)
+      merge_kernel<1><<<mgrid, 256, 0, st>>>(oslot, lslot, L.nsel, Ob, LSE, (int)bg0, n_rows, pb.T, Ks, pb.G, pb.Hq, pb.Hkv);
+    else if (pb.G <= 4)
+      merge_kernel<2><<<mgrid, 256, 0, st>>>(oslot, lslot, L.nsel, Ob, LSE, (int)bg0, n_rows, pb.T, Ks, pb.G, pb.Hq, pb.Hkv);
+    else if (pb.G <= 6)
+      merge_kernel<3><<<mgrid, 256, 0, st>>>(oslot, lslot, L.nsel, Ob, LSE, (int)bg0, n_rows, pb.T, Ks, pb.G, pb.Hq, pb.Hkv);
+    else if (pb.G <= 8)
+      merge_kernel<4><<<mgrid, 256, 0, st>>>(oslot, lslot, L.nsel, Ob, LSE, (int)bg0, n_rows, pb.T, Ks, pb.G, pb.Hq, pb.Hkv);
+    else
+      merge_kernel<8><<<mgrid, 256, 0, st>>>(oslot, lslot, L.nsel, Ob, LSE, (int)bg0, n_rows, pb.T, Ks, pb.G, pb.Hq, pb.Hkv);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -44,13 +44,28 @@ __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], i
   const int lane = threadIdx.x & 31;
   uint32_t tkey = 0u, asc = 0u;
   int tidx = -1;
-  // The ascending list (a second warp sort) only when it is requested.
-  if (H <= 32 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, out ? &asc : nullptr)) {
+  // The ascending list (a second warp sort) only when it is requested. Budgets
+  // up to 16 blocks bound the threshold by the lanes' largest keys, larger ones
+  // (up to 63) by their two largest.
+  if (H <= 16 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, out ? &asc : nullptr)) {
     if (lane == 0) {
       *tau_out = key_float(tkey);
       *tidx_out = base + tidx;
     }
     if (out && lane < H) out[lane] = base + (int32_t)asc;   // exactly H blocks, ascending
+    return;
+  }
+  uint32_t asc2[2];
+  if (H > 16 && H <= 63 &&
+      pivot2_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, out ? &asc2 : nullptr)) {
+    if (lane == 0) {
+      *tau_out = key_float(tkey);
+      *tidx_out = base + tidx;
+    }
+    if (out) {
+      if (lane < H) out[lane] = base + (int32_t)asc2[0];
+      if (lane + 32 < H) out[lane + 32] = base + (int32_t)asc2[1];
+    }
     return;
   }
   int take_eq = 0;

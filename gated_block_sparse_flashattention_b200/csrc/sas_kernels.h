@@ -67,8 +67,8 @@ constexpr int32_t kEntryPosMask = (1 << kEntrySlotShift) - 1;
 struct BlockLists {
   int32_t* cnt;      // [nbg * NB] selecting positions per block
   int32_t* off;      // [nbg * NB] first entry of each block's list
-  int32_t* cursor;   // [nbg * NB]
   int32_t* cap;      // [nbg * NB] entries of each list that fit its region
+  int32_t* ccnt;     // [nbg * chunks * NB] per-chunk counts, then each chunk's first entry
   int32_t* list;     // [nbg * region] entries
   int32_t* nsel;     // [nbg * T] selected blocks per row (capped at K-1)
   int32_t* total;    // [nbg] entries in use

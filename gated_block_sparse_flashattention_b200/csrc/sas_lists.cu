@@ -13,8 +13,10 @@
 // selected blocks; a threshold that keeps more has its extra pairs dropped and
 // is reported as a device-side bounds error.
 //
-// Three kernels: per-block counts, their offsets (a scan per (b, g)), and the
-// lists. A list entry packs the position (bits 0-17) and the slot (bits 18-30).
+// Three kernels: per-block counts (also kept per chunk of 256 positions), their
+// offsets and each chunk's first entry in every list (scans per (b, g)), and the
+// lists, placed in one more pass over the rows. A list entry packs the position
+// (bits 0-17) and the slot (bits 18-30).
 #include <algorithm>
 
 #include "sas_common.cuh"
@@ -81,11 +83,13 @@ __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, co
 }
 
 // Count, per (b, g, block), the positions whose selection contains the block
-// (pairs beyond the row's K-1 slots excluded). Grid: (chunks of T, B * Hkv);
-// dynamic shared memory: NB ints.
+// (pairs beyond the row's K-1 slots excluded), and keep each chunk's counts
+// ccnt[b, g, chunk, block] for the fill. Grid: (chunks of T, B * Hkv); dynamic
+// shared memory: NB ints.
 __global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
                                                     const int32_t* __restrict__ tau_idx, int32_t* __restrict__ cnt,
-                                                    int32_t* status, int T, int NB, int H) {
+                                                    int32_t* __restrict__ ccnt, int32_t* status, int T, int NB,
+                                                    int H) {
   extern __shared__ int32_t hist[];
   const long long bg = blockIdx.y;
   const int t0 = blockIdx.x * kChunkRows;
@@ -100,15 +104,22 @@ __global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ lo
       [&](int, int n) { over |= n > H; });
   if (over) set_status(status, SAS_DEV_ERR_BOUNDS);
   __syncthreads();
-  for (int m = threadIdx.x; m < NB; m += blockDim.x)
-    if (hist[m]) atomicAdd(cnt + bg * NB + m, hist[m]);
+  int32_t* cc = ccnt + (bg * gridDim.x + blockIdx.x) * NB;
+  for (int m = threadIdx.x; m < NB; m += blockDim.x) {
+    const int v = hist[m];
+    cc[m] = v;
+    if (v) atomicAdd(cnt + bg * NB + m, v);
+  }
 }
 
-// Offsets: each (b, g) owns a region of T * min(H, NB) entries; off = region + prefix of counts.
+// Offsets: each (b, g) owns a region of T * min(H, NB) entries; off = region +
+// prefix of the block counts. Then each chunk's first entry in each block's list:
+// ccnt[b, g, chunk, m] becomes the prefix of the earlier chunks' counts (chunk
+// order = position order, so every list is ordered by chunk).
 __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ cnt, int32_t* __restrict__ off,
-                                                       int32_t* __restrict__ cursor, int32_t* __restrict__ cap,
+                                                       int32_t* __restrict__ ccnt, int32_t* __restrict__ cap,
                                                        int32_t* __restrict__ total, int32_t* status, int NB,
-                                                       long long region) {
+                                                       int n_chunks, long long region) {
   __shared__ int32_t warp_sums[32];
   const long long bg = blockIdx.x;
   int base = 0;
@@ -143,7 +154,18 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
       off[bg * NB + j] = (int32_t)(bg * region + (start < region ? start : region));
       cap[bg * NB + j] = (int32_t)(room <= 0 ? 0 : (room < v ? room : v));
       if (room < v) set_status(status, SAS_DEV_ERR_BOUNDS);
-      cursor[bg * NB + j] = 0;
+      int32_t* cc = ccnt + bg * n_chunks * NB + j;
+      int run = 0;
+      for (int c0 = 0; c0 < n_chunks; c0 += 16) {   // 16 loads in flight, then their prefix
+        int x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) x[u] = (c0 + u < n_chunks) ? cc[(long long)(c0 + u) * NB] : 0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if (c0 + u < n_chunks) cc[(long long)(c0 + u) * NB] = run;
+          run += x[u];
+        }
+      }
     }
     base += warp_sums[31];
     __syncthreads();
@@ -151,36 +173,25 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
   if (threadIdx.x == 0) total[bg] = (int32_t)(base < region ? base : region);   // entries in use
 }
 
-// Writes the lists: the chunk's pairs are counted per block in shared memory,
-// each (chunk, block) reserves its range of the block's list with one global
-// atomic, and the entries are placed in that range. Also writes nsel[t], the
-// number of selected blocks of each row (capped at H), when nsel is not null.
-// Grid: (chunks of T, B * Hkv); dynamic shared memory: 2 * NB ints.
+// Writes the lists: each chunk places its pairs of block m from its own first
+// entry on (offsets_kernel), a shared-memory counter per block giving the next
+// free one. Also writes nsel[t], the number of selected blocks of each row
+// (capped at H), when nsel is not null. Grid: (chunks of T, B * Hkv); dynamic
+// shared memory: 2 * NB ints.
 __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
                                                    const int32_t* __restrict__ tau_idx,
                                                    const int32_t* __restrict__ off, const int32_t* __restrict__ cap,
-                                                   int32_t* __restrict__ cursor, int32_t* __restrict__ list,
+                                                   const int32_t* __restrict__ cbase, int32_t* __restrict__ list,
                                                    int32_t* __restrict__ nsel, int T, int NB, int H) {
   extern __shared__ int32_t sm[];
-  int32_t* lcnt = sm;        // pairs of the chunk per block, then the running slot
-  int32_t* lbase = sm + NB;  // the chunk's first slot in each block's list
+  int32_t* lcnt = sm;        // entries placed so far per block
+  int32_t* lbase = sm + NB;  // the chunk's first entry in each block's list
   const long long bg = blockIdx.y;
   const int t0 = blockIdx.x * kChunkRows;
-  for (int m = threadIdx.x; m < NB; m += blockDim.x) lcnt[m] = 0;
-  __syncthreads();
-  for_each_pair(
-      logG, tau, tau_idx, bg, t0, T, NB,
-      [&](int, int m, int rank) {
-        if (rank < H) atomicAdd(lcnt + m, 1);
-      },
-      [&](int t, int n) {
-        if (nsel) nsel[bg * T + t] = min(n, H);
-      });
-  __syncthreads();
+  const int32_t* cb = cbase + (bg * gridDim.x + blockIdx.x) * NB;
   for (int m = threadIdx.x; m < NB; m += blockDim.x) {
-    const int n = lcnt[m];
-    lbase[m] = n ? atomicAdd(cursor + bg * NB + m, n) : 0;
     lcnt[m] = 0;
+    lbase[m] = cb[m];
   }
   __syncthreads();
   for_each_pair(
@@ -190,18 +201,23 @@ __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ log
         const int at = lbase[m] + atomicAdd(lcnt + m, 1);
         if (at < cap[bg * NB + m]) list[off[bg * NB + m] + at] = t | ((rank + 1) << kEntrySlotShift);
       },
-      [&](int, int) {});
+      [&](int t, int n) {
+        if (nsel) nsel[bg * T + t] = min(n, H);
+      });
 }
 
 }  // namespace lists
 
+static int n_chunks_of(int T) { return (T + lists::kChunkRows - 1) / lists::kChunkRows; }
+
 size_t block_lists_bytes(long long nbg, int T, int NB, int K) {
   const long long region = (long long)T * std::max(1, std::min(K - 1, NB));
   auto a256 = [](size_t x) { return (x + 255) / 256 * 256; };
-  return 4 * a256((size_t)nbg * NB * sizeof(int32_t))      // counts, offsets, caps, cursors
-         + a256((size_t)nbg * region * sizeof(int32_t))     // entries
-         + a256((size_t)nbg * T * sizeof(int32_t))          // selected blocks per row
-         + a256((size_t)nbg * sizeof(int32_t));             // entries in use per (b, g)
+  return 3 * a256((size_t)nbg * NB * sizeof(int32_t))                 // counts, offsets, caps
+         + a256((size_t)nbg * n_chunks_of(T) * NB * sizeof(int32_t))   // per-chunk counts, then bases
+         + a256((size_t)nbg * region * sizeof(int32_t))                // entries
+         + a256((size_t)nbg * T * sizeof(int32_t))                     // selected blocks per row
+         + a256((size_t)nbg * sizeof(int32_t));                        // entries in use per (b, g)
 }
 
 BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int K) {
@@ -213,10 +229,10 @@ BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int
   o += a256((size_t)nbg * NB * sizeof(int32_t));
   L.off = reinterpret_cast<int32_t*>(scratch + o);
   o += a256((size_t)nbg * NB * sizeof(int32_t));
-  L.cursor = reinterpret_cast<int32_t*>(scratch + o);
-  o += a256((size_t)nbg * NB * sizeof(int32_t));
   L.cap = reinterpret_cast<int32_t*>(scratch + o);
   o += a256((size_t)nbg * NB * sizeof(int32_t));
+  L.ccnt = reinterpret_cast<int32_t*>(scratch + o);
+  o += a256((size_t)nbg * n_chunks_of(T) * NB * sizeof(int32_t));
   L.list = reinterpret_cast<int32_t*>(scratch + o);
   o += a256((size_t)nbg * L.region * sizeof(int32_t));
   L.nsel = reinterpret_cast<int32_t*>(scratch + o);
@@ -230,14 +246,16 @@ cudaError_t launch_block_lists(const float* logG, const float* tau, const int32_
                                cudaStream_t st) {
   using namespace lists;
   const int H = std::max(0, K - 1);
+  const int n_chunks = n_chunks_of(T);
   cudaError_t e = cudaMemsetAsync(L.cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
-  const dim3 chunks((unsigned)((T + kChunkRows - 1) / kChunkRows), (unsigned)nbg);
-  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(logG, tau, tau_idx, L.cnt, status, T, NB, H);
+  const dim3 chunks((unsigned)n_chunks, (unsigned)nbg);
+  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(logG, tau, tau_idx, L.cnt, L.ccnt, status, T, NB, H);
   count_launch();
-  offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(L.cnt, L.off, L.cursor, L.cap, L.total, status, NB, L.region);
+  offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(L.cnt, L.off, L.ccnt, L.cap, L.total, status, NB, n_chunks,
+                                                   L.region);
   count_launch();
-  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(logG, tau, tau_idx, L.off, L.cap, L.cursor, L.list,
+  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(logG, tau, tau_idx, L.off, L.cap, L.ccnt, L.list,
                                                               want_nsel ? L.nsel : nullptr, T, NB, H);
   count_launch();
   return cudaGetLastError();
