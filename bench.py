@@ -139,12 +139,13 @@ def executed_flops(w, sel):
     return fwd, bwd
 
 
-def gate_select_bytes(w) -> float:
-    """HBM bytes of the fused normalise + select: the causal part of s read once, the full logG row written,
-    tau and tau_idx written."""
+def gate_select_bytes(w, compact: bool = False) -> float:
+    """HBM bytes of the fused normalise + select: the causal part of s read once, tau and tau_idx written, and
+    the full logG row written (compact gates: the row's score LSE, 4 bytes, instead)."""
     c = np.minimum(np.arange(w.T) // w.block, w.NB).astype(np.float64)
     rows = w.B * w.Hkv
-    return rows * (4.0 * c.sum() + 4.0 * w.NB * w.T + 8.0 * w.T)
+    out = 4.0 * w.T if compact else 4.0 * w.NB * w.T
+    return rows * (4.0 * c.sum() + out + 8.0 * w.T)
 
 
 def gate_grad_bytes(w) -> float:
@@ -365,7 +366,9 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
     if host is None:
         host = rank_inputs(w, rank)
     Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
-    logG = torch.empty_like(s)
+    # Compact gates: the fused selection keeps each row's score LSE instead of writing logG; the attention
+    # and gradient calls rebuild log g = s - LSE (bit-identical to logG).
+    gate_lse = torch.empty(w.B, w.Hkv, w.T, device=device)
     tau = torch.empty(w.B, w.Hkv, w.T, device=device)
     tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
     O = torch.empty_like(Q)
@@ -379,17 +382,17 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        binding.sas_gate_normalize_select(s, logG, tau, tidx, None, w.K, stream=stream)
+        binding.sas_gate_normalize_select_compact(s, gate_lse, tau, tidx, None, w.K, stream=stream)
         if ev:
             ev[1].record(stream)
-        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream)
+        binding.sas_fwd(Q, K, V, s, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream, gate_lse=gate_lse)
         if ev:
             ev[2].record(stream)
-        binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
-                        stream=stream)
+        binding.sas_bwd(Q, K, V, O, dO, s, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
+                        stream=stream, gate_lse=gate_lse)
         if ev:
             ev[3].record(stream)
-        binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
+        binding.sas_gate_grad(s, dLogG, ds, stream=stream, gate_lse=gate_lse)
         if ev:
             ev[4].record(stream)
 
@@ -425,7 +428,7 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
         ("sas_fwd", fwd_avg, fwd_flops)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     sel = torch.empty(w.B, w.Hkv, w.T, w.K - 1, dtype=torch.int32, device=device)
-    binding.sas_select_threshold(logG, tau, tidx, sel, w.K, stream=stream)
+    binding.sas_gate_normalize_select_compact(s, gate_lse, tau, tidx, sel, w.K, stream=stream)
     torch.cuda.synchronize(device)
     ex_fwd, ex_bwd = executed_flops(w, sel)
     del sel
@@ -445,12 +448,18 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
                 "bwd_tflops": round(bwd_flops / (bwd_avg * 1e-3) / 1e12, 2),
                 "bwd_executed_tflops": round(ex_bwd / (bwd_avg * 1e-3) / 1e12, 2),
                 "bwd_inflation": round(ex_bwd / bwd_flops, 3),
+                "gate_select": "compact (row score LSE instead of logG)",
                 "gate_select_ms": round(gate_avg, 4),
-                "gate_select_gbs": round(gate_select_bytes(w) / (gate_avg * 1e-3) / 1e9, 1),
+                "gate_select_bytes": gate_select_bytes(w, compact=True),
+                "gate_select_bytes_with_logg": gate_select_bytes(w),
+                "gate_select_gbs": round(gate_select_bytes(w, compact=True) / (gate_avg * 1e-3) / 1e9, 1),
                 "gate_grad_ms": round(grad_avg, 4),
                 "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1)}
     if noisy:
+        logG = torch.empty_like(s)   # the noisy selection draws on normalised gates
+        binding.sas_gate_normalize(s, logG, stream=stream)
         noisy_ms = time_noisy_select(w, logG, flush, stream, binding, device)
+        del logG
         roofline["noisy_select_ms"] = round(noisy_ms, 4)
         roofline["noisy_select_gbs"] = round(noisy_select_bytes(w) / (noisy_ms * 1e-3) / 1e9, 1)
     res = {"workload": workload_desc(w), "value": round(job_throughput(step_flops, args.steps, total_ms, world), 3),
@@ -471,7 +480,7 @@ def run_gpu(args):
 
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    w = workloads.WORKLOADS[BENCH_WORKLOAD]
+    w = workloads.WORKLOADS[args.workload]
     fwd_flops, bwd_flops = attended_flops(w)
     step_flops = fwd_flops + bwd_flops
     peaks = measured_peaks()
@@ -499,7 +508,8 @@ def run_gpu(args):
     host = None
     torch.cuda.empty_cache()
     dec = run_decode(args, device, stream, binding, peaks, clk) if "decode" in legs else None
-    dec_paged = run_decode_paged(args, device, stream, binding, peaks, clk) if "paged" in legs else None
+    dec_paged = run_decode_paged(args, device, stream, binding, peaks, clk, args.paged_workload) \
+        if "paged" in legs else None
     varlen = run_varlen(args, device, stream, binding, rank) if "varlen" in legs else None
     clk.active = False
     clk.__exit__(None, None, None)
@@ -691,11 +701,11 @@ def run_decode(args, device, stream, binding, peaks, clk=None):
             "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
 
 
-def run_decode_paged(args, device, stream, binding, peaks, clk=None):
+def run_decode_paged(args, device, stream, binding, peaks, clk=None, name=PAGED_DECODE_WORKLOAD):
     """Long-context decode over a paged cache: 8 sequences x 1 token at 524288 tokens of context (8192 pages
     of 64 tokens per sequence, shuffled in a 19 GB pool), budget 32 blocks, 16 steps per CUDA graph with
     rotating seeded score tensors as in run_decode."""
-    w = workloads.WORKLOADS[PAGED_DECODE_WORKLOAD]
+    w = workloads.WORKLOADS[name]
     n_rot = 16
     inp = workloads.make_paged_decode_inputs(w, seed=0, device=device)
     gen = torch.Generator(device=device).manual_seed(1)
@@ -712,8 +722,8 @@ def run_decode_paged(args, device, stream, binding, peaks, clk=None):
     gbs = nbytes / (med * 1e-3) / 1e9
     pool_gb = 2 * inp["Kp"].numel() * inp["Kp"].element_size() / 1e9
     del inp
-    return {"workload": f"decode_b8_l512k_paged: 8 seqs x 1 token, context 524288 (8192 pages of 64 tokens "
-                        f"each, {pool_gb:.1f} GB K/V pool), Hq=32 Hkv=8 d=128 K=32",
+    return {"workload": f"{w.name}: {w.B} seqs x 1 token, context {w.T} ({w.NB} pages of 64 tokens "
+                        f"each, {pool_gb:.1f} GB K/V pool), Hq={w.Hq} Hkv={w.Hkv} d={w.d} K={w.K}",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": nbytes, "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
             "traffic": measured_traffic("decode_paged"), "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
@@ -726,7 +736,7 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    w = workloads.WORKLOADS[BENCH_WORKLOAD]
+    w = workloads.WORKLOADS[args.workload]
     per_step = max(2.0, args.cpu_seconds / max(1, args.steps))
     for _ in range(args.warmup):
         oracle_sample(w, 0.5)
@@ -756,6 +766,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=[BENCH_WORKLOAD, *LEG_WORKLOADS],
+                    help="layer of the step leg (default: the headline layer; the others make smaller profiling runs)")
+    ap.add_argument("--paged-workload", default=PAGED_DECODE_WORKLOAD,
+                    choices=[PAGED_DECODE_WORKLOAD, "decode_b8_l64k_paged"],
+                    help="paged decode leg (the 64K one keeps the pool at 2 GB for profiling runs)")
     ap.add_argument("--legs", default="step,legs,e2e,decode,paged,varlen,cpu",
                     help="comma list of what to measure and report: step (device-resident timed steps of the "
                          "headline layer), legs (the same step on the 8K and 64K layers), e2e (host buffers through "

@@ -34,14 +34,15 @@ _SIGNATURES = {
     "sas_select_threshold": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_gate_normalize_select": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _vp]),
+    "sas_gate_normalize_select_compact": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_vp]),
     "sas_gate_normalize_select_varlen": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_vp, _c_int, _vp]),
     "sas_select_noisy": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
-    "sas_gate_grad": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "sas_gate_grad": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "sas_fwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_bwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_decode_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
-    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_f, _vp, _sz, _vp]),
-    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7
+    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_f, _vp, _sz, _vp]),
+    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7
                 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                        + [_c_f, _vp, _sz, _vp]),
@@ -139,6 +140,12 @@ def sas_gate_normalize_select(s, logG, tau, tau_idx, sel, K, block=BLOCK, stream
         _ptr(s), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
 
 
+def sas_gate_normalize_select_compact(s, gate_lse, tau, tau_idx, sel, K, block=BLOCK, stream=None):
+    B, Hkv, T, NB = s.shape
+    _check("sas_gate_normalize_select_compact", lib().sas_gate_normalize_select_compact(
+        _ptr(s), _ptr(gate_lse), _ptr(tau), _ptr(tau_idx), _ptr(sel), B, Hkv, T, NB, block, K, _stream(stream)))
+
+
 def sas_gate_normalize_select_varlen(s, logG, tau, tau_idx, sel, K, cu_seqlens, block=BLOCK, stream=None):
     """cu_seqlens: host sequence of n_docs + 1 token offsets (multiples of 64, from 0 to T)."""
     B, Hkv, T, NB = s.shape
@@ -155,10 +162,11 @@ def sas_select_noisy(logG, noise, logG_sel, tau, tau_idx, sel, K, block=BLOCK, s
         _stream(stream)))
 
 
-def sas_gate_grad(logG, dLogG, ds, block=BLOCK, stream=None):
+def sas_gate_grad(logG, dLogG, ds, block=BLOCK, stream=None, gate_lse=None):
+    """gate_lse: the row log-sum-exp of compact gates (then logG holds the raw scores s)."""
     B, Hkv, T, NB = logG.shape
     _check("sas_gate_grad", lib().sas_gate_grad(
-        _ptr(logG), _ptr(dLogG), _ptr(ds), B, Hkv, T, NB, block, _stream(stream)))
+        _ptr(logG), _ptr(gate_lse), _ptr(dLogG), _ptr(ds), B, Hkv, T, NB, block, _stream(stream)))
 
 
 def _ws_size(name, *args) -> int:
@@ -184,21 +192,25 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block=BLOCK, stream=None):
+def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block=BLOCK, stream=None, gate_lse=None):
+    """gate_lse: the row log-sum-exp of compact gates (then logG holds the raw scores s)."""
     B, Hq, T, d = Q.shape
     Hkv = K.shape[1]
     _check("sas_fwd", lib().sas_fwd(
-        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(logG), _ptr(tau), _ptr(tau_idx), _ptr(O), _ptr(LSE),
+        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(logG), _ptr(gate_lse), _ptr(tau), _ptr(tau_idx), _ptr(O),
+        _ptr(LSE),
         B, Hq, Hkv, T, d, block, int(Kbudget), float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
 
 
 def sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block=BLOCK,
-            stream=None):
+            stream=None, gate_lse=None):
+    """gate_lse: the row log-sum-exp of compact gates (then logG holds the raw scores s)."""
     B, Hq, T, d = Q.shape
     Hkv = K.shape[1]
     _check("sas_bwd", lib().sas_bwd(
-        _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), _ptr(logG), _ptr(tau), _ptr(tau_idx),
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), _ptr(logG), _ptr(gate_lse), _ptr(tau),
+        _ptr(tau_idx),
         _ptr(LSE), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dLogG), B, Hq, Hkv, T, d, block, int(Kbudget),
         float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
@@ -269,10 +281,23 @@ def gate_and_select(s, K, block=BLOCK, want_sel=False, stream=None):
     return logG, tau, tidx, sel
 
 
-def gate_grad(logG, dLogG, block=BLOCK, stream=None):
-    """ds = dL/ds [B,Hkv,T,NB] from the log-gate gradient of ``backward`` and the gates of ``gate_and_select``."""
+def gate_and_select_compact(s, K, block=BLOCK, want_sel=False, stream=None):
+    """gate_lse, tau, tau_idx (and sel) of compact gates from selector scores s [B,Hkv,T,NB] on the device:
+    pass s as the gates and gate_lse to forward / backward / gate_grad."""
+    B, Hkv, T, NB = s.shape
+    gate_lse = torch.empty(B, Hkv, T, dtype=torch.float32, device=s.device)
+    tau = torch.empty(B, Hkv, T, dtype=torch.float32, device=s.device)
+    tidx = torch.empty(B, Hkv, T, dtype=torch.int32, device=s.device)
+    sel = torch.empty(B, Hkv, T, max(K - 1, 1), dtype=torch.int32, device=s.device) if want_sel else None
+    sas_gate_normalize_select_compact(s, gate_lse, tau, tidx, sel, K, block, stream)
+    return gate_lse, tau, tidx, sel
+
+
+def gate_grad(logG, dLogG, block=BLOCK, stream=None, gate_lse=None):
+    """ds = dL/ds [B,Hkv,T,NB] from the log-gate gradient of ``backward`` and the gates of ``gate_and_select``
+    (or the scores and ``gate_lse`` of ``gate_and_select_compact``)."""
     ds = torch.empty_like(dLogG)
-    sas_gate_grad(logG, dLogG, ds, block, stream)
+    sas_gate_grad(logG, dLogG, ds, block, stream, gate_lse=gate_lse)
     return ds
 
 
@@ -282,29 +307,32 @@ def _check_device_status(fn, ws, stream):
         raise SasError(fn, -4)
 
 
-def forward(Q, K, V, logG, tau, tau_idx, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None, check=True):
+def forward(Q, K, V, logG, tau, tau_idx, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None, check=True,
+            gate_lse=None):
     """O, LSE of ``sas_fwd``. With ``check`` the stream is synchronised and the
-    kernel status word is read (raises ``SasError`` on a kernel-side error)."""
+    kernel status word is read (raises ``SasError`` on a kernel-side error).
+    With ``gate_lse`` (compact gates) ``logG`` holds the raw scores s."""
     B, Hq, T, d = Q.shape
     O = torch.empty_like(Q)
     LSE = torch.empty(B, Hq, T, dtype=torch.float32, device=Q.device)
     if ws is None:
         ws = workspace(sas_fwd_workspace_size(B, Hq, K.shape[1], T, d, Kbudget, _dtype_code(Q), block), Q.device)
-    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block, stream)
+    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block, stream, gate_lse=gate_lse)
     if check:
         _check_device_status("sas_fwd", ws, stream)
     return O, LSE
 
 
 def backward(Q, K, V, O, dO, logG, tau, tau_idx, LSE, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None,
-             check=True):
-    """dQ, dK, dV, dLogG of ``sas_bwd`` (``check`` as in ``forward``)."""
+             check=True, gate_lse=None):
+    """dQ, dK, dV, dLogG of ``sas_bwd`` (``check`` and ``gate_lse`` as in ``forward``)."""
     B, Hq, T, d = Q.shape
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     dLogG = torch.empty_like(logG)
     if ws is None:
         ws = workspace(sas_bwd_workspace_size(B, Hq, K.shape[1], T, d, Kbudget, _dtype_code(Q), block), Q.device)
-    sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block, stream)
+    sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block, stream,
+            gate_lse=gate_lse)
     if check:
         _check_device_status("sas_bwd", ws, stream)
     return dQ, dK, dV, dLogG

@@ -119,6 +119,18 @@ int sas_gate_normalize_select(const float* s, float* logG, float* tau, int32_t* 
       launch_normalize_select(s, logG, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB, K - 1, as_stream(stream)));
 }
 
+int sas_gate_normalize_select_compact(const float* s, float* gate_lse, float* tau, int32_t* tau_idx, int32_t* sel,
+                                      int B, int Hkv, int T, int NB, int block, int K, void* stream) {
+  if (!s || !gate_lse || !tau || !tau_idx) return SAS_ERR_INVALID_ARG;
+  if (!aligned16(s) || !aligned16(gate_lse) || !aligned16(tau) || !aligned16(tau_idx)) return SAS_ERR_INVALID_ARG;
+  if (sel && !aligned16(sel)) return SAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || T <= 0 || NB <= 0 || block != 64 || K < 1) return SAS_ERR_INVALID_ARG;
+  if ((long long)NB * 64 < T) return SAS_ERR_INVALID_ARG;
+  if (NB > 1024) return SAS_ERR_UNSUPPORTED;   // rows are held in registers
+  return cuda_status(launch_normalize_select_compact(s, gate_lse, tau, tau_idx, sel, (long long)B * Hkv * T, T, NB,
+                                                     K - 1, as_stream(stream)));
+}
+
 int sas_gate_normalize_select_varlen(const float* s, float* logG, float* tau, int32_t* tau_idx, int32_t* sel, int B,
                                      int Hkv, int T, int NB, int block, int K, const int32_t* cu_seqlens,
                                      int n_docs, void* stream) {
@@ -154,13 +166,14 @@ int sas_select_noisy(const float* logG, const float* noise, float* logG_sel, flo
                                          K - 1, as_stream(stream)));
 }
 
-int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int B, int Hkv, int T, int NB, int block,
-                  void* stream) {
+int sas_gate_grad(const float* logG, const float* gate_lse, const float* dLogG, float* ds, int B, int Hkv, int T, int NB,
+                  int block, void* stream) {
   if (!logG || !dLogG || !ds || ds == logG || ds == dLogG) return SAS_ERR_INVALID_ARG;
   if (!aligned16(logG) || !aligned16(dLogG) || !aligned16(ds)) return SAS_ERR_INVALID_ARG;
+  if (gate_lse && (!aligned16(gate_lse) || gate_lse == ds)) return SAS_ERR_INVALID_ARG;
   if (B <= 0 || Hkv <= 0 || T <= 0 || NB <= 0 || block != 64) return SAS_ERR_INVALID_ARG;
   if ((long long)NB * 64 < T) return SAS_ERR_INVALID_ARG;
-  return cuda_status(launch_gate_grad(logG, dLogG, ds, (long long)B * Hkv * T, T, NB, as_stream(stream)));
+  return cuda_status(launch_gate_grad(logG, gate_lse, dLogG, ds, (long long)B * Hkv * T, T, NB, as_stream(stream)));
 }
 
 int sas_fwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int block, int K, int dtype, size_t* bytes) {
@@ -193,12 +206,13 @@ int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int block
   return SAS_OK;
 }
 
-int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* tau,
-            const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d, int block,
-            int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* gate_lse,
+            const float* tau, const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d,
+            int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
   const void* ptrs[] = {Q, K, V, logG, tau, tau_idx, O, LSE};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
+  if (gate_lse && !aligned16(gate_lse)) return SAS_ERR_INVALID_ARG;
   int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
   if (!(sm_scale > 0.f) || Kbudget < 1) return SAS_ERR_INVALID_ARG;
@@ -218,6 +232,7 @@ int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float*
   pb.K = K;
   pb.V = V;
   pb.logG = logG;
+  pb.gate_lse = gate_lse;
   pb.tau = tau;
   pb.tau_idx = tau_idx;
   cudaStream_t s = as_stream(stream);
@@ -230,12 +245,13 @@ int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float*
 }
 
 int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
-            const float* logG, const float* tau, const int32_t* tau_idx, const float* LSE, void* dQ, void* dK,
-            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget, float sm_scale,
-            void* ws, size_t ws_bytes, void* stream) {
+            const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx, const float* LSE,
+            void* dQ, void* dK, void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget,
+            float sm_scale, void* ws, size_t ws_bytes, void* stream) {
   const void* ptrs[] = {Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
+  if (gate_lse && !aligned16(gate_lse)) return SAS_ERR_INVALID_ARG;
   int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
   if (!(sm_scale > 0.f)) return SAS_ERR_INVALID_ARG;
@@ -258,6 +274,7 @@ int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   pb.O = O;
   pb.dO = dO;
   pb.logG = logG;
+  pb.gate_lse = gate_lse;
   pb.tau = tau;
   pb.tau_idx = tau_idx;
   pb.LSE = LSE;

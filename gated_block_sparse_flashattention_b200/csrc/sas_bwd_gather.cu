@@ -59,12 +59,13 @@ constexpr uint32_t OFF_V = 2 * KV_HALF;
 constexpr uint32_t OFF_QD = 4 * KV_HALF;                  // stage s: Q at +2s*TILE, dO at +(2s+1)*TILE
 constexpr uint32_t OFF_P = OFF_QD + NST * 2 * TILE;       // P  [128 rows][64 keys] bf16 (16 KiB)
 constexpr uint32_t OFF_DS = OFF_P + 128 * 128;            // dS [128 rows][64 keys] bf16 (16 KiB)
-// Per stage: the tile's positions [128] int, the log gate of each position for
-// block j [128] float, and the chunk tails (LSE and Delta of the G heads) of
+// Per stage: the tile's positions [128] int, the gate score of each position for
+// block j [128] float and its row's score LSE [128] float (0 unless the gates
+// come as raw scores), and the chunk tails (LSE and Delta of the G heads) of
 // each position, `tail` bytes apiece (P positions * tail <= 2 KiB for every G).
 constexpr uint32_t CMETA_STAGE = 2048;
 constexpr uint32_t OFF_META = OFF_DS + 128 * 128;
-constexpr uint32_t META_STAGE = 128 * 4 + 128 * 4;
+constexpr uint32_t META_STAGE = 3 * 128 * 4;   // positions, gate scores, row score LSEs (compact gates)
 constexpr uint32_t OFF_CMETA = OFF_META + NST * META_STAGE;
 constexpr uint32_t OFF_QROW = OFF_CMETA + NST * CMETA_STAGE;   // [2][128] global row of each dQ buffer row (-1: none)
 constexpr uint32_t OFF_RED = OFF_QROW + 2 * 128 * 4;      // [2][128] fp32 row sums for dLogG
@@ -81,7 +82,8 @@ constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
 constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DV = 128, COL_DK = 192, COL_DQ0 = 256, TMEM_COLS = 512;
 
 struct Params {
-  const float* logG;
+  const float* logG;         // log gates, or raw scores when gate_lse is set
+  const float* gate_lse;     // null, or the LSE of each row's historical scores
   const float* tau;
   const int32_t* tau_idx;
   const float* LSE;
@@ -264,15 +266,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
       float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
+      float* glse = gate + 128;
       const int first = pos[0];
-      // The log gate of block j for each selecting position (0 for own positions
-      // and empty slots), copied in the same group as the rows.
+      // The gate of block j for each selecting position (0 for own positions and
+      // empty slots), with its row's score LSE when the gates come as raw scores,
+      // copied in the same group as the rows.
       for (int pp = lt; pp < PP; pp += NL) {
         const int t = pos[pp];
-        if (t >= 0 && t / kBlock != j)
+        if (t >= 0 && t / kBlock != j) {
           cp_async4(smem_u32(gate + pp), p.logG + ((long long)bg * p.T + t) * p.NB + j);
-        else
+          if (p.gate_lse)
+            cp_async4(smem_u32(glse + pp), p.gate_lse + (long long)bg * p.T + t);
+          else
+            glse[pp] = 0.f;
+        } else {
           gate[pp] = 0.f;
+          glse[pp] = 0.f;
+        }
       }
       const uint32_t qd = s_base + OFF_QD + st * 2 * TILE;
       const uint32_t cm = s_base + OFF_CMETA + st * CMETA_STAGE;
@@ -424,7 +434,9 @@ __global__ void __launch_bounds__(THREADS, 1)
               reinterpret_cast<const float*>(smem + OFF_CMETA + st * CMETA_STAGE + pp * (p.chunk - 512 * G));
           lse2 = tail[hh] * kLog2e;
           dlt = tail[G + hh];
-          bias2 = reinterpret_cast<const float*>(smem + OFF_META + st * META_STAGE + 128 * 4)[pp] * kLog2e;
+          // log g = s - LSE(s) in fp32 (bit-identical to the normalised gate), then log2 units
+          const float* gm = reinterpret_cast<const float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
+          bias2 = (gm[pp] - gm[128 + pp]) * kLog2e;
         }
       }
       const bool valid = step_ok && t >= 0;
@@ -660,7 +672,8 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   if ((e = cudaMemsetAsync(dLogG, 0, (size_t)rows * NB * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dQacc, 0, (size_t)qrows * D * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(eps, 0, (size_t)qrows * sizeof(float), st)) != cudaSuccess) return e;
-  if ((e = launch_block_lists(pb.logG, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, false, status, st)) != cudaSuccess)
+  if ((e = launch_block_lists(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, false, status, st)) !=
+      cudaSuccess)
     return e;
   pack_kernel<<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(pb.Q), reinterpret_cast<const __nv_bfloat16*>(pb.dO),
@@ -675,6 +688,7 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
     return cudaErrorInvalidValue;
   Params prm;
   prm.logG = pb.logG;
+  prm.gate_lse = pb.gate_lse;
   prm.tau = pb.tau;
   prm.tau_idx = pb.tau_idx;
   prm.LSE = pb.LSE;

@@ -52,8 +52,9 @@ constexpr uint32_t KV_HALF = 64 * 128;           // 64 keys x 64 features, bf16
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = 2 * KV_HALF;
 constexpr uint32_t OFF_Q = 4 * KV_HALF;          // stage s at OFF_Q + s * QTILE
-// Per stage: position [128] int, log gate of block j [128] float, slot [128] int.
-constexpr uint32_t META_STAGE = 3 * 128 * 4;
+// Per stage: position [128] int, gate score of block j [128] float, slot [128]
+// int, and the row's score LSE [128] float (0 unless the gates come as raw scores).
+constexpr uint32_t META_STAGE = 4 * 128 * 4;
 constexpr uint32_t OFF_META = OFF_Q + NST * QTILE;
 // Per O buffer and row: partial row index (or -1), 1/l, log2-sum-exp.
 struct RowInfo {
@@ -75,7 +76,8 @@ constexpr uint32_t COL_S = 0, COL_O = 128, TMEM_COLS = 512;   // S/P buffer b at
 
 struct Params {
   const __nv_bfloat16* Q;
-  const float* logG;
+  const float* logG;         // log gates, or raw scores when gate_lse is set
+  const float* gate_lse;     // null, or the LSE of each row's historical scores
   const int32_t* cnt;        // per-block lists (sas_lists.cu), indexed by the global (b, g)
   const int32_t* off;
   const int32_t* list;
@@ -216,15 +218,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
       float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE) + 128;
+      float* glse = gate + 256;
       const uint32_t qd = s_base + OFF_Q + st * QTILE;
-      // The log gate of block j for each selecting position (0 for own positions
-      // and empty slots), copied in the same group as the rows.
+      // The gate of block j for each selecting position (0 for own positions and
+      // empty slots), with its row's score LSE when the gates come as raw scores,
+      // copied in the same group as the rows.
       for (int pp = lt; pp < PP; pp += NL) {
         const int t = pos[pp];
-        if (t >= 0 && t / kBlock != j)
+        if (t >= 0 && t / kBlock != j) {
           cp_async4(smem_u32(gate + pp), p.logG + ((long long)bg * p.T + t) * p.NB + j);
-        else
+          if (p.gate_lse)
+            cp_async4(smem_u32(glse + pp), p.gate_lse + (long long)bg * p.T + t);
+          else
+            glse[pp] = 0.f;
+        } else {
           gate[pp] = 0.f;
+          glse[pp] = 0.f;
+        }
       }
       // Pieces ordered (position, head, 16-byte chunk): consecutive lanes copy
       // consecutive bytes of one 256-byte row.
@@ -385,7 +395,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       float bias2 = 0.f;
       if (r < rows_used) {
         t = pos[pp];
-        bias2 = reinterpret_cast<const float*>(pos + 128)[pp] * kLog2e;
+        // log g = s - LSE(s) in fp32 (bit-identical to the normalised gate), then log2 units
+        bias2 = (reinterpret_cast<const float*>(pos + 128)[pp] - reinterpret_cast<const float*>(pos + 384)[pp]) *
+                kLog2e;
         sl = pos[256 + pp];
       }
       uint32_t sr[2][32];
@@ -576,7 +588,8 @@ cudaError_t launch_fwd_gather(const TcProblem& pb, int K, void* O, float* LSE, i
   o += a256((size_t)slot_rows * D * 2);
   float* lslot = reinterpret_cast<float*>(scratch + o);
 
-  cudaError_t e = launch_block_lists(pb.logG, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, true, status, st);
+  cudaError_t e =
+      launch_block_lists(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, true, status, st);
   if (e != cudaSuccess) return e;
   const QTileShape qs = qtile_shape(pb.G, pb.T, NB);
   CUtensorMap tk, tv;
@@ -586,6 +599,7 @@ cudaError_t launch_fwd_gather(const TcProblem& pb, int K, void* O, float* LSE, i
   Params prm;
   prm.Q = reinterpret_cast<const __nv_bfloat16*>(pb.Q);
   prm.logG = pb.logG;
+  prm.gate_lse = pb.gate_lse;
   prm.cnt = L.cnt;
   prm.off = L.off;
   prm.list = L.list;

@@ -48,7 +48,8 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 
 struct Params {
-  const float* logG;
+  const float* logG;       // log gates, or raw scores when gate_lse is set
+  const float* gate_lse;   // null, or the LSE of each row's historical scores
   const float* tau;
   const int32_t* tau_idx;
   const uint32_t* masks;
@@ -252,6 +253,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const float tau_t = valid ? p.tau[grow] : INFINITY;
     const int tidx_t = valid ? p.tau_idx[grow] : -1;
     const float* gate_row = p.logG + grow * (long long)p.NB;
+    const float grl = (valid && p.gate_lse) ? p.gate_lse[grow] : 0.f;   // log g = s - LSE(s) for raw scores
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float m_used = -INFINITY;
     float l = 0.f;
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     float gate_next = 0.f;
     if (n > 0) {
       const int m0 = list[0];
-      gate_next = (valid && m0 < c_t) ? __ldg(gate_row + m0) : 0.f;
+      gate_next = (valid && m0 < c_t) ? __ldg(gate_row + m0) - grl : 0.f;
     }
     for (int j = 0; j < n; ++j) {
       const int m = list[j];
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const float gv = gate_next;
       if (j + 1 < n) {
         const int mn = list[j + 1];
-        gate_next = (valid && mn < c_t) ? __ldg(gate_row + mn) : 0.f;
+        gate_next = (valid && mn < c_t) ? __ldg(gate_row + mn) - grl : 0.f;
       }
       // Row bias for this block: own block causal, selected historical gated, rest masked.
       bool masked = true;
@@ -384,7 +386,8 @@ __global__ void __launch_bounds__(THREADS, 2)
 cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* status, uint32_t* masks,
                           cudaStream_t st) {
   const QTileShape qs = qtile_shape(pb.G, pb.T, pb.NB);
-  cudaError_t e = launch_tile_union(pb.logG, pb.tau, pb.tau_idx, masks, (long long)pb.B * pb.Hkv, pb.T, pb.NB, qs.P,
+  cudaError_t e = launch_tile_union(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, masks, (long long)pb.B * pb.Hkv, pb.T,
+                                    pb.NB, qs.P,
                                     qs.n_ptiles, qs.NBW, st);
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv;
@@ -394,6 +397,7 @@ cudaError_t launch_fwd_tc(const TcProblem& pb, void* O, float* LSE, int32_t* sta
     return cudaErrorInvalidValue;
   fwd::Params prm;
   prm.logG = pb.logG;
+  prm.gate_lse = pb.gate_lse;
   prm.tau = pb.tau;
   prm.tau_idx = pb.tau_idx;
   prm.masks = masks;

@@ -180,10 +180,13 @@ __global__ void __launch_bounds__(256) select_threshold_kernel(const float* __re
 // outputs equal the two separate calls bit for bit. Rows longer than
 // 32 * kSelectReg blocks use the two kernels.
 // ---------------------------------------------------------------------------
+// With lse_out set (compact gates) the row's LSE of s goes there and no logG is
+// written (dst unused): consumers rebuild logG[m] = s[m] - LSE, the same fp32
+// subtraction as here.
 template <int KREG>
 __device__ __forceinline__ void normalize_select_row(const float* __restrict__ src, float* __restrict__ dst, int c_lo,
                                                      int c, int NB, int H, uint32_t* hist, float* tau_out,
-                                                     int32_t* tidx_out, int32_t* out) {
+                                                     int32_t* tidx_out, int32_t* out, float* lse_out = nullptr) {
   // The row's historical blocks are c_lo .. c-1 (c_lo > 0 only for a later document of a packed sequence).
   const int lane = threadIdx.x & 31;
   const int n = c - c_lo;
@@ -207,12 +210,16 @@ __device__ __forceinline__ void normalize_select_row(const float* __restrict__ s
   for (int i = 0; i < KREG; ++i) {
     const int q = lane + 32 * i;
     const float lg = (q < n) ? v[i] - lse : -INFINITY;
-    if (c_lo + q < NB) dst[c_lo + q] = lg;
+    if (!lse_out && c_lo + q < NB) dst[c_lo + q] = lg;
     keys[i] = (q < n) ? float_key(lg) : 0u;
     v[i] = lg;
   }
-  for (int m = lane; m < c_lo; m += 32) dst[m] = -INFINITY;
-  for (int m = c_lo + lane + 32 * KREG; m < NB; m += 32) dst[m] = -INFINITY;
+  if (lse_out) {
+    if (lane == 0) *lse_out = lse;
+  } else {
+    for (int m = lane; m < c_lo; m += 32) dst[m] = -INFINITY;
+    for (int m = c_lo + lane + 32 * KREG; m < NB; m += 32) dst[m] = -INFINITY;
+  }
   if (c_lo == 0) {
     if (select_trivial_row(c, H, tau_out, tidx_out, out)) return;
   } else if (min(n, H) == 0 || n <= H) {
@@ -259,6 +266,26 @@ __global__ void __launch_bounds__(256) normalize_select_kernel(const float* __re
   int32_t* out = sel ? sel + row * (long long)H : nullptr;
   normalize_select_row<KREG>(s + row * (long long)NB, logG + row * (long long)NB, 0, c, NB, H, hist_all[wid],
                              tau + row, tau_idx + row, out);
+}
+
+// Compact gates: the same per row, writing the LSE of the row's historical
+// scores instead of the logG row.
+template <int KREG>
+__global__ void __launch_bounds__(256) normalize_select_compact_kernel(const float* __restrict__ s,
+                                                                       float* __restrict__ lse,
+                                                                       float* __restrict__ tau,
+                                                                       int32_t* __restrict__ tau_idx,
+                                                                       int32_t* __restrict__ sel, long long rows,
+                                                                       int T, int NB, int H) {
+  __shared__ __align__(16) uint32_t hist_all[8][256];   // per-warp scratch of the select
+  const int wid = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * 8 + wid;
+  if (row >= rows) return;
+  const int t = (int)(row % T);
+  const int c = min(t / kBlock, NB);
+  int32_t* out = sel ? sel + row * (long long)H : nullptr;
+  normalize_select_row<KREG>(s + row * (long long)NB, nullptr, 0, c, NB, H, hist_all[wid], tau + row, tau_idx + row,
+                             out, lse + row);
 }
 
 // Packed sequences: the same per row, over the blocks of the row's own document
@@ -392,8 +419,9 @@ __global__ void __launch_bounds__(256) select_noisy_kernel(const float* __restri
 // gate gradient in log form): ds[m] = dLogG[m] - exp(logG[m]) * sum_{l<c} dLogG[l]
 // for m < c_t, 0 otherwise. One warp per row; HBM-bound.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) gate_grad_kernel(const float* __restrict__ logG, const float* __restrict__ dLogG,
-                                                        float* __restrict__ ds, long long rows, int T, int NB) {
+__global__ void __launch_bounds__(256) gate_grad_kernel(const float* __restrict__ logG, const float* __restrict__ lse,
+                                                        const float* __restrict__ dLogG, float* __restrict__ ds,
+                                                        long long rows, int T, int NB) {
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -406,7 +434,8 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const float* __restrict_
   for (int m = lane; m < c; m += 32) sum += __ldg(dl + m);
 #pragma unroll
   for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  for (int m = lane; m < NB; m += 32) out[m] = (m < c) ? __ldg(dl + m) - expf(__ldg(lg + m)) * sum : 0.f;
+  const float rl = (lse && c > 0) ? lse[row] : 0.f;   // raw scores: log g = s - LSE(s)
+  for (int m = lane; m < NB; m += 32) out[m] = (m < c) ? __ldg(dl + m) - expf(__ldg(lg + m) - rl) * sum : 0.f;
 }
 
 // ---------------------------------------------------------------------------
@@ -415,7 +444,8 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const float* __restrict_
 // masks[(bg * n_ptiles + pt) * NBW + w] bit i = block 32w + i is selected by
 // at least one position of the tile (current blocks not included).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) tile_union_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
+__global__ void __launch_bounds__(256) tile_union_kernel(const float* __restrict__ logG, const float* __restrict__ lse,
+                                                         const float* __restrict__ tau,
                                                          const int32_t* __restrict__ tau_idx,
                                                          uint32_t* __restrict__ masks, int T, int NB, int P,
                                                          int n_ptiles, int NBW) {
@@ -436,12 +466,13 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const float* __restrict
     const float tv = tau[row];
     const int ti = tau_idx[row];
     const float* v = logG + row * (long long)NB;
+    const float rl = (lse && c > 0) ? lse[row] : 0.f;   // raw scores: log g = s - LSE(s)
     for (int base = 0; base < c; base += 128) {   // four 32-block spans per round trip
       float x[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int m = base + 32 * u + lane;
-        x[u] = (m < c) ? v[m] : 0.f;
+        x[u] = (m < c) ? v[m] - rl : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -530,18 +561,34 @@ cudaError_t launch_select_noisy(const float* logG, const float* noise, float* lo
   return cudaGetLastError();
 }
 
-cudaError_t launch_gate_grad(const float* logG, const float* dLogG, float* ds, long long rows, int T, int NB,
-                             cudaStream_t st) {
-  gate_grad_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(logG, dLogG, ds, rows, T, NB);
+cudaError_t launch_normalize_select_compact(const float* s, float* lse, float* tau, int32_t* tau_idx, int32_t* sel,
+                                            long long rows, int T, int NB, int H, cudaStream_t st) {
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (NB <= 128)
+    normalize_select_compact_kernel<4><<<grid, 256, 0, st>>>(s, lse, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 256)
+    normalize_select_compact_kernel<8><<<grid, 256, 0, st>>>(s, lse, tau, tau_idx, sel, rows, T, NB, H);
+  else if (NB <= 512)
+    normalize_select_compact_kernel<16><<<grid, 256, 0, st>>>(s, lse, tau, tau_idx, sel, rows, T, NB, H);
+  else
+    normalize_select_compact_kernel<kSelectReg><<<grid, 256, 0, st>>>(s, lse, tau, tau_idx, sel, rows, T, NB, H);
   count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t launch_tile_union(const float* logG, const float* tau, const int32_t* tau_idx, uint32_t* masks,
-                              long long n_bg, int T, int NB, int P, int n_ptiles, int NBW, cudaStream_t st) {
+cudaError_t launch_gate_grad(const float* logG, const float* gate_lse, const float* dLogG, float* ds, long long rows,
+                             int T, int NB, cudaStream_t st) {
+  gate_grad_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(logG, gate_lse, dLogG, ds, rows, T, NB);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_union(const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
+                              uint32_t* masks, long long n_bg, int T, int NB, int P, int n_ptiles, int NBW,
+                              cudaStream_t st) {
   const long long blocks = n_bg * n_ptiles;
-  tile_union_kernel<<<(unsigned)blocks, 256, NBW * sizeof(uint32_t), st>>>(logG, tau, tau_idx, masks, T, NB, P,
-                                                                           n_ptiles, NBW);
+  tile_union_kernel<<<(unsigned)blocks, 256, NBW * sizeof(uint32_t), st>>>(logG, gate_lse, tau, tau_idx, masks, T, NB,
+                                                                           P, n_ptiles, NBW);
   count_launch();
   return cudaGetLastError();
 }

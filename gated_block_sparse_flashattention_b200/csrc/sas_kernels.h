@@ -30,10 +30,15 @@ cudaError_t launch_normalize_select_varlen(const float* s, float* logG, float* t
                                            cudaStream_t st);
 cudaError_t launch_select_noisy(const float* logG, const float* noise, float* logG_sel, float* tau, int32_t* tau_idx,
                                 int32_t* sel, long long rows, int T, int NB, int H, cudaStream_t st);
-cudaError_t launch_gate_grad(const float* logG, const float* dLogG, float* ds, long long rows, int T, int NB,
-                             cudaStream_t st);
-cudaError_t launch_tile_union(const float* logG, const float* tau, const int32_t* tau_idx, uint32_t* masks,
-                              long long n_bg, int T, int NB, int P, int n_ptiles, int NBW, cudaStream_t st);
+cudaError_t launch_gate_grad(const float* logG, const float* gate_lse, const float* dLogG, float* ds, long long rows,
+                             int T, int NB, cudaStream_t st);
+cudaError_t launch_tile_union(const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
+                              uint32_t* masks, long long n_bg, int T, int NB, int P, int n_ptiles, int NBW,
+                              cudaStream_t st);
+// Fused normalise + select writing the row LSE of the scores instead of logG
+// (rows of at most 32 * kSelectReg blocks).
+cudaError_t launch_normalize_select_compact(const float* s, float* lse, float* tau, int32_t* tau_idx, int32_t* sel,
+                                            long long rows, int T, int NB, int H, cudaStream_t st);
 
 // Shape of the query tiles of the tensor-core kernels: P consecutive positions
 // of one (b, g) times the G heads of the group, P a multiple of 8 with G*P <= 128.
@@ -52,7 +57,8 @@ struct TcProblem {
   const void* V;
   const void* O;    // bwd only
   const void* dO;   // bwd only
-  const float* logG;
+  const float* logG;      // log gates, or the raw scores s when gate_lse is set
+  const float* gate_lse;  // null, or [B*Hkv*T] LSE of each row's historical scores: log g = s - gate_lse
   const float* tau;
   const int32_t* tau_idx;
   const float* LSE;  // bwd only
@@ -76,7 +82,8 @@ struct BlockLists {
 };
 size_t block_lists_bytes(long long nbg, int T, int NB, int K);
 BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int K);
-cudaError_t launch_block_lists(const float* logG, const float* tau, const int32_t* tau_idx, const BlockLists& L,
+cudaError_t launch_block_lists(const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
+                               const BlockLists& L,
                                long long nbg, int T, int NB, int K, bool want_nsel, int32_t* status,
                                cudaStream_t st);
 

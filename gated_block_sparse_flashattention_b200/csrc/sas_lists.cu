@@ -37,15 +37,15 @@ constexpr int kChunkRows = 256;
 // 4 rows' 128-block spans are issued together, so a warp pays one round trip per
 // group and pass instead of one per row and 32 blocks.
 template <typename F, typename Done>
-__device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, const float* __restrict__ tau,
-                                              const int32_t* __restrict__ tau_idx, long long bg, int t0, int T,
-                                              int NB, F&& f, Done&& done) {
+__device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, const float* __restrict__ lse,
+                                              const float* __restrict__ tau, const int32_t* __restrict__ tau_idx,
+                                              long long bg, int t0, int T, int NB, F&& f, Done&& done) {
   constexpr int R = 4, U = 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
   const uint32_t below = (1u << lane) - 1u;
   const int t_end = min(T, t0 + kChunkRows);
   for (int tb = t0 + warp * R; tb < t_end; tb += n_warps * R) {
-    float tv[R];
+    float tv[R], rl[R];
     int ti[R], c[R], run[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -53,6 +53,7 @@ __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, co
       c[r] = (t < t_end) ? min(t / kBlock, NB) : 0;
       tv[r] = c[r] ? tau[bg * T + t] : 0.f;
       ti[r] = c[r] ? tau_idx[bg * T + t] : 0;
+      rl[r] = (c[r] && lse) ? lse[bg * T + t] : 0.f;   // compact gates: log g = s - LSE(s)
       run[r] = 0;
     }
     const int cmax = max(max(c[0], c[1]), max(c[2], c[3]));
@@ -62,7 +63,7 @@ __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, co
       for (int u = 0; u < U; ++u) {
         const int m = m0 + 32 * u + lane;
 #pragma unroll
-        for (int r = 0; r < R; ++r) x[u][r] = (m < c[r]) ? logG[(bg * T + tb + r) * (long long)NB + m] : 0.f;
+        for (int r = 0; r < R; ++r) x[u][r] = (m < c[r]) ? logG[(bg * T + tb + r) * (long long)NB + m] - rl[r] : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -86,7 +87,8 @@ __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, co
 // (pairs beyond the row's K-1 slots excluded), and keep each chunk's counts
 // ccnt[b, g, chunk, block] for the fill. Grid: (chunks of T, B * Hkv); dynamic
 // shared memory: NB ints.
-__global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
+__global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ lse,
+                                                    const float* __restrict__ tau,
                                                     const int32_t* __restrict__ tau_idx, int32_t* __restrict__ cnt,
                                                     int32_t* __restrict__ ccnt, int32_t* status, int T, int NB,
                                                     int H) {
@@ -97,7 +99,7 @@ __global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ lo
   __syncthreads();
   bool over = false;
   for_each_pair(
-      logG, tau, tau_idx, bg, t0, T, NB,
+      logG, lse, tau, tau_idx, bg, t0, T, NB,
       [&](int, int m, int rank) {
         if (rank < H) atomicAdd(hist + m, 1);
       },
@@ -178,7 +180,8 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
 // free one. Also writes nsel[t], the number of selected blocks of each row
 // (capped at H), when nsel is not null. Grid: (chunks of T, B * Hkv); dynamic
 // shared memory: 2 * NB ints.
-__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ tau,
+__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ lse,
+                                                   const float* __restrict__ tau,
                                                    const int32_t* __restrict__ tau_idx,
                                                    const int32_t* __restrict__ off, const int32_t* __restrict__ cap,
                                                    const int32_t* __restrict__ cbase, int32_t* __restrict__ list,
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ log
   }
   __syncthreads();
   for_each_pair(
-      logG, tau, tau_idx, bg, t0, T, NB,
+      logG, lse, tau, tau_idx, bg, t0, T, NB,
       [&](int t, int m, int rank) {
         if (rank >= H) return;
         const int at = lbase[m] + atomicAdd(lcnt + m, 1);
@@ -241,7 +244,8 @@ BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int
   return L;
 }
 
-cudaError_t launch_block_lists(const float* logG, const float* tau, const int32_t* tau_idx, const BlockLists& L,
+cudaError_t launch_block_lists(const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
+                               const BlockLists& L,
                                long long nbg, int T, int NB, int K, bool want_nsel, int32_t* status,
                                cudaStream_t st) {
   using namespace lists;
@@ -250,12 +254,13 @@ cudaError_t launch_block_lists(const float* logG, const float* tau, const int32_
   cudaError_t e = cudaMemsetAsync(L.cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const dim3 chunks((unsigned)n_chunks, (unsigned)nbg);
-  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(logG, tau, tau_idx, L.cnt, L.ccnt, status, T, NB, H);
+  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(logG, gate_lse, tau, tau_idx, L.cnt, L.ccnt, status, T,
+                                                           NB, H);
   count_launch();
   offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(L.cnt, L.off, L.ccnt, L.cap, L.total, status, NB, n_chunks,
                                                    L.region);
   count_launch();
-  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(logG, tau, tau_idx, L.off, L.cap, L.ccnt, L.list,
+  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(logG, gate_lse, tau, tau_idx, L.off, L.cap, L.ccnt, L.list,
                                                               want_nsel ? L.nsel : nullptr, T, NB, H);
   count_launch();
   return cudaGetLastError();

@@ -18,7 +18,8 @@ struct Params {
   const float* V;
   const float* O;
   const float* dO;
-  const float* logG;
+  const float* logG;       // log gates, or raw scores when gate_lse is set
+  const float* gate_lse;   // null, or the LSE of each row's historical scores
   const float* tau;
   const int32_t* tau_idx;
   const float* LSE;
@@ -46,11 +47,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Next attended block after `m` for this row, in the order: current block c,
 // then historical blocks 0..c-1 that pass the threshold. Returns -1 at the end.
-__device__ __forceinline__ int next_block(int m, int c, const float* gate, float tau, int tidx) {
+__device__ __forceinline__ int next_block(int m, int c, const float* gate, float rl, float tau, int tidx) {
   int cand = (m == c) ? 0 : m + 1;
   if (m < 0) return c;
   for (; cand < c; ++cand) {
-    const float v = gate[cand];
+    const float v = gate[cand] - rl;
     if (v > tau || (v == tau && cand <= tidx)) return cand;
   }
   return -1;
@@ -73,6 +74,7 @@ __global__ void fwd_kernel(const Params p) {
   const float* Kb = p.K + bg * (long long)p.T * D;
   const float* Vb = p.V + bg * (long long)p.T * D;
   const float* gate = p.logG + row * (long long)p.NB;
+  const float rl = p.gate_lse ? p.gate_lse[row] : 0.f;   // raw scores: log g = s - LSE(s)
   const float tau = p.tau[row];
   const int tidx = p.tau_idx[row];
   const int c = t / kBlock;
@@ -80,8 +82,8 @@ __global__ void fwd_kernel(const Params p) {
   float acc[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) acc[i] = 0.f;
-  for (int m = next_block(-1, c, gate, tau, tidx); m >= 0; m = next_block(m, c, gate, tau, tidx)) {
-    const float bias = (m == c) ? 0.f : gate[m];
+  for (int m = next_block(-1, c, gate, rl, tau, tidx); m >= 0; m = next_block(m, c, gate, rl, tau, tidx)) {
+    const float bias = (m == c) ? 0.f : gate[m] - rl;
     for (int ch = 0; ch < 2; ++ch) {
       const int key = m * kBlock + ch * 32 + lane;
       const bool ok = (m != c) || key <= t;
@@ -153,6 +155,7 @@ __global__ void bwd_kernel(const Params p) {
   float* dKb = p.dK + bg * (long long)p.T * D;
   float* dVb = p.dV + bg * (long long)p.T * D;
   const float* gate = p.logG + row * (long long)p.NB;
+  const float rl = p.gate_lse ? p.gate_lse[row] : 0.f;   // raw scores: log g = s - LSE(s)
   const float tau = p.tau[row];
   const int tidx = p.tau_idx[row];
   const int c = t / kBlock;
@@ -161,8 +164,8 @@ __global__ void bwd_kernel(const Params p) {
   float dq[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) dq[i] = 0.f;
-  for (int m = next_block(-1, c, gate, tau, tidx); m >= 0; m = next_block(m, c, gate, tau, tidx)) {
-    const float bias = (m == c) ? 0.f : gate[m];
+  for (int m = next_block(-1, c, gate, rl, tau, tidx); m >= 0; m = next_block(m, c, gate, rl, tau, tidx)) {
+    const float bias = (m == c) ? 0.f : gate[m] - rl;
     float blk = 0.f;
     for (int ch = 0; ch < 2; ++ch) {
       const int key = m * kBlock + ch * 32 + lane;
@@ -218,6 +221,7 @@ Params make_params(const TcProblem& pb) {
   prm.O = static_cast<const float*>(pb.O);
   prm.dO = static_cast<const float*>(pb.dO);
   prm.logG = pb.logG;
+  prm.gate_lse = pb.gate_lse;
   prm.tau = pb.tau;
   prm.tau_idx = pb.tau_idx;
   prm.LSE = pb.LSE;

@@ -68,6 +68,8 @@ WORKLOADS = {
     # Long-context decode over a paged cache: 8 sequences, one new token each at 512K
     # context, budget 2048 tokens (32 blocks, the current one included).
     "decode_b8_l512k_paged": Workload("decode_b8_l512k_paged", "bf16", 8, 32, 8, 128, 524288, 32, decode=True),
+    # The same at 64K context (a 2 GB pool), for profiling runs.
+    "decode_b8_l64k_paged": Workload("decode_b8_l64k_paged", "bf16", 8, 32, 8, 128, 65536, 32, decode=True),
 }
 
 

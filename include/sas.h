@@ -22,7 +22,8 @@
  *     sequences of documents (§5.1).
  *
  * Entry points: sas_gate_normalize, sas_select_threshold and their fused form
- * sas_gate_normalize_select (and _varlen for packed documents), sas_select_noisy,
+ * sas_gate_normalize_select (and _varlen for packed documents, _compact for
+ * gates kept as scores + a row log-sum-exp), sas_select_noisy,
  * sas_fwd, sas_bwd, sas_gate_grad, sas_decode_fwd (and _paged, _static), the
  * workspace sizes, the device status word, sas_status_string, sas_version and
  * sas_launch_count.
@@ -139,6 +140,24 @@ SAS_API int sas_gate_normalize_select(const float* s, float* logG, float* tau, i
                                       int Hkv, int T, int NB, int block, int K, void* stream);
 
 /*
+ * sas_gate_normalize_select_compact - sas_gate_normalize_select without the logG
+ * tensor (SAS paper §4.2 eq. 6: log g = s - log sum exp over the historical
+ * blocks; Appendix D.3). It writes, per (b, g, t), the log-sum-exp of the row's
+ * historical scores,
+ *   gate_lse[b,g,t] = log sum_{m < c_t} exp(s[b,g,t,m])     (-inf when c_t = 0),
+ * and tau, tau_idx, sel exactly as sas_gate_normalize_select does (bit for bit):
+ * the selection is taken on logG[m] = s[m] - gate_lse (one fp32 subtraction,
+ * the value sas_gate_normalize writes). sas_fwd, sas_bwd and sas_gate_grad given
+ * s in place of logG together with gate_lse rebuild the same gates, so a
+ * training step reads s where it read logG and never writes the dense logG.
+ * gate_lse: [B, Hkv, T] fp32. Other arguments as for sas_gate_normalize_select;
+ * NB <= 1024 (else SAS_ERR_UNSUPPORTED).
+ */
+SAS_API int sas_gate_normalize_select_compact(const float* s, float* gate_lse, float* tau, int32_t* tau_idx,
+                                              int32_t* sel, int B, int Hkv, int T, int NB, int block, int K,
+                                              void* stream);
+
+/*
  * sas_gate_normalize_select_varlen - sas_gate_normalize_select for a packed
  * sequence of documents (SAS paper §5.1: training on packed sequences). Document
  * i covers tokens cu_seqlens[i] .. cu_seqlens[i+1]-1 and blocks
@@ -194,10 +213,13 @@ SAS_API int sas_select_noisy(const float* logG, const float* noise, float* logG_
  *   ds[b,g,t,m] = dLogG[b,g,t,m] - exp(logG[b,g,t,m]) * sum_{l < c_t} dLogG[b,g,t,l]  for m < c_t,
  *   ds[b,g,t,m] = 0                                                                   for m >= c_t.
  * logG (from sas_gate_normalize), dLogG, ds: [B,Hkv,T,NB] fp32; ds may not alias
- * either input. NB >= ceil(T / block), block == 64.
+ * either input. With gate_lse non-null (compact gates from
+ * sas_gate_normalize_select_compact), `logG` holds the raw scores s and
+ * logG[m] = s[m] - gate_lse[b,g,t] is rebuilt in fp32. NB >= ceil(T / block),
+ * block == 64.
  */
-SAS_API int sas_gate_grad(const float* logG, const float* dLogG, float* ds, int B, int Hkv, int T, int NB, int block,
-                          void* stream);
+SAS_API int sas_gate_grad(const float* logG, const float* gate_lse, const float* dLogG, float* ds, int B, int Hkv,
+                          int T, int NB, int block, void* stream);
 
 /*
  * Workspace sizes (bytes) for sas_fwd, sas_bwd and sas_decode_fwd with the given
@@ -221,6 +243,10 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * -inf for every other key.
  * Q [B,Hq,T,d], K/V [B,Hkv,T,d] of `dtype`; logG [B,Hkv,T,NB], tau, tau_idx as
  * produced by the two calls above (any values obeying their contract work).
+ * gate_lse: null, or (compact gates, sas_gate_normalize_select_compact) the
+ * [B,Hkv,T] log-sum-exp of each row's historical scores, with the raw scores s
+ * passed as `logG`: the gate is then s[m] - gate_lse[b,g,t] in fp32, bit for bit
+ * the normalised gate.
  * O [B,Hq,T,d] of `dtype`; LSE [B,Hq,T] fp32. T % 64 == 0, NB == T / 64,
  * Hq % Hkv == 0, d in {64, 128} (fp32) or d == 128 (bf16).
  * Kbudget: the budget K given to the selection (the threshold keeps at most K-1
@@ -233,9 +259,9 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * workspace is small.
  * ws: workspace of sas_fwd_workspace_size bytes (same K).
  */
-SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* tau,
-            const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d, int block,
-            int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream);
+SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* gate_lse,
+            const float* tau, const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d,
+            int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * sas_bwd - gradients of a scalar loss through sas_fwd (SAS paper Appendix E
@@ -243,7 +269,8 @@ SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, cons
  *   P = exp(z - LSE), Delta = rowsum(O * dO), dS = P * (dO V^T - Delta),
  *   dQ = sm_scale dS K,  dK = sm_scale sum_{h in g} dS^T Q,  dV = sum_{h in g} P^T dO,
  *   dLogG[b,g,t,m] = sum_{h in g} sum_{i in block m} dS[h,t,i] for selected m, 0 otherwise.
- * Inputs as for sas_fwd plus O (the forward output), dO and LSE (the forward's).
+ * Inputs as for sas_fwd (gate_lse included) plus O (the forward output), dO and
+ * LSE (the forward's).
  * Outputs dQ [B,Hq,T,d], dK/dV [B,Hkv,T,d] of `dtype`; dLogG [B,Hkv,T,NB] fp32
  * (fully written: zero outside the selection). Kbudget: the budget K given to
  * sas_select_threshold (the threshold keeps at most K-1 historical blocks per row;
@@ -252,9 +279,9 @@ SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, cons
  * (for bf16 it holds an fp32 dQ accumulator and the per-block row lists).
  */
 SAS_API int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
-            const float* logG, const float* tau, const int32_t* tau_idx, const float* LSE, void* dQ, void* dK,
-            void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget, float sm_scale,
-            void* ws, size_t ws_bytes, void* stream);
+            const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx, const float* LSE,
+            void* dQ, void* dK, void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget,
+            float sm_scale, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * sas_decode_fwd - one sparse decode step per sequence (SAS paper §4.3

@@ -72,6 +72,27 @@ def gate_normalize(s, block: int):
     return out
 
 
+def gate_lse(s, block: int):
+    """Return ``lse[..., t] = log sum_{m < c_t} exp(s[..., t, m])``, the normaliser of eq. 6 (SAS paper
+    §4.2 "Activation function": log g = s - log sum exp over the historical blocks).
+
+    The compact form of the gates keeps s and this per-row value instead of logG:
+    ``logG[..., t, m] = s[..., t, m] - lse[..., t]`` for m < c_t. Rows with ``c_t == 0``
+    have no historical block: -inf. s: [B, Hkv, T, NB]. Returns float64 [B, Hkv, T].
+    """
+    s = _f64(s)
+    B, Hkv, T, NB = s.shape
+    out = np.full((B, Hkv, T), NEG_INF)
+    for t in range(T):
+        c = t // block
+        if c == 0:
+            continue
+        hist = s[:, :, t, :c]
+        mx = hist.max(axis=-1)
+        out[:, :, t] = mx + np.log(np.exp(hist - mx[..., None]).sum(axis=-1))
+    return out
+
+
 # --------------------------------------------------------------------------------------
 # Selector-score gradient: SAS paper Appendix D.3 "Gradient Derivation for Training
 # Scope" (the softmax backward ds_m = g_m (dg_m - sum_l g_l dg_l)) and §4.2 eq. 8.

@@ -108,9 +108,15 @@ def test_invalid_calls_return_errors_without_launching(lib):
     assert vl(cu(0, 128, 128, 256), 3) == -1     # an empty document
     assert vl(cu(0, 256), 0) == -1               # no document
     assert vl(cu(*range(0, 64 * 258, 64)), 257, T=64 * 257) == -2   # more than 256 documents
-    assert lib.sas_gate_grad(fake, fake + 64, fake + 64, 1, 1, 128, 2, 64, None) == -1   # ds aliases dLogG
-    assert lib.sas_gate_grad(fake, fake + 64, fake + 132, 1, 1, 128, 2, 64, None) == -1  # misaligned ds
-    assert lib.sas_gate_grad(fake, fake + 64, fake + 128, 1, 1, 128, 2, 32, None) == -1  # block != 64
+    assert lib.sas_gate_grad(fake, None, fake + 64, fake + 64, 1, 1, 128, 2, 64, None) == -1   # ds aliases dLogG
+    assert lib.sas_gate_grad(fake, None, fake + 64, fake + 132, 1, 1, 128, 2, 64, None) == -1  # misaligned ds
+    assert lib.sas_gate_grad(fake, None, fake + 64, fake + 128, 1, 1, 128, 2, 32, None) == -1  # block != 64
+    assert lib.sas_gate_grad(fake, fake + 4, fake + 64, fake + 128, 1, 1, 128, 2, 64, None) == -1  # misaligned LSE
+    # compact normalise + select: rows over 1024 blocks, a missing LSE output
+    assert lib.sas_gate_normalize_select_compact(fake, fake + 64, fake + 128, fake + 192, None, 1, 1, 128 * 64, 2048,
+                                                 64, 4, None) == -2
+    assert lib.sas_gate_normalize_select_compact(fake, None, fake + 128, fake + 192, None, 1, 1, 128, 2, 64, 4,
+                                                 None) == -1
     # paged decode: fp32 storage is not implemented; NBmax below max_pages is invalid
     paged = [fake] * 3 + [binding.SAS_DT_F32, fake, 4, 8, fake, fake, 4, 0, fake, None, 1, 4, 1, 4, 128, 64,
                           ctypes.c_float(0.1), fake, 1 << 20, None]
@@ -119,14 +125,17 @@ def test_invalid_calls_return_errors_without_launching(lib):
     paged[16] = 3                 # NBmax < max_pages
     assert lib.sas_decode_fwd_paged(*paged) == -1
     # sas_fwd: missing workspace / bad sizes
-    args = [fake] * 3 + [binding.SAS_DT_BF16] + [fake] * 5 + [1, 4, 1, 128, 128, 64, 2, ctypes.c_float(0.1), None, 0,
-                                                              None]
+    args = ([fake] * 3 + [binding.SAS_DT_BF16] + [fake, None] + [fake] * 4
+            + [1, 4, 1, 128, 128, 64, 2, ctypes.c_float(0.1), None, 0, None])
     assert lib.sas_fwd(*args) == -5
     args[-3] = fake
     args[-2] = 1 << 30
-    args[12] = 100   # T not a multiple of 64
+    args[13] = 100   # T not a multiple of 64
     assert lib.sas_fwd(*args) == -1
-    args[12] = 128
-    args[15] = 0     # budget K < 1
+    args[13] = 128
+    args[16] = 0     # budget K < 1
+    assert lib.sas_fwd(*args) == -1
+    args[16] = 2
+    args[5] = fake + 4   # misaligned row LSE of compact gates
     assert lib.sas_fwd(*args) == -1
     assert lib.sas_launch_count() == before

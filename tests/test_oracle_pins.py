@@ -88,6 +88,37 @@ def test_normalize_matches_log_softmax_prefix():
             np.testing.assert_allclose(logG[:, :, t, :c], ref, rtol=1e-13, atol=1e-13)
 
 
+def test_gate_lse_matches_torch_logsumexp_prefix():
+    """The compact gates' row normaliser is torch.logsumexp over the causal block prefix, -inf with no
+    history; with it the raw scores give back gate_normalize's log gates (eq. 6)."""
+    block, T = 16, 112
+    s = 3.0 * _rand((2, 2, T, T // block), 21)
+    lse = orc.gate_lse(s, block)
+    st = torch.from_numpy(s)
+    for t in range(T):
+        c = t // block
+        if c == 0:
+            assert np.all(np.isneginf(lse[:, :, t]))
+            continue
+        ref = torch.logsumexp(st[:, :, t, :c], dim=-1).numpy()
+        assert np.allclose(lse[:, :, t], ref, rtol=0, atol=1e-12)
+    lg = orc.gate_normalize(s, block)
+    c_t = np.arange(T) // block
+    hist = np.arange(T // block)[None, :] < c_t[:, None]
+    assert np.allclose(np.where(hist, s - lse[..., None], -np.inf)[..., hist], lg[..., hist], rtol=0, atol=1e-12)
+
+
+def test_gate_lse_pin_catches_a_planted_mistake():
+    """A normaliser over the wrong prefix (the current block included) fails the logsumexp pin."""
+    block, T = 16, 80
+    s = _rand((1, 1, T, T // block), 22)
+    wrong = np.array([[[np.logaddexp.reduce(s[0, 0, t, :t // block + 1]) if t >= block else -np.inf
+                        for t in range(T)]]])
+    ref = torch.logsumexp(torch.from_numpy(s)[0, 0, 40, :40 // block], dim=-1).item()
+    assert abs(orc.gate_lse(s, block)[0, 0, 40] - ref) < 1e-12
+    assert abs(wrong[0, 0, 40] - ref) > 1e-3
+
+
 def test_normalize_shift_invariance_and_unit_mass():
     block, T = 8, 96
     s = _rand((1, 2, T, T // block), 2) * 3
