@@ -40,17 +40,23 @@ namespace sas {
 namespace gbwd {
 
 constexpr int D = 128;
-// Warps 0-3: softmax / dS (one thread per tile row); warp 4: control (row
-// positions of each tile, the next tile's loaded ahead; K/V load); warp 5: MMA
-// issuer; warps 6-9: dQ flush (TMEM -> shared-memory staging -> fp32 reductions
-// of whole row segments); warps 10-15: Q/dO row
-// and gate gathers. The gather
-// bandwidth one SM sustains grows with the number of warps issuing copies, so
-// most warps load; the softmax works on 32 key columns at a time to keep the
-// kernel within 128 registers per thread.
+// Warps 0-3: softmax / dS (one thread per tile row); warp 4: control (K/V
+// load; per tile the row positions, then the copies of each row's gate, score
+// LSE and chunk tail into a metadata ring that runs up to MST tiles ahead of
+// the rows); warp 5: MMA issuer; warps 6-9: dQ flush (TMEM -> shared-memory
+// staging -> fp32 reductions of whole row segments); warps 10-15: Q/dO row
+// gathers. A Q/dO stage is busy from its gather to the tile's dK/dV MMAs, and
+// only two fit in shared memory, so the gather of a tile starts when the tile
+// two back has finished: the small scattered metadata loads (with the longest
+// latency of the tile's copies) are taken out of that cycle by the metadata
+// ring. The gather bandwidth one SM sustains grows with the number of warps
+// issuing copies, so most warps load; the softmax works on 32 key columns at a
+// time to keep the kernel within 128 registers per thread.
 constexpr int THREADS = 512;
 constexpr int LOADER_WARP0 = 10, N_LOADER_WARPS = 6;
 constexpr int NST = 2;                           // Q/dO gather stages
+constexpr int MST = 4;                           // metadata stages
+constexpr int MLAG = 2;                          // metadata tiles in flight per control lane beyond the oldest
 constexpr uint32_t HALF128 = 128 * 128;          // one d-half of a 128-row tile
 constexpr uint32_t TILE = 2 * HALF128;           // 128 rows x 128 features, bf16
 constexpr uint32_t KV_HALF = 64 * 128;
@@ -59,15 +65,16 @@ constexpr uint32_t OFF_V = 2 * KV_HALF;
 constexpr uint32_t OFF_QD = 4 * KV_HALF;                  // stage s: Q at +2s*TILE, dO at +(2s+1)*TILE
 constexpr uint32_t OFF_P = OFF_QD + NST * 2 * TILE;       // P  [128 rows][64 keys] bf16 (16 KiB)
 constexpr uint32_t OFF_DS = OFF_P + 128 * 128;            // dS [128 rows][64 keys] bf16 (16 KiB)
-// Per stage: the tile's positions [128] int, the gate score of each position for
-// block j [128] float and its row's score LSE [128] float (0 unless the gates
-// come as raw scores), and the chunk tails (LSE and Delta of the G heads) of
-// each position, `tail` bytes apiece (P positions * tail <= 2 KiB for every G).
+// Per metadata stage: the tile's positions [128] int, the gate score of each
+// position for block j [128] float and its row's score LSE [128] float (0 unless
+// the gates come as raw scores), and the chunk tails (LSE and Delta of the G
+// heads) of each position, `tail` bytes apiece (P positions * tail <= 2 KiB for
+// every G).
 constexpr uint32_t CMETA_STAGE = 2048;
 constexpr uint32_t OFF_META = OFF_DS + 128 * 128;
 constexpr uint32_t META_STAGE = 3 * 128 * 4;   // positions, gate scores, row score LSEs (compact gates)
-constexpr uint32_t OFF_CMETA = OFF_META + NST * META_STAGE;
-constexpr uint32_t OFF_QROW = OFF_CMETA + NST * CMETA_STAGE;   // [2][128] global row of each dQ buffer row (-1: none)
+constexpr uint32_t OFF_CMETA = OFF_META + MST * META_STAGE;
+constexpr uint32_t OFF_QROW = OFF_CMETA + MST * CMETA_STAGE;   // [2][128] global row of each dQ buffer row (-1: none)
 constexpr uint32_t OFF_RED = OFF_QROW + 2 * 128 * 4;      // [2][128] fp32 row sums for dLogG
 // dQ flush staging: per flush warp one 32-column chunk of its 32 rows (fp32,
 // 16-byte pieces XOR-swizzled by row), so that each reduction instruction adds
@@ -78,6 +85,7 @@ constexpr uint32_t DQS_WARP_BYTES = 32 * 128;
 constexpr uint32_t OFF_BAR = OFF_DQS + 4 * DQS_WARP_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 // TMEM columns
 constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DV = 128, COL_DK = 192, COL_DQ0 = 256, TMEM_COLS = 512;
 
@@ -104,15 +112,17 @@ struct Params {
   int32_t* dl_idx;           // [list entry] t * NB + j of the entry's dLogG element within its (b, g)
   int32_t* status;
   int B, Hq, Hkv, T, NB, G, P;
+  int group_major;           // CTA order: 1 group-major, 0 block-major
   float scale_log2;
   float sm_scale;
   uint64_t wait_ns;          // limit of one bounded wait
 };
 
 struct Bars {
-  uint64_t kv_full, pos_ready[NST], qd_full[NST], qd_empty[NST], s_full, sp_free, p_full, pd_free, dq_done[2],
-      dq_free[2], qrow_full[2], fin;
+  uint64_t kv_full, pos_ready[MST], meta_full[MST], meta_empty[MST], qd_full[NST], qd_empty[NST], s_full, sp_free,
+      p_full, pd_free, dq_done[2], dq_free[2], qrow_full[2], fin;
 };
+static_assert(sizeof(Bars) <= 256, "barrier area");
 
 // Position of list entry `idx` of block j: the block's own positions first, then the selecting rows.
 __device__ __forceinline__ int tile_position(const int32_t* lst, int own_n, int total, int j, int idx) {
@@ -159,15 +169,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Block-major order: block j is attended by its own positions and by the later
-  // positions that select it, so small j carry the longest row lists. Launching
-  // them first (all groups' block 0, then block 1, ...) leaves the short lists to
-  // fill the SMs at the end. (Measured: group-major order, which keeps one
-  // group's rows in L2, was 17% slower at 8K tokens and no faster at 32K: its
-  // last group's long lists start late.)
+  // CTA order. Block j is attended by its own positions and by the later
+  // positions that select it, so small j carry the longest row lists. Group-major
+  // order (all blocks of (b, g) 0, then of (b, g) 1, ...) keeps the rows that the
+  // running CTAs gather and reduce into within about one group, which fits L2
+  // far better than all groups' (DRAM traffic of the 32K-token layer: 14 GB
+  // instead of 61 GB), but the last group's long lists start late. That tail
+  // matters when a group is less than two waves of CTAs; those problems run
+  // block-major (every group's block 0, then block 1, ...), which starts all
+  // long lists first.
   const int n_bg = p.B * p.Hkv;
-  const int bg = blockIdx.x % n_bg;
-  const int j = blockIdx.x / n_bg;
+  const int bg = p.group_major ? (int)(blockIdx.x / p.NB) : (int)(blockIdx.x % n_bg);
+  const int j = p.group_major ? (int)(blockIdx.x % p.NB) : (int)(blockIdx.x / n_bg);
   const uint64_t wait_ns = p.wait_ns;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int PP = p.P, G = p.G;
@@ -183,9 +196,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 5) tmem_alloc(tmem_slot, TMEM_COLS);
   if (tid == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int i = 0; i < NST; ++i) {
+    for (int i = 0; i < MST; ++i) {
       mbar_init(&bars->pos_ready[i], 1);
-      mbar_init(&bars->qd_full[i], 1 + N_LOADER_WARPS);   // control (metadata) + loader warps (rows)
+      mbar_init(&bars->meta_full[i], 1);
+      mbar_init(&bars->meta_empty[i], 4);   // softmax warps
+    }
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&bars->qd_full[i], N_LOADER_WARPS);
       mbar_init(&bars->qd_empty[i], 1);
     }
     mbar_init(&bars->s_full, 1);
@@ -231,48 +248,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int u = 0; u < 4; ++u)
         tl[u] = (lane + 32 * u < PP) ? tile_position(lst, own_n, total, j, i * PP + lane + 32 * u) : -1;
     };
+    const int tail_bytes = p.chunk - 512 * G;   // LSE and Delta of the G heads, padded to 16 bytes
+    const uint8_t* base = p.packed + (long long)bg * p.T * p.chunk;
     int cur[4], nxt[4] = {-1, -1, -1, -1};
     load_pos(0, cur);
+    int issued = 0;
     for (int i = 0; i < n_tiles; ++i) {
-      const int st = i % NST;
+      const int ms = i % MST;
       if (i + 1 < n_tiles) load_pos(i + 1, nxt);
       bool ok = true;
-      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status, wait_ns);
+      if (i >= MST) ok = mbar_wait(&bars->meta_empty[ms], ((i / MST) - 1) & 1, status, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      int* pos = reinterpret_cast<int*>(smem + OFF_META + st * META_STAGE);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (lane + 32 * u < PP) pos[lane + 32 * u] = cur[u];
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars->pos_ready[st]);
-        mbar_arrive(&bars->qd_full[st]);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
-    }
-    if (lane == 0) mbar_wait_drain(&bars->kv_full, 0);
-  } else if (warp >= LOADER_WARP0) {
-    // ------------------------------------------------------------------ loaders: Q / dO row gathers
-    const int lt = tid - LOADER_WARP0 * 32;
-    constexpr int NL = N_LOADER_WARPS * 32;
-    for (int i = 0; i < n_tiles; ++i) {
-      const int st = i % NST;
-      bool ok = true;
-      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status, wait_ns);
-      if (ok) ok = mbar_wait(&bars->pos_ready[st], (i / NST) & 1, status, wait_ns);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
-      float* gate = reinterpret_cast<float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
+      int* pos = reinterpret_cast<int*>(smem + OFF_META + ms * META_STAGE);
+      float* gate = reinterpret_cast<float*>(pos + 128);
       float* glse = gate + 128;
-      const int first = pos[0];
-      // The gate of block j for each selecting position (0 for own positions and
-      // empty slots), with its row's score LSE when the gates come as raw scores,
-      // copied in the same group as the rows.
-      for (int pp = lt; pp < PP; pp += NL) {
-        const int t = pos[pp];
+      const uint32_t cm = s_base + OFF_CMETA + ms * CMETA_STAGE;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int pp = lane + 32 * u;
+        if (pp >= PP) continue;
+        const int t = cur[u];
+        pos[pp] = t;
+        // The gate of block j for each selecting position (0 for own positions and
+        // empty slots), with its row's score LSE when the gates come as raw scores.
         if (t >= 0 && t / kBlock != j) {
           cp_async4(smem_u32(gate + pp), p.logG + ((long long)bg * p.T + t) * p.NB + j);
           if (p.gate_lse)
@@ -283,36 +282,64 @@ __global__ void __launch_bounds__(THREADS, 1)
           gate[pp] = 0.f;
           glse[pp] = 0.f;
         }
+        if (t >= 0)
+          for (int k = 0; k < tail_bytes; k += 16)
+            cp_async16(cm + pp * tail_bytes + k, base + (long long)t * p.chunk + 512 * G + k);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->pos_ready[ms]);
+      cp_async_commit();
+      ++issued;
+      // Tile i-MLAG's metadata is published once it has landed, with the copies of
+      // tiles i-MLAG+1 .. i still in flight.
+      if (i >= MLAG) {
+        cp_async_wait_group<MLAG>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->meta_full[(i - MLAG) % MST]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
+    }
+    cp_async_wait_all();   // after a failed wait too: no copy may outlive the CTA
+    __syncwarp();
+    if (lane == 0)
+      for (int k = max(0, issued - MLAG); k < issued; ++k) mbar_arrive(&bars->meta_full[k % MST]);
+    if (lane == 0) mbar_wait_drain(&bars->kv_full, 0);
+  } else if (warp >= LOADER_WARP0) {
+    // ------------------------------------------------------------------ loaders: Q / dO row gathers
+    const int lt = tid - LOADER_WARP0 * 32;
+    constexpr int NL = N_LOADER_WARPS * 32;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i % NST, ms = i % MST;
+      bool ok = true;
+      if (i >= NST) ok = mbar_wait(&bars->qd_empty[st], ((i / NST) - 1) & 1, status, wait_ns);
+      if (ok) ok = mbar_wait(&bars->pos_ready[ms], (i / MST) & 1, status, wait_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int* pos = reinterpret_cast<const int*>(smem + OFF_META + ms * META_STAGE);
+      const int first = pos[0];
       const uint32_t qd = s_base + OFF_QD + st * 2 * TILE;
-      const uint32_t cm = s_base + OFF_CMETA + st * CMETA_STAGE;
-      // Pieces of 16 bytes of each position's chunk: 32*G of Q/dO rows (ordered
-      // tensor, head, piece), then the tail. The loaders walk (position, piece)
-      // with a stride of NL pieces, so consecutive lanes copy consecutive bytes.
+      // Pieces of 16 bytes of the Q/dO rows of each position's chunk: 32*G of them
+      // (ordered tensor, head, piece). The loaders walk (position, piece) with a
+      // stride of NL pieces, so consecutive lanes copy consecutive bytes.
       const int rows_pieces = 32 * G;
-      const int per_pos = p.chunk >> 4;
-      const int tail_bytes = p.chunk - rows_pieces * 16;
       const uint8_t* base = p.packed + (long long)bg * p.T * p.chunk;
       int pp = 0, piece = lt;
-      while (piece >= per_pos) {
-        piece -= per_pos;
+      while (piece >= rows_pieces) {
+        piece -= rows_pieces;
         ++pp;
       }
       while (pp < PP) {
         const int t0 = pos[pp];
         const uint8_t* src = base + (long long)(t0 >= 0 ? t0 : first) * p.chunk + piece * 16;
-        if (piece < rows_pieces) {
-          const int tensor = piece >= 16 * G;
-          const int rem2 = piece - tensor * 16 * G;
-          const int hh = rem2 >> 4, c16 = rem2 & 15;
-          const int half = c16 >> 3, ch = c16 & 7;
-          cp_async16(qd + tensor * TILE + half * HALF128 + sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)ch), src);
-        } else {
-          cp_async16(cm + pp * tail_bytes + (piece - rows_pieces) * 16, src);
-        }
+        const int tensor = piece >= 16 * G;
+        const int rem2 = piece - tensor * 16 * G;
+        const int hh = rem2 >> 4, c16 = rem2 & 15;
+        const int half = c16 >> 3, ch = c16 & 7;
+        cp_async16(qd + tensor * TILE + half * HALF128 + sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)ch), src);
         piece += NL;
-        while (piece >= per_pos) {
-          piece -= per_pos;
+        while (piece >= rows_pieces) {
+          piece -= rows_pieces;
           ++pp;
         }
       }
@@ -422,23 +449,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      const int st = i % NST, qb = i & 1;
-      bool step_ok = warp_wait(&bars->qd_full[st], (i / NST) & 1, status, wait_ns);
+      const int st = i % NST, ms = i % MST, qb = i & 1;
+      bool step_ok = warp_wait(&bars->meta_full[ms], (i / MST) & 1, status, wait_ns);
+      if (step_ok) step_ok = warp_wait(&bars->qd_full[st], (i / NST) & 1, status, wait_ns);
       int t = -1;
       float lse2 = 0.f, dlt = 0.f, bias2 = 0.f;
       if (step_ok && r < rows_used) {
         const int pp = r % PP;
-        t = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE)[pp];
+        t = reinterpret_cast<const int*>(smem + OFF_META + ms * META_STAGE)[pp];
         if (t >= 0) {
           const float* tail =
-              reinterpret_cast<const float*>(smem + OFF_CMETA + st * CMETA_STAGE + pp * (p.chunk - 512 * G));
+              reinterpret_cast<const float*>(smem + OFF_CMETA + ms * CMETA_STAGE + pp * (p.chunk - 512 * G));
           lse2 = tail[hh] * kLog2e;
           dlt = tail[G + hh];
           // log g = s - LSE(s) in fp32 (bit-identical to the normalised gate), then log2 units
-          const float* gm = reinterpret_cast<const float*>(smem + OFF_META + st * META_STAGE + 128 * 4);
+          const float* gm = reinterpret_cast<const float*>(smem + OFF_META + ms * META_STAGE + 128 * 4);
           bias2 = (gm[pp] - gm[128 + pp]) * kLog2e;
         }
       }
+      // The metadata stage is read (and the loaders, done with tile i, read its
+      // positions before): the control warp may refill it.
+      __syncwarp();
+      if (step_ok && lane == 0) mbar_arrive(&bars->meta_empty[ms]);
       const bool valid = step_ok && t >= 0;
       const bool own = valid && (t / kBlock == j);
       const int lim = own ? t - j * kBlock : 63;
@@ -713,6 +745,9 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   prm.NB = NB;
   prm.G = pb.G;
   prm.P = qs.P;
+  int dev = 0, n_sm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  prm.group_major = NB >= 2 * n_sm ? 1 : 0;
   prm.scale_log2 = pb.sm_scale * kLog2e;
   prm.sm_scale = pb.sm_scale;
   prm.wait_ns = wait_limit_ns();

@@ -209,11 +209,44 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int NL = N_LOADER_WARPS * 32;
     const int per_pos = 16 * G;   // 16-byte pieces of a position's G rows
     const char* qbase = reinterpret_cast<const char*>(p.Q) + (long long)(b * p.Hq + g * G) * p.T * (D * 2);
-    int issued = 0;
+    // Tiles are signalled in order as they land. A tile's copies are one cp.async
+    // group per thread, so `issued - signalled` groups are in flight; waiting for
+    // all but the newest n - 1 of them lands the oldest.
+    int issued = 0, signalled = 0;
+    auto signal_oldest = [&]() {
+      const int n = issued - signalled;
+      if (n >= 4)
+        cp_async_wait_group<3>();
+      else if (n == 3)
+        cp_async_wait_group<2>();
+      else if (n == 2)
+        cp_async_wait_group<1>();
+      else
+        cp_async_wait_group<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_full[signalled % NST]);
+      ++signalled;
+    };
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST;
       bool ok = true;
-      if (i >= NST) ok = mbar_wait(&bars->st_free[st], ((i / NST) - 1) & 1, status, wait_ns);
+      if (i >= NST) {
+        // Until stage st is free again, signal the tiles in flight as they land:
+        // the consumer of the stage waits on one of them.
+        const uint32_t par = ((i / NST) - 1) & 1;
+        while (true) {
+          bool free_now = lane == 0 ? mbar_test_wait(&bars->st_free[st], par) : false;
+          free_now = __shfl_sync(0xffffffffu, free_now, 0);
+          if (free_now) break;
+          if (issued > signalled) {
+            signal_oldest();
+            continue;
+          }
+          ok = mbar_wait(&bars->st_free[st], par, status, wait_ns);
+          break;
+        }
+      }
       if (ok) ok = mbar_wait(&bars->pos_ready[st], (i / NST) & 1, status, wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + st * META_STAGE);
@@ -249,20 +282,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       cp_async_commit();
       issued = i + 1;
-      // Tile i-LAG is signalled once it has landed, with tiles i-LAG+1 .. i still
-      // in flight: the gathers of several tiles overlap.
-      if (i >= LAG) {
-        cp_async_wait_group<LAG>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->q_full[(i - LAG) % NST]);
-      }
+      // At most LAG tiles in flight beyond the oldest: the gathers of several tiles overlap.
+      if (issued - signalled > LAG) signal_oldest();
     }
     cp_async_wait_all();   // also after a failed wait: no copy may outlive the CTA
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0)
-      for (int k = max(0, issued - LAG); k < issued; ++k) mbar_arrive(&bars->q_full[k % NST]);
+      for (int k = signalled; k < issued; ++k) mbar_arrive(&bars->q_full[k % NST]);
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
     // A polling state machine: S of the next tile and P V of the oldest tile are
