@@ -139,13 +139,15 @@ def executed_flops(w, sel):
     return fwd, bwd
 
 
-def gate_select_bytes(w, compact: bool = False) -> float:
+def gate_select_bytes(w, compact: bool = False, with_sel: bool = False) -> float:
     """HBM bytes of the fused normalise + select: the causal part of s read once, tau and tau_idx written, and
-    the full logG row written (compact gates: the row's score LSE, 4 bytes, instead)."""
+    the full logG row written (compact gates: the row's score LSE, 4 bytes, instead), plus the K-1 selected
+    block indices of each row when the index list is written."""
     c = np.minimum(np.arange(w.T) // w.block, w.NB).astype(np.float64)
     rows = w.B * w.Hkv
     out = 4.0 * w.T if compact else 4.0 * w.NB * w.T
-    return rows * (4.0 * c.sum() + out + 8.0 * w.T)
+    sel = 4.0 * max(w.K - 1, 0) * w.T if with_sel else 0.0
+    return rows * (4.0 * c.sum() + out + 8.0 * w.T + sel)
 
 
 def gate_grad_bytes(w) -> float:
@@ -367,10 +369,12 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
         host = rank_inputs(w, rank)
     Q, K, V, dO, s = (host[k].to(device) for k in ("Q", "K", "V", "dO", "s"))
     # Compact gates: the fused selection keeps each row's score LSE instead of writing logG; the attention
-    # and gradient calls rebuild log g = s - LSE (bit-identical to logG).
+    # and gradient calls rebuild log g = s - LSE (bit-identical to logG). The selection also writes each
+    # row's sorted block list, from which the attention calls build their per-block row lists.
     gate_lse = torch.empty(w.B, w.Hkv, w.T, device=device)
     tau = torch.empty(w.B, w.Hkv, w.T, device=device)
     tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
+    sel = torch.empty(w.B, w.Hkv, w.T, max(w.K - 1, 1), dtype=torch.int32, device=device)
     O = torch.empty_like(Q)
     LSE = torch.empty(w.B, w.Hq, w.T, device=device)
     dQ, dK, dV, dLogG = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s)
@@ -382,14 +386,15 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        binding.sas_gate_normalize_select_compact(s, gate_lse, tau, tidx, None, w.K, stream=stream)
+        binding.sas_gate_normalize_select_compact(s, gate_lse, tau, tidx, sel, w.K, stream=stream)
         if ev:
             ev[1].record(stream)
-        binding.sas_fwd(Q, K, V, s, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream, gate_lse=gate_lse)
+        binding.sas_fwd(Q, K, V, s, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream, gate_lse=gate_lse,
+                        sel=sel)
         if ev:
             ev[2].record(stream)
         binding.sas_bwd(Q, K, V, O, dO, s, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
-                        stream=stream, gate_lse=gate_lse)
+                        stream=stream, gate_lse=gate_lse, sel=sel)
         if ev:
             ev[3].record(stream)
         binding.sas_gate_grad(s, dLogG, ds, stream=stream, gate_lse=gate_lse)
@@ -427,11 +432,8 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
     dom_name, dom_ms, dom_flops = ("sas_bwd", bwd_avg, bwd_flops) if bwd_avg >= fwd_avg else \
         ("sas_fwd", fwd_avg, fwd_flops)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    sel = torch.empty(w.B, w.Hkv, w.T, w.K - 1, dtype=torch.int32, device=device)
-    binding.sas_gate_normalize_select_compact(s, gate_lse, tau, tidx, sel, w.K, stream=stream)
     torch.cuda.synchronize(device)
     ex_fwd, ex_bwd = executed_flops(w, sel)
-    del sel
     gate_avg = statistics.mean(gate_ms)
     grad_avg = statistics.mean(grad_ms)
     traffic_key = f"{dom_name}:{w.name}"
@@ -448,11 +450,12 @@ def run_training(w, args, device, stream, binding, peaks, rank, world, host=None
                 "bwd_tflops": round(bwd_flops / (bwd_avg * 1e-3) / 1e12, 2),
                 "bwd_executed_tflops": round(ex_bwd / (bwd_avg * 1e-3) / 1e12, 2),
                 "bwd_inflation": round(ex_bwd / bwd_flops, 3),
-                "gate_select": "compact (row score LSE instead of logG)",
+                "gate_select": "compact (row score LSE instead of logG) + sorted block list per row",
                 "gate_select_ms": round(gate_avg, 4),
-                "gate_select_bytes": gate_select_bytes(w, compact=True),
+                "gate_select_bytes": gate_select_bytes(w, compact=True, with_sel=True),
                 "gate_select_bytes_with_logg": gate_select_bytes(w),
-                "gate_select_gbs": round(gate_select_bytes(w, compact=True) / (gate_avg * 1e-3) / 1e9, 1),
+                "gate_select_gbs": round(gate_select_bytes(w, compact=True, with_sel=True) / (gate_avg * 1e-3) / 1e9,
+                                         1),
                 "gate_grad_ms": round(grad_avg, 4),
                 "gate_grad_gbs": round(gate_grad_bytes(w) / (grad_avg * 1e-3) / 1e9, 1)}
     if noisy:
@@ -557,6 +560,7 @@ def run_varlen(args, device, stream, binding, rank):
     logG = torch.empty_like(s)
     tau = torch.empty(w.B, w.Hkv, w.T, device=device)
     tidx = torch.empty(w.B, w.Hkv, w.T, dtype=torch.int32, device=device)
+    sel = torch.empty(w.B, w.Hkv, w.T, max(w.K - 1, 1), dtype=torch.int32, device=device)
     O, LSE = torch.empty_like(Q), torch.empty(w.B, w.Hq, w.T, device=device)
     dQ, dK, dV, dLogG, ds = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(s),
                              torch.empty_like(s))
@@ -565,10 +569,10 @@ def run_varlen(args, device, stream, binding, rank):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     def step():
-        binding.sas_gate_normalize_select_varlen(s, logG, tau, tidx, None, w.K, cu, stream=stream)
-        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream)
+        binding.sas_gate_normalize_select_varlen(s, logG, tau, tidx, sel, w.K, cu, stream=stream)
+        binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws_f, stream=stream, sel=sel)
         binding.sas_bwd(Q, K, V, O, dO, logG, tau, tidx, LSE, dQ, dK, dV, dLogG, w.K, w.sm_scale, ws_b,
-                        stream=stream)
+                        stream=stream, sel=sel)
         binding.sas_gate_grad(logG, dLogG, ds, stream=stream)
 
     for _ in range(max(args.warmup, 3)):
@@ -607,12 +611,14 @@ def run_e2e(args, w, host, device, stream, binding, step_flops, world):
     def e2e_step():
         for k, v in pinned.items():
             dev_in[k].copy_(v, non_blocking=True)
-        logG, tau, tidx, _ = binding.gate_and_select(dev_in["s"], w.K, stream=stream)
-        O, LSE = binding.forward(dev_in["Q"], dev_in["K"], dev_in["V"], logG, tau, tidx, w.K, w.sm_scale,
-                                 stream=stream, check=False)
-        dQ, dK, dV, dLogG = binding.backward(dev_in["Q"], dev_in["K"], dev_in["V"], O, dev_in["dO"], logG, tau,
-                                             tidx, LSE, w.K, w.sm_scale, stream=stream, check=False)
-        ds = binding.gate_grad(logG, dLogG, stream=stream)
+        s = dev_in["s"]
+        lse, tau, tidx, sel = binding.gate_and_select_compact(s, w.K, want_sel=True, stream=stream)
+        O, LSE = binding.forward(dev_in["Q"], dev_in["K"], dev_in["V"], s, tau, tidx, w.K, w.sm_scale,
+                                 stream=stream, check=False, gate_lse=lse, sel=sel)
+        dQ, dK, dV, dLogG = binding.backward(dev_in["Q"], dev_in["K"], dev_in["V"], O, dev_in["dO"], s, tau,
+                                             tidx, LSE, w.K, w.sm_scale, stream=stream, check=False, gate_lse=lse,
+                                             sel=sel)
+        ds = binding.gate_grad(s, dLogG, stream=stream, gate_lse=lse)
         for k, v in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV), ("ds", ds)):
             out_host[k].copy_(v, non_blocking=True)
 

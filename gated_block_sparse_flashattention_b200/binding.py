@@ -41,9 +41,10 @@ _SIGNATURES = {
     "sas_fwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_bwd_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_sz)]),
     "sas_decode_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_sz)]),
-    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_f, _vp, _sz, _vp]),
-    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7
+    "sas_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp] + [_c_int] * 7
                 + [_c_f, _vp, _sz, _vp]),
+    "sas_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+                + [_c_int] * 7 + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _vp, _vp] + [_c_int] * 7
                        + [_c_f, _vp, _sz, _vp]),
     "sas_decode_fwd_paged": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _c_int, _c_int, _vp,
@@ -192,25 +193,27 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block=BLOCK, stream=None, gate_lse=None):
-    """gate_lse: the row log-sum-exp of compact gates (then logG holds the raw scores s)."""
+def sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block=BLOCK, stream=None, gate_lse=None,
+            sel=None):
+    """gate_lse: the row log-sum-exp of compact gates (then logG holds the raw scores s); sel: the
+    selection call's index list [B, Hkv, T, Kbudget-1] (the row lists are then built from it)."""
     B, Hq, T, d = Q.shape
     Hkv = K.shape[1]
     _check("sas_fwd", lib().sas_fwd(
-        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(logG), _ptr(gate_lse), _ptr(tau), _ptr(tau_idx), _ptr(O),
-        _ptr(LSE),
+        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(logG), _ptr(gate_lse), _ptr(tau), _ptr(tau_idx), _ptr(sel),
+        _ptr(O), _ptr(LSE),
         B, Hq, Hkv, T, d, block, int(Kbudget), float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
 
 
 def sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block=BLOCK,
-            stream=None, gate_lse=None):
-    """gate_lse: the row log-sum-exp of compact gates (then logG holds the raw scores s)."""
+            stream=None, gate_lse=None, sel=None):
+    """gate_lse and sel as for ``sas_fwd``."""
     B, Hq, T, d = Q.shape
     Hkv = K.shape[1]
     _check("sas_bwd", lib().sas_bwd(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), _ptr(logG), _ptr(gate_lse), _ptr(tau),
-        _ptr(tau_idx),
+        _ptr(tau_idx), _ptr(sel),
         _ptr(LSE), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dLogG), B, Hq, Hkv, T, d, block, int(Kbudget),
         float(sm_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
@@ -308,31 +311,32 @@ def _check_device_status(fn, ws, stream):
 
 
 def forward(Q, K, V, logG, tau, tau_idx, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None, check=True,
-            gate_lse=None):
+            gate_lse=None, sel=None):
     """O, LSE of ``sas_fwd``. With ``check`` the stream is synchronised and the
     kernel status word is read (raises ``SasError`` on a kernel-side error).
-    With ``gate_lse`` (compact gates) ``logG`` holds the raw scores s."""
+    With ``gate_lse`` (compact gates) ``logG`` holds the raw scores s; ``sel`` is
+    the selection's index list, from which the row lists are built."""
     B, Hq, T, d = Q.shape
     O = torch.empty_like(Q)
     LSE = torch.empty(B, Hq, T, dtype=torch.float32, device=Q.device)
     if ws is None:
         ws = workspace(sas_fwd_workspace_size(B, Hq, K.shape[1], T, d, Kbudget, _dtype_code(Q), block), Q.device)
-    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block, stream, gate_lse=gate_lse)
+    sas_fwd(Q, K, V, logG, tau, tau_idx, O, LSE, Kbudget, sm_scale, ws, block, stream, gate_lse=gate_lse, sel=sel)
     if check:
         _check_device_status("sas_fwd", ws, stream)
     return O, LSE
 
 
 def backward(Q, K, V, O, dO, logG, tau, tau_idx, LSE, Kbudget, sm_scale, block=BLOCK, stream=None, ws=None,
-             check=True, gate_lse=None):
-    """dQ, dK, dV, dLogG of ``sas_bwd`` (``check`` and ``gate_lse`` as in ``forward``)."""
+             check=True, gate_lse=None, sel=None):
+    """dQ, dK, dV, dLogG of ``sas_bwd`` (``check``, ``gate_lse`` and ``sel`` as in ``forward``)."""
     B, Hq, T, d = Q.shape
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     dLogG = torch.empty_like(logG)
     if ws is None:
         ws = workspace(sas_bwd_workspace_size(B, Hq, K.shape[1], T, d, Kbudget, _dtype_code(Q), block), Q.device)
     sas_bwd(Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG, Kbudget, sm_scale, ws, block, stream,
-            gate_lse=gate_lse)
+            gate_lse=gate_lse, sel=sel)
     if check:
         _check_device_status("sas_bwd", ws, stream)
     return dQ, dK, dV, dLogG

@@ -207,12 +207,12 @@ int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int block
 }
 
 int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* gate_lse,
-            const float* tau, const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d,
-            int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+            const float* tau, const int32_t* tau_idx, const int32_t* sel, void* O, float* LSE, int B, int Hq, int Hkv,
+            int T, int d, int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
   const void* ptrs[] = {Q, K, V, logG, tau, tau_idx, O, LSE};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
-  if (gate_lse && !aligned16(gate_lse)) return SAS_ERR_INVALID_ARG;
+  if ((gate_lse && !aligned16(gate_lse)) || (sel && !aligned16(sel))) return SAS_ERR_INVALID_ARG;
   int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
   if (!(sm_scale > 0.f) || Kbudget < 1) return SAS_ERR_INVALID_ARG;
@@ -235,6 +235,7 @@ int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float*
   pb.gate_lse = gate_lse;
   pb.tau = tau;
   pb.tau_idx = tau_idx;
+  pb.sel = sel;
   cudaStream_t s = as_stream(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
   if (dtype == SAS_DT_F32) return cuda_status(launch_fwd_simt(pb, static_cast<float*>(O), LSE, s));
@@ -245,13 +246,13 @@ int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float*
 }
 
 int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
-            const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx, const float* LSE,
-            void* dQ, void* dK, void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget,
-            float sm_scale, void* ws, size_t ws_bytes, void* stream) {
+            const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx, const int32_t* sel,
+            const float* LSE, void* dQ, void* dK, void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d,
+            int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream) {
   const void* ptrs[] = {Q, K, V, O, dO, logG, tau, tau_idx, LSE, dQ, dK, dV, dLogG};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAS_ERR_INVALID_ARG;
-  if (gate_lse && !aligned16(gate_lse)) return SAS_ERR_INVALID_ARG;
+  if ((gate_lse && !aligned16(gate_lse)) || (sel && !aligned16(sel))) return SAS_ERR_INVALID_ARG;
   int st = check_attention_shape(B, Hq, Hkv, T, d, block, dtype);
   if (st != SAS_OK) return st;
   if (!(sm_scale > 0.f)) return SAS_ERR_INVALID_ARG;
@@ -277,6 +278,7 @@ int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const vo
   pb.gate_lse = gate_lse;
   pb.tau = tau;
   pb.tau_idx = tau_idx;
+  pb.sel = sel;
   pb.LSE = LSE;
   cudaStream_t s = as_stream(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);

@@ -704,8 +704,8 @@ cudaError_t launch_bwd_gather(const TcProblem& pb, int K, void* dQ, void* dK, vo
   if ((e = cudaMemsetAsync(dLogG, 0, (size_t)rows * NB * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dQacc, 0, (size_t)qrows * D * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(eps, 0, (size_t)qrows * sizeof(float), st)) != cudaSuccess) return e;
-  if ((e = launch_block_lists(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, false, status, st)) !=
-      cudaSuccess)
+  if ((e = launch_block_lists(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, pb.sel, L, nbg, pb.T, NB, K, false, status,
+                              st)) != cudaSuccess)
     return e;
   pack_kernel<<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(pb.Q), reinterpret_cast<const __nv_bfloat16*>(pb.dO),

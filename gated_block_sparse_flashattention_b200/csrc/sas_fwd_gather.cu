@@ -616,7 +616,7 @@ cudaError_t launch_fwd_gather(const TcProblem& pb, int K, void* O, float* LSE, i
   float* lslot = reinterpret_cast<float*>(scratch + o);
 
   cudaError_t e =
-      launch_block_lists(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, L, nbg, pb.T, NB, K, true, status, st);
+      launch_block_lists(pb.logG, pb.gate_lse, pb.tau, pb.tau_idx, pb.sel, L, nbg, pb.T, NB, K, true, status, st);
   if (e != cudaSuccess) return e;
   const QTileShape qs = qtile_shape(pb.G, pb.T, NB);
   CUtensorMap tk, tv;

@@ -61,6 +61,7 @@ struct TcProblem {
   const float* gate_lse;  // null, or [B*Hkv*T] LSE of each row's historical scores: log g = s - gate_lse
   const float* tau;
   const int32_t* tau_idx;
+  const int32_t* sel;  // null, or [B*Hkv*T][K-1] the selection's ascending block lists (-1 padded)
   const float* LSE;  // bwd only
 };
 
@@ -83,7 +84,7 @@ struct BlockLists {
 size_t block_lists_bytes(long long nbg, int T, int NB, int K);
 BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int K);
 cudaError_t launch_block_lists(const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
-                               const BlockLists& L,
+                               const int32_t* sel, const BlockLists& L,
                                long long nbg, int T, int NB, int K, bool want_nsel, int32_t* status,
                                cudaStream_t st);
 

@@ -13,6 +13,10 @@
 // selected blocks; a threshold that keeps more has its extra pairs dropped and
 // is reported as a device-side bounds error.
 //
+// The pairs come from thresholding the gates, or, when the caller passes the
+// selection's sorted index list (sel), from that list, which is 4*(K-1) bytes
+// per row instead of the row's gates.
+//
 // Three kernels: per-block counts (also kept per chunk of 256 positions), their
 // offsets and each chunk's first entry in every list (scans per (b, g)), and the
 // lists, placed in one more pass over the rows. A list entry packs the position
@@ -83,13 +87,53 @@ __device__ __forceinline__ void for_each_pair(const float* __restrict__ logG, co
   }
 }
 
+// The same pairs from the selection's index list: sel[b, g, t, k] (k < H) holds
+// row t's selected blocks in ascending order, -1 after the last one, so the
+// rank of an entry is its index. This reads 4*H bytes per row instead of the
+// row's c_t gates. An entry that is not a historical block of its row (m >= c_t)
+// is skipped and reported as a bounds error. One warp per group of 4 rows, the
+// rows' loads issued together.
+template <typename F, typename Done>
+__device__ __forceinline__ void for_each_pair_sel(const int32_t* __restrict__ sel, int H, long long bg, int t0, int T,
+                                                  int NB, int32_t* status, F&& f, Done&& done) {
+  constexpr int R = 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+  const int t_end = min(T, t0 + kChunkRows);
+  for (int tb = t0 + warp * R; tb < t_end; tb += n_warps * R) {
+    int n[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) n[r] = 0;
+    for (int k0 = 0; k0 < H; k0 += 32) {
+      const int k = k0 + lane;
+      int m[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        m[r] = (k < H && tb + r < t_end) ? sel[(bg * T + tb + r) * (long long)H + k] : -1;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int c = min((tb + r) / kBlock, NB);
+        const bool bad = m[r] >= c;
+        if (bad) set_status(status, SAS_DEV_ERR_BOUNDS);
+        const bool take = m[r] >= 0 && !bad;
+        if (take) f(tb + r, m[r], k);
+        n[r] += __popc(__ballot_sync(0xffffffffu, take));
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (lane == r && tb + r < t_end) done(tb + r, n[r]);
+  }
+}
+
 // Count, per (b, g, block), the positions whose selection contains the block
 // (pairs beyond the row's K-1 slots excluded), and keep each chunk's counts
-// ccnt[b, g, chunk, block] for the fill. Grid: (chunks of T, B * Hkv); dynamic
-// shared memory: NB ints.
+// ccnt[b, g, chunk, block] for the fill. The pairs come from the selection's
+// index list when sel is set, else from thresholding the gates. Grid: (chunks of
+// T, B * Hkv); dynamic shared memory: NB ints.
 __global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ logG, const float* __restrict__ lse,
                                                     const float* __restrict__ tau,
-                                                    const int32_t* __restrict__ tau_idx, int32_t* __restrict__ cnt,
+                                                    const int32_t* __restrict__ tau_idx,
+                                                    const int32_t* __restrict__ sel, int32_t* __restrict__ cnt,
                                                     int32_t* __restrict__ ccnt, int32_t* status, int T, int NB,
                                                     int H) {
   extern __shared__ int32_t hist[];
@@ -98,12 +142,14 @@ __global__ void __launch_bounds__(256) count_kernel(const float* __restrict__ lo
   for (int m = threadIdx.x; m < NB; m += blockDim.x) hist[m] = 0;
   __syncthreads();
   bool over = false;
-  for_each_pair(
-      logG, lse, tau, tau_idx, bg, t0, T, NB,
-      [&](int, int m, int rank) {
-        if (rank < H) atomicAdd(hist + m, 1);
-      },
-      [&](int, int n) { over |= n > H; });
+  auto add = [&](int, int m, int rank) {
+    if (rank < H) atomicAdd(hist + m, 1);
+  };
+  auto row_done = [&](int, int n) { over |= n > H; };
+  if (sel)
+    for_each_pair_sel(sel, H, bg, t0, T, NB, status, add, row_done);
+  else
+    for_each_pair(logG, lse, tau, tau_idx, bg, t0, T, NB, add, row_done);
   if (over) set_status(status, SAS_DEV_ERR_BOUNDS);
   __syncthreads();
   int32_t* cc = ccnt + (bg * gridDim.x + blockIdx.x) * NB;
@@ -183,6 +229,7 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
 __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ logG, const float* __restrict__ lse,
                                                    const float* __restrict__ tau,
                                                    const int32_t* __restrict__ tau_idx,
+                                                   const int32_t* __restrict__ sel, int32_t* status,
                                                    const int32_t* __restrict__ off, const int32_t* __restrict__ cap,
                                                    const int32_t* __restrict__ cbase, int32_t* __restrict__ list,
                                                    int32_t* __restrict__ nsel, int T, int NB, int H) {
@@ -197,16 +244,18 @@ __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ log
     lbase[m] = cb[m];
   }
   __syncthreads();
-  for_each_pair(
-      logG, lse, tau, tau_idx, bg, t0, T, NB,
-      [&](int t, int m, int rank) {
-        if (rank >= H) return;
-        const int at = lbase[m] + atomicAdd(lcnt + m, 1);
-        if (at < cap[bg * NB + m]) list[off[bg * NB + m] + at] = t | ((rank + 1) << kEntrySlotShift);
-      },
-      [&](int t, int n) {
-        if (nsel) nsel[bg * T + t] = min(n, H);
-      });
+  auto place = [&](int t, int m, int rank) {
+    if (rank >= H) return;
+    const int at = lbase[m] + atomicAdd(lcnt + m, 1);
+    if (at < cap[bg * NB + m]) list[off[bg * NB + m] + at] = t | ((rank + 1) << kEntrySlotShift);
+  };
+  auto row_done = [&](int t, int n) {
+    if (nsel) nsel[bg * T + t] = min(n, H);
+  };
+  if (sel)
+    for_each_pair_sel(sel, H, bg, t0, T, NB, status, place, row_done);
+  else
+    for_each_pair(logG, lse, tau, tau_idx, bg, t0, T, NB, place, row_done);
 }
 
 }  // namespace lists
@@ -245,7 +294,7 @@ BlockLists carve_block_lists(uint8_t* scratch, long long nbg, int T, int NB, int
 }
 
 cudaError_t launch_block_lists(const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
-                               const BlockLists& L,
+                               const int32_t* sel, const BlockLists& L,
                                long long nbg, int T, int NB, int K, bool want_nsel, int32_t* status,
                                cudaStream_t st) {
   using namespace lists;
@@ -254,13 +303,14 @@ cudaError_t launch_block_lists(const float* logG, const float* gate_lse, const f
   cudaError_t e = cudaMemsetAsync(L.cnt, 0, (size_t)nbg * NB * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const dim3 chunks((unsigned)n_chunks, (unsigned)nbg);
-  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(logG, gate_lse, tau, tau_idx, L.cnt, L.ccnt, status, T,
-                                                           NB, H);
+  count_kernel<<<chunks, 256, NB * sizeof(int32_t), st>>>(logG, gate_lse, tau, tau_idx, H > 0 ? sel : nullptr,
+                                                           L.cnt, L.ccnt, status, T, NB, H);
   count_launch();
   offsets_kernel<<<(unsigned)nbg, 1024, 0, st>>>(L.cnt, L.off, L.ccnt, L.cap, L.total, status, NB, n_chunks,
                                                    L.region);
   count_launch();
-  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(logG, gate_lse, tau, tau_idx, L.off, L.cap, L.ccnt, L.list,
+  fill_kernel<<<chunks, 256, 2 * NB * sizeof(int32_t), st>>>(logG, gate_lse, tau, tau_idx, H > 0 ? sel : nullptr,
+                                                              status, L.off, L.cap, L.ccnt, L.list,
                                                               want_nsel ? L.nsel : nullptr, T, NB, H);
   count_launch();
   return cudaGetLastError();

@@ -247,6 +247,12 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * [B,Hkv,T] log-sum-exp of each row's historical scores, with the raw scores s
  * passed as `logG`: the gate is then s[m] - gate_lse[b,g,t] in fp32, bit for bit
  * the normalised gate.
+ * sel: null, or the index list the selection call wrote with the same tau and
+ * tau_idx ([B,Hkv,T,Kbudget-1] int32, each row's selected blocks ascending, -1
+ * padded). The bf16 kernels then build their per-block row lists from it (4 bytes
+ * per selected block) instead of thresholding each row's gates again; the
+ * attended set and the results are the same. An entry that is not an earlier
+ * block of its row is skipped and reported as a device-side bounds error.
  * O [B,Hq,T,d] of `dtype`; LSE [B,Hq,T] fp32. T % 64 == 0, NB == T / 64,
  * Hq % Hkv == 0, d in {64, 128} (fp32) or d == 128 (bf16).
  * Kbudget: the budget K given to the selection (the threshold keeps at most K-1
@@ -260,8 +266,9 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * ws: workspace of sas_fwd_workspace_size bytes (same K).
  */
 SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* gate_lse,
-            const float* tau, const int32_t* tau_idx, void* O, float* LSE, int B, int Hq, int Hkv, int T, int d,
-            int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes, void* stream);
+                    const float* tau, const int32_t* tau_idx, const int32_t* sel, void* O, float* LSE, int B, int Hq,
+                    int Hkv, int T, int d, int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes,
+                    void* stream);
 
 /*
  * sas_bwd - gradients of a scalar loss through sas_fwd (SAS paper Appendix E
@@ -269,8 +276,8 @@ SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, cons
  *   P = exp(z - LSE), Delta = rowsum(O * dO), dS = P * (dO V^T - Delta),
  *   dQ = sm_scale dS K,  dK = sm_scale sum_{h in g} dS^T Q,  dV = sum_{h in g} P^T dO,
  *   dLogG[b,g,t,m] = sum_{h in g} sum_{i in block m} dS[h,t,i] for selected m, 0 otherwise.
- * Inputs as for sas_fwd (gate_lse included) plus O (the forward output), dO and
- * LSE (the forward's).
+ * Inputs as for sas_fwd (gate_lse and sel included) plus O (the forward output),
+ * dO and LSE (the forward's).
  * Outputs dQ [B,Hq,T,d], dK/dV [B,Hkv,T,d] of `dtype`; dLogG [B,Hkv,T,NB] fp32
  * (fully written: zero outside the selection). Kbudget: the budget K given to
  * sas_select_threshold (the threshold keeps at most K-1 historical blocks per row;
@@ -279,9 +286,10 @@ SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, cons
  * (for bf16 it holds an fp32 dQ accumulator and the per-block row lists).
  */
 SAS_API int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
-            const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx, const float* LSE,
-            void* dQ, void* dK, void* dV, float* dLogG, int B, int Hq, int Hkv, int T, int d, int block, int Kbudget,
-            float sm_scale, void* ws, size_t ws_bytes, void* stream);
+                    const float* logG, const float* gate_lse, const float* tau, const int32_t* tau_idx,
+                    const int32_t* sel, const float* LSE, void* dQ, void* dK, void* dV, float* dLogG, int B, int Hq,
+                    int Hkv, int T, int d, int block, int Kbudget, float sm_scale, void* ws, size_t ws_bytes,
+                    void* stream);
 
 /*
  * sas_decode_fwd - one sparse decode step per sequence (SAS paper §4.3

@@ -125,17 +125,20 @@ def test_invalid_calls_return_errors_without_launching(lib):
     paged[16] = 3                 # NBmax < max_pages
     assert lib.sas_decode_fwd_paged(*paged) == -1
     # sas_fwd: missing workspace / bad sizes
-    args = ([fake] * 3 + [binding.SAS_DT_BF16] + [fake, None] + [fake] * 4
+    args = ([fake] * 3 + [binding.SAS_DT_BF16] + [fake, None] + [fake, fake, None, fake, fake]
             + [1, 4, 1, 128, 128, 64, 2, ctypes.c_float(0.1), None, 0, None])
     assert lib.sas_fwd(*args) == -5
     args[-3] = fake
     args[-2] = 1 << 30
-    args[13] = 100   # T not a multiple of 64
+    args[14] = 100   # T not a multiple of 64
     assert lib.sas_fwd(*args) == -1
-    args[13] = 128
-    args[16] = 0     # budget K < 1
+    args[14] = 128
+    args[17] = 0     # budget K < 1
     assert lib.sas_fwd(*args) == -1
-    args[16] = 2
+    args[17] = 2
     args[5] = fake + 4   # misaligned row LSE of compact gates
+    assert lib.sas_fwd(*args) == -1
+    args[5] = None
+    args[8] = fake + 4   # misaligned selection index list
     assert lib.sas_fwd(*args) == -1
     assert lib.sas_launch_count() == before

@@ -102,6 +102,8 @@ def test_gate_kernel_byte_counts_brute_force():
     thr = w.T * 8 * w.B * w.Hkv                                                   # tau + tau_idx
     assert bench.gate_select_bytes(w) == rd_c + full + thr
     assert bench.gate_select_bytes(w, compact=True) == rd_c + w.T * 4 * w.B * w.Hkv + thr   # row LSE instead of logG
+    sel = w.T * (w.K - 1) * 4 * w.B * w.Hkv                                       # the sorted block list
+    assert bench.gate_select_bytes(w, compact=True, with_sel=True) == rd_c + w.T * 4 * w.B * w.Hkv + thr + sel
     assert bench.gate_grad_bytes(w) == 2 * rd_c + full
     assert bench.noisy_select_bytes(w) == 2 * rd_c + full + thr
 
