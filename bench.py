@@ -95,11 +95,15 @@ def attended_flops(w) -> tuple[float, float]:
 SLOT_BUDGET = 8 << 30   # bytes of forward partials per batch of (b, g) groups
 
 
+MERGE_LSE_CAP = 1024    # slots x heads of one row that the partials' merge takes
+
+
 def fwd_uses_gather(w) -> bool:
     """Whether sas_fwd runs the KV-block-outer forward (per-pair partials of one (b, g) within the slot budget:
-    T * min(K, NB+1) slots of G x (128 bf16 + one fp32)) or the q-tile union forward."""
+    T * min(K, NB+1) slots of G x (128 bf16 + one fp32), and at most MERGE_LSE_CAP slots x heads per row) or
+    the q-tile union forward."""
     slots = 1 + max(0, min(w.K - 1, w.NB))
-    return w.T * slots * w.G * (128 * 2 + 4) <= SLOT_BUDGET
+    return w.T * slots * w.G * (128 * 2 + 4) <= SLOT_BUDGET and slots * w.G <= MERGE_LSE_CAP
 
 
 def executed_flops(w, sel):

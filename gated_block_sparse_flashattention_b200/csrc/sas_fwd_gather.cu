@@ -478,13 +478,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 // 16-byte chunks l, l + 32, ... (KC of them, KC = ceil(G / 2)) and folds them
 // over the slots with the weights exp2(lse_s - LSE) of their head. n = 1 +
 // nsel[t] slots: slot 0 (own block) and the selected blocks.
+// The kernel streams the partials once from HBM, so what matters is the number
+// of loads in flight: the row's n * G log-sum-exps come in one coalesced pass
+// into shared memory, where the per-head LSE is taken and each entry turned
+// into its weight, while the first batch of slot loads is in flight.
+constexpr int kMergeLseCap = 1024;   // Ks * G of the rows the merge takes
 template <int KC>
-__global__ void __launch_bounds__(256) merge_kernel(const __nv_bfloat16* __restrict__ oslot,
+__global__ void __launch_bounds__(256, 2) merge_kernel(const __nv_bfloat16* __restrict__ oslot,
                                                     const float* __restrict__ lslot,
                                                     const int32_t* __restrict__ nsel, __nv_bfloat16* __restrict__ O,
                                                     float* __restrict__ LSE, int bg0, long long n_rows, int T, int Ks,
                                                     int G, int Hq, int Hkv) {
   __shared__ float lse_sh[8][16];
+  __shared__ float ls_sh[8][kMergeLseCap];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long w = (long long)blockIdx.x * 8 + wid;
   if (w >= n_rows) return;
@@ -495,14 +501,29 @@ __global__ void __launch_bounds__(256) merge_kernel(const __nv_bfloat16* __restr
   const int n = 1 + min(nsel[bg * T + t], Ks - 1);
   const long long row0 = (bgl * T + t) * Ks;   // first slot of the row
   const float* ls = lslot + row0 * G;          // [slot][head]
+  const int n_chunks = 16 * G;
+  const uint4* os = reinterpret_cast<const uint4*>(oslot + row0 * G * 128);   // slot s: G * 16 chunks
+  constexpr int U = KC <= 4 ? 4 : 2;   // slots per batch of loads
+  uint4 v[U][KC];
+  // First batch of slot loads, in flight during the log-sum-exp reduction.
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      v[u][k] = (u < n && c < n_chunks) ? os[(long long)u * n_chunks + c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  float* lsw = ls_sh[wid];
+  for (int e = lane; e < n * G; e += 32) lsw[e] = ls[e];
+  __syncwarp();
   for (int hh = 0; hh < G; ++hh) {
     float M = -INFINITY;
-    for (int s = lane; s < n; s += 32) M = fmaxf(M, ls[(long long)s * G + hh]);
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, lsw[s * G + hh]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
     if (M != -INFINITY)
-      for (int s = lane; s < n; s += 32) L += ex2(ls[(long long)s * G + hh] - M);
+      for (int s = lane; s < n; s += 32) L += ex2(lsw[s * G + hh] - M);
 #pragma unroll
     for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     // No finite partial cannot happen for valid inputs (the own block holds key t).
@@ -513,33 +534,34 @@ __global__ void __launch_bounds__(256) merge_kernel(const __nv_bfloat16* __restr
     }
   }
   __syncwarp();
-  const int n_chunks = 16 * G;
+  // Each slot's weight per head, exp2(lse_s - LSE), in place (0 for an empty partial).
+  for (int e = lane; e < n * G; e += 32) {
+    const float x = lsw[e];
+    lsw[e] = x == -INFINITY ? 0.f : ex2(x - lse_sh[wid][e % G]);
+  }
+  __syncwarp();
   float acc[KC][8];
 #pragma unroll
   for (int k = 0; k < KC; ++k)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
-  const uint4* os = reinterpret_cast<const uint4*>(oslot + row0 * G * 128);   // slot s: G * 16 chunks
-  constexpr int U = KC <= 2 ? 4 : 2;   // slots per batch of loads
   for (int s0 = 0; s0 < n; s0 += U) {
-    uint4 v[U][KC];
-    float wt[U][KC];
+    if (s0 > 0) {
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+          const int c = lane + 32 * k;
+          v[u][k] = (s0 + u < n && c < n_chunks) ? os[(long long)(s0 + u) * n_chunks + c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int k = 0; k < KC; ++k) {
         const int c = lane + 32 * k;
-        const bool on = s0 + u < n && c < n_chunks;
-        v[u][k] = on ? os[(long long)(s0 + u) * n_chunks + c] : make_uint4(0u, 0u, 0u, 0u);
-        wt[u][k] = on ? ls[(long long)(s0 + u) * G + (c >> 4)] : -INFINITY;
-      }
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int k = 0; k < KC; ++k) {
-        const int c = lane + 32 * k;
-        if (c >= n_chunks || wt[u][k] == -INFINITY) continue;
-        const float wu = ex2(wt[u][k] - lse_sh[wid][c >> 4]);
+        if (s0 + u >= n || c >= n_chunks) continue;
+        const float wu = lsw[(s0 + u) * G + (c >> 4)];
         const uint32_t x[4] = {v[u][k].x, v[u][k].y, v[u][k].z, v[u][k].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -587,7 +609,8 @@ int groups_per_batch(int B, int Hq, int Hkv, int T, int K) {
 
 bool fwd_gather_applies(int B, int Hq, int Hkv, int T, int K) {
   (void)B;
-  return gfwd::slot_bytes_per_group(Hq, Hkv, T, K) <= gfwd::kSlotBudget;
+  return gfwd::slot_bytes_per_group(Hq, Hkv, T, K) <= gfwd::kSlotBudget &&
+         gfwd::slots_per_row(K, T / kBlock) * (Hq / Hkv) <= gfwd::kMergeLseCap;
 }
 
 size_t fwd_gather_workspace_bytes(int B, int Hq, int Hkv, int T, int K) {

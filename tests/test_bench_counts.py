@@ -86,7 +86,7 @@ def test_forward_path_rule_matches_the_library_workspace():
         import pytest
         pytest.skip("library not built")
     for (B, Hq, Hkv, T, K) in [(1, 32, 8, 8192, 16), (2, 32, 8, 32768, 32), (1, 40, 8, 65536, 16),
-                               (1, 4, 1, 262144, 64), (1, 8, 1, 131072, 300)]:
+                               (1, 4, 1, 262144, 64), (1, 8, 1, 131072, 300), (1, 32, 2, 8192, 100)]:
         w = workloads.custom("rule", "bf16", B=B, Hq=Hq, Hkv=Hkv, d=128, T=T, K=K)
         ws = binding.sas_fwd_workspace_size(B, Hq, Hkv, T, 128, K, binding.SAS_DT_BF16)
         P = (128 // w.G) & ~7
