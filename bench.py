@@ -39,13 +39,19 @@ import torch  # noqa: E402
 
 from gated_block_sparse_flashattention_b200 import workloads  # noqa: E402
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture, cold caches),
-# reported as the roofline "traffic" only while the kernel sources still match the ones measured
-# (sha256 prefixes); after any change they read as unmeasured (null).
+# DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum of the call's kernels, from one ncu
+# capture, cold caches), reported as the roofline "traffic" only while the kernel sources still match the
+# ones measured (sha256 prefixes); after any change they read as unmeasured (null). Keys: call:workload. The
+# paged decode was captured on its 64K-token pool only (the 512K pool is too large to capture), so the 512K
+# leg reports no traffic.
+_BWD_SRC = {"sas_bwd_gather.cu": "349b886374f66745", "sas_lists.cu": "c8917b447428d9c8",
+            "sas_common.cuh": "c8fb05e97eabbdee"}
+_DEC_SRC = {"sas_decode.cu": "c6c2dab8a9031aee", "sas_common.cuh": "c8fb05e97eabbdee"}
 MEASURED_TRAFFIC = {
-    "sas_bwd": (2441994240, {"sas_bwd_gather.cu": "33071cc059fe81d6", "sas_common.cuh": "d3c29d493fc4dfcf"}),
-    "decode": (67355136, {"sas_decode.cu": "fe0147b988941a3e", "sas_common.cuh": "d3c29d493fc4dfcf"}),
-    "decode_paged": (68085760, {"sas_decode.cu": "fe0147b988941a3e", "sas_common.cuh": "d3c29d493fc4dfcf"}),
+    "sas_bwd:qwen3_8b_t32k": (19847566250, _BWD_SRC),
+    "sas_bwd:qwen3_4b_t8k": (2495377397, _BWD_SRC),
+    "decode:decode_b16_l32k": (71996160, _DEC_SRC),
+    "decode_paged:decode_b8_l64k_paged": (71999360, _DEC_SRC),
 }
 
 
@@ -705,7 +711,7 @@ def run_decode(args, device, stream, binding, peaks, clk=None):
     return {"workload": "decode_b16_l32k: 16 seqs x 1 token, cache 32768, Hq=32 Hkv=8 d=128 K=16",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": decode_bytes(w), "peak": peaks["hbm_gbs"],
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": measured_traffic("decode"),
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": measured_traffic("decode:" + DECODE_WORKLOAD),
             "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
             "launches_per_step": per_call, "device_status": binding.sas_device_status(ws),
             "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
@@ -736,7 +742,8 @@ def run_decode_paged(args, device, stream, binding, peaks, clk=None, name=PAGED_
                         f"each, {pool_gb:.1f} GB K/V pool), Hq={w.Hq} Hkv={w.Hkv} d={w.d} K={w.K}",
             "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(med * 1e3, 2),
             "bytes_per_step": nbytes, "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
-            "traffic": measured_traffic("decode_paged"), "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
+            "traffic": measured_traffic("decode_paged:" + name) if "decode_paged:" + name in MEASURED_TRAFFIC
+            else None, "graph": f"{n_rot} steps per graph", "steps": reps * n_rot,
             "launches_per_step": per_call, "device_status": binding.sas_device_status(ws),
             "l2": "not flushed; each step attends a different random block set (16 seeded score tensors)"}
 
