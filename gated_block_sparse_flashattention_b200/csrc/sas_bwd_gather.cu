@@ -309,6 +309,30 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------------ loaders: Q / dO row gathers
     const int lt = tid - LOADER_WARP0 * 32;
     constexpr int NL = N_LOADER_WARPS * 32;
+    // Pieces of 16 bytes of the Q/dO rows of each position's chunk: 32*G of them
+    // (ordered tensor, head, piece), piece lt + k * NL of the tile for this
+    // thread, so consecutive lanes copy consecutive bytes. The map from a piece to
+    // its tile position, shared-memory offset and offset in the chunk is the same
+    // for every tile: it is taken once, and a tile then only reads its positions.
+    constexpr int MAXP = (128 * 32 + NL - 1) / NL;   // G * P <= 128 rows of 16 pieces, Q and dO
+    const int rows_pieces = 32 * G;
+    const int n_pieces = PP * rows_pieces;
+    int pk_pp[MAXP];
+    uint32_t pk_dst[MAXP], pk_src[MAXP];
+#pragma unroll
+    for (int k = 0; k < MAXP; ++k) {
+      const int piece = lt + k * NL;
+      const int pp = piece < n_pieces ? piece / rows_pieces : 0;
+      const int rem = piece < n_pieces ? piece - pp * rows_pieces : 0;
+      const int tensor = rem >= 16 * G;
+      const int rem2 = rem - tensor * 16 * G;
+      const int hh = rem2 >> 4, c16 = rem2 & 15;
+      pk_pp[k] = piece < n_pieces ? pp : -1;
+      pk_dst[k] = (uint32_t)tensor * TILE + (uint32_t)(c16 >> 3) * HALF128 +
+                  sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)(c16 & 7));
+      pk_src[k] = (uint32_t)rem * 16;
+    }
+    const uint8_t* base = p.packed + (long long)bg * p.T * p.chunk;
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % NST, ms = i % MST;
       bool ok = true;
@@ -319,29 +343,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int* pos = reinterpret_cast<const int*>(smem + OFF_META + ms * META_STAGE);
       const int first = pos[0];
       const uint32_t qd = s_base + OFF_QD + st * 2 * TILE;
-      // Pieces of 16 bytes of the Q/dO rows of each position's chunk: 32*G of them
-      // (ordered tensor, head, piece). The loaders walk (position, piece) with a
-      // stride of NL pieces, so consecutive lanes copy consecutive bytes.
-      const int rows_pieces = 32 * G;
-      const uint8_t* base = p.packed + (long long)bg * p.T * p.chunk;
-      int pp = 0, piece = lt;
-      while (piece >= rows_pieces) {
-        piece -= rows_pieces;
-        ++pp;
-      }
-      while (pp < PP) {
-        const int t0 = pos[pp];
-        const uint8_t* src = base + (long long)(t0 >= 0 ? t0 : first) * p.chunk + piece * 16;
-        const int tensor = piece >= 16 * G;
-        const int rem2 = piece - tensor * 16 * G;
-        const int hh = rem2 >> 4, c16 = rem2 & 15;
-        const int half = c16 >> 3, ch = c16 & 7;
-        cp_async16(qd + tensor * TILE + half * HALF128 + sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)ch), src);
-        piece += NL;
-        while (piece >= rows_pieces) {
-          piece -= rows_pieces;
-          ++pp;
-        }
+#pragma unroll
+      for (int k = 0; k < MAXP; ++k) {
+        if (pk_pp[k] < 0) continue;
+        const int t0 = pos[pk_pp[k]];
+        cp_async16(qd + pk_dst[k], base + (long long)(t0 >= 0 ? t0 : first) * p.chunk + pk_src[k]);
       }
       cp_async_commit_wait_all();
       fence_proxy_async_smem();

@@ -209,6 +209,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int NL = N_LOADER_WARPS * 32;
     const int per_pos = 16 * G;   // 16-byte pieces of a position's G rows
     const char* qbase = reinterpret_cast<const char*>(p.Q) + (long long)(b * p.Hq + g * G) * p.T * (D * 2);
+    // Pieces ordered (position, head, 16-byte chunk), piece lt + k * NL for this
+    // thread, so consecutive lanes copy consecutive bytes of one 256-byte row. The
+    // map from a piece to its tile position, shared-memory offset and source
+    // offset (head row, chunk) is the same for every tile: it is taken once, and
+    // a tile then only reads its positions.
+    constexpr int MAXP = (128 * 16 + NL - 1) / NL;   // G * P <= 128 rows of 16 pieces
+    const int n_pieces = PP * per_pos;
+    int pk_pp[MAXP];
+    uint32_t pk_dst[MAXP], pk_src[MAXP];
+#pragma unroll
+    for (int k = 0; k < MAXP; ++k) {
+      const int piece = lt + k * NL;
+      const int pp = piece < n_pieces ? piece / per_pos : 0;
+      const int rem = piece < n_pieces ? piece - pp * per_pos : 0;
+      const int hh = rem >> 4, c16 = rem & 15;
+      pk_pp[k] = piece < n_pieces ? pp : -1;
+      pk_dst[k] = (uint32_t)(c16 >> 3) * HALF128 + sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)(c16 & 7));
+      pk_src[k] = (uint32_t)hh * (uint32_t)p.T * (D * 2) + (uint32_t)c16 * 16;   // < 2^31: G <= 16, T < 2^18
+    }
     // Tiles are signalled in order as they land. A tile's copies are one cp.async
     // group per thread, so `issued - signalled` groups are in flight; waiting for
     // all but the newest n - 1 of them lands the oldest.
@@ -269,16 +288,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           glse[pp] = 0.f;
         }
       }
-      // Pieces ordered (position, head, 16-byte chunk): consecutive lanes copy
-      // consecutive bytes of one 256-byte row.
-      for (int piece = lt; piece < PP * per_pos; piece += NL) {
-        const int pp = piece / per_pos, rem = piece - pp * per_pos;
-        const int t = pos[pp];
+#pragma unroll
+      for (int k = 0; k < MAXP; ++k) {
+        if (pk_pp[k] < 0) continue;
+        const int t = pos[pk_pp[k]];
         if (t < 0) continue;
-        const int hh = rem >> 4, c16 = rem & 15;
-        const int half = c16 >> 3, ch = c16 & 7;
-        cp_async16(qd + half * HALF128 + sw128_offset((uint32_t)(hh * PP + pp), (uint32_t)ch),
-                   qbase + ((long long)hh * p.T + t) * (D * 2) + c16 * 16);
+        cp_async16(qd + pk_dst[k], qbase + pk_src[k] + (long long)t * (D * 2));
       }
       cp_async_commit();
       issued = i + 1;
