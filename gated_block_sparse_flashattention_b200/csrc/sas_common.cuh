@@ -538,13 +538,12 @@ __device__ __forceinline__ void warp_sort64_desc(T (&v)[2]) {
 // largest keys give 64 values whose H-th largest is a lower bound of the
 // threshold (H distinct keys reach it); with about H + a few keys at or above it,
 // the candidates are sorted across the warp two per lane by (key descending,
-// index ascending). *asc gets the selected indices in ascending order, element e
-// (lane + 32 r) in asc[r] for e < H (when asc != null). Returns false, with
-// nothing written, when more than 64 keys reach the bound. Requires c > H. `cand`
+// index ascending). Returns false, with nothing written, when more than 64 keys
+// reach the bound. Requires c > H. `cand`
 // is 64 uint2 of this warp's shared memory.
 template <int KREG>
 __device__ __forceinline__ bool pivot2_select_keys(const uint32_t (&keys)[KREG], int c, int H, uint2* cand,
-                                                   uint32_t* tkey, int* tidx, uint32_t (*asc)[2] = nullptr) {
+                                                   uint32_t* tkey, int* tidx) {
   const int lane = threadIdx.x & 31;
   uint32_t top[2] = {0u, 0u};   // this lane's two largest keys (empty slots hold key 0)
 #pragma unroll
@@ -591,16 +590,6 @@ __device__ __forceinline__ bool pivot2_select_keys(const uint32_t (&keys)[KREG],
   const uint64_t th = __shfl_sync(0xffffffffu, v[hb >> 5], hb & 31);
   *tkey = (uint32_t)(th >> 32);
   *tidx = (int)(0xffffffffu - (uint32_t)th);
-  if (asc) {
-    // Elements 0..H-1 hold the selection; order it by index (complements sorted
-    // descending), the unselected elements last.
-    uint32_t comp[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) comp[r] = (lane + 32 * r < H) ? (uint32_t)v[r] : 0u;
-    warp_sort64_desc(comp);
-#pragma unroll
-    for (int r = 0; r < 2; ++r) (*asc)[r] = 0xffffffffu - comp[r];
-  }
   return true;
 }
 

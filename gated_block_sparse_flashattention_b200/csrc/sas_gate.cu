@@ -55,22 +55,14 @@ __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], i
     if (out && lane < H) out[lane] = base + (int32_t)asc;   // exactly H blocks, ascending
     return;
   }
-  uint32_t asc2[2];
-  if (H > 16 && H <= 63 &&
-      pivot2_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, out ? &asc2 : nullptr)) {
-    if (lane == 0) {
-      *tau_out = key_float(tkey);
-      *tidx_out = base + tidx;
-    }
-    if (out) {
-      if (lane < H) out[lane] = base + (int32_t)asc2[0];
-      if (lane + 32 < H) out[lane + 32] = base + (int32_t)asc2[1];
-    }
-    return;
+  // Larger budgets: the threshold from the lanes' two largest keys when that
+  // bounds it, else the bisection; the ascending list (when requested) then by a
+  // ballot over the row's keys in block order.
+  if (!(H > 16 && H <= 63 && pivot2_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx))) {
+    int take_eq = 0;
+    tkey = radix_select_keys(keys, c, H, nullptr, &take_eq);
+    tidx = tie_index_keys(keys, c, tkey, take_eq);
   }
-  int take_eq = 0;
-  tkey = radix_select_keys(keys, c, H, nullptr, &take_eq);
-  tidx = tie_index_keys(keys, c, tkey, take_eq);
   if (lane == 0) {
     *tau_out = key_float(tkey);
     *tidx_out = base + tidx;

@@ -260,9 +260,10 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * device-side bounds error and its extra blocks are not attended). For bf16 the
  * workspace holds per-block row lists and one partial output per (position,
  * attended block), about T * K * Hq/Hkv KiB per (b, g), processed in batches of
- * (b, g) of at most 8 GiB of partials; when one (b, g) alone needs more, the
- * call runs a q-tile kernel over the union of each tile's blocks instead and the
- * workspace is small.
+ * (b, g) of at most 8 GiB of partials; when one (b, g) alone needs more, or a
+ * row has more than 1024 partials (min(K, NB + 1) x Hq/Hkv), the call runs a
+ * q-tile kernel over the union of each tile's blocks instead and the workspace is
+ * small.
  * ws: workspace of sas_fwd_workspace_size bytes (same K).
  */
 SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, const float* logG, const float* gate_lse,
