@@ -363,6 +363,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idesc_s = make_idesc_bf16(128, 64, 0, 0);    // rows x keys, K = features
       const uint32_t idesc_t = make_idesc_bf16(128, 64, 1, 1);    // features x keys, K = rows
       const uint32_t idesc_q = make_idesc_bf16(128, D, 0, 1);     // rows x features, K = keys
+      // Shared-memory descriptors: the address field is the byte address / 16, so
+      // an operand at base + off (off a multiple of 16, inside the 256 KiB the
+      // field spans) has descriptor desc(base) + off / 16. The bases are taken
+      // once; each MMA adds a constant.
+      const uint64_t d_k = make_sdesc(s_base + OFF_K, 16, 1024);             // K_j, K-major (S, dQ's B below)
+      const uint64_t d_v = make_sdesc(s_base + OFF_V, 16, 1024);             // V_j, K-major
+      const uint64_t d_qd = make_sdesc(s_base + OFF_QD, 16, 1024);           // stage 0 Q; dO at + TILE
+      const uint64_t d_qd_t = make_sdesc(s_base + OFF_QD, HALF128, 1024);    // the same, MN-major
+      const uint64_t d_p_t = make_sdesc(s_base + OFF_P, HALF128, 1024);
+      const uint64_t d_ds_t = make_sdesc(s_base + OFF_DS, HALF128, 1024);
+      const uint64_t d_ds = make_sdesc(s_base + OFF_DS, 16, 1024);
+      const uint64_t d_k_q = make_sdesc(s_base + OFF_K, KV_HALF, 1024);
       bool ok = mbar_wait(&bars->kv_full, 0, status, wait_ns);
       int ns = 0, nb = 0;
       uint64_t t_last = global_ns();
@@ -374,18 +386,18 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (mbar_test_wait(&bars->qd_full[st], (ns / NST) & 1) &&
               (ns == 0 || mbar_test_wait(&bars->sp_free, (ns - 1) & 1))) {
             tc_fence_after();
-            const uint32_t qb = s_base + OFF_QD + st * 2 * TILE;
+            const uint64_t qs = (uint64_t)(st * 2 * TILE) >> 4;   // this stage's offset in descriptor units
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
-              umma_ss(tmem + COL_S, make_sdesc(qb + half * HALF128 + koff, 16, 1024),
-                      make_sdesc(s_base + OFF_K + half * KV_HALF + koff, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+              umma_ss(tmem + COL_S, d_qd + qs + ((half * HALF128 + koff) >> 4), d_k + ((half * KV_HALF + koff) >> 4),
+                      idesc_s, ks > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
-              umma_ss(tmem + COL_DP, make_sdesc(qb + TILE + half * HALF128 + koff, 16, 1024),
-                      make_sdesc(s_base + OFF_V + half * KV_HALF + koff, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+              umma_ss(tmem + COL_DP, d_qd + qs + ((TILE + half * HALF128 + koff) >> 4),
+                      d_v + ((half * KV_HALF + koff) >> 4), idesc_s, ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars->s_full);
             ++ns;
@@ -396,22 +408,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             (nb < 2 || mbar_test_wait(&bars->dq_free[nb & 1], ((nb - 2) >> 1) & 1))) {
           tc_fence_after();
           const int st = nb % NST, qb_ = nb & 1;
-          const uint32_t qb = s_base + OFF_QD + st * 2 * TILE;
+          const uint64_t qs = (uint64_t)(st * 2 * TILE) >> 4;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per MMA
-            umma_ss(tmem + COL_DV, make_sdesc(qb + TILE + ks * 2048, HALF128, 1024),
-                    make_sdesc(s_base + OFF_P + ks * 2048, HALF128, 1024), idesc_t, (nb > 0 || ks > 0) ? 1u : 0u);
+            umma_ss(tmem + COL_DV, d_qd_t + qs + ((TILE + ks * 2048) >> 4), d_p_t + ((ks * 2048) >> 4), idesc_t,
+                    (nb > 0 || ks > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            umma_ss(tmem + COL_DK, make_sdesc(qb + ks * 2048, HALF128, 1024),
-                    make_sdesc(s_base + OFF_DS + ks * 2048, HALF128, 1024), idesc_t, (nb > 0 || ks > 0) ? 1u : 0u);
+            umma_ss(tmem + COL_DK, d_qd_t + qs + ((ks * 2048) >> 4), d_ds_t + ((ks * 2048) >> 4), idesc_t,
+                    (nb > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&bars->qd_empty[st]);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {   // dQ partial = dS K_j, K = 64 keys
-            umma_ss(tmem + COL_DQ0 + 128 * qb_, make_sdesc(s_base + OFF_DS + ks * 32, 16, 1024),
-                    make_sdesc(s_base + OFF_K + ks * 2048, KV_HALF, 1024), idesc_q, ks > 0 ? 1u : 0u);
+            umma_ss(tmem + COL_DQ0 + 128 * qb_, d_ds + ((ks * 32) >> 4), d_k_q + ((ks * 2048) >> 4), idesc_q,
+                    ks > 0 ? 1u : 0u);
           }
           umma_commit(&bars->dq_done[qb_]);
           umma_commit(&bars->pd_free);

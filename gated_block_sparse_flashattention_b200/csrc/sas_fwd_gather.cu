@@ -312,6 +312,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc_bf16(128, 64, 0, 0);    // rows x keys, K = features
       const uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);    // rows x features, K = keys
+      // Shared-memory descriptors: the address field is the byte address / 16, so
+      // an operand at base + off (off a multiple of 16, inside the 256 KiB the
+      // field spans) has descriptor desc(base) + off / 16. The bases are taken
+      // once; each MMA adds a constant.
+      const uint64_t d_q = make_sdesc(s_base + OFF_Q, 16, 1024);
+      const uint64_t d_k = make_sdesc(s_base + OFF_K, 16, 1024);
+      const uint64_t d_v = make_sdesc(s_base + OFF_V, KV_HALF, 1024);
       bool ok = mbar_wait(&bars->kv_full, 0, status, wait_ns);
       int ns = 0, np = 0;
       uint64_t t_last = global_ns();
@@ -323,12 +330,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (mbar_test_wait(&bars->q_full[st], (ns / NST) & 1) &&
               (ns < 2 || mbar_test_wait(&bars->s_free[sb], ((ns - 2) >> 1) & 1))) {
             tc_fence_after();
-            const uint32_t qb = s_base + OFF_Q + st * QTILE;
+            const uint64_t qs = (uint64_t)(st * QTILE) >> 4;   // this stage's offset in descriptor units
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
-              umma_ss(tmem + COL_S + 64 * sb, make_sdesc(qb + half * HALF128 + koff, 16, 1024),
-                      make_sdesc(s_base + OFF_K + half * KV_HALF + koff, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+              umma_ss(tmem + COL_S + 64 * sb, d_q + qs + ((half * HALF128 + koff) >> 4),
+                      d_k + ((half * KV_HALF + koff) >> 4), idesc_s, ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars->s_full[sb]);
             ++ns;
@@ -340,11 +347,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (mbar_test_wait(&bars->p_full[pb], (np >> 1) & 1) &&
               (np < 2 || mbar_test_wait(&bars->o_free[pb], ((np - 2) >> 1) & 1))) {
             tc_fence_after();
-            const uint32_t vb = s_base + OFF_V;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {   // K = 64 keys, 16 per MMA; A = P (bf16 pairs) in TMEM
-              umma_ts(tmem + COL_O + 128 * pb, tmem + COL_S + 64 * pb + ks * 8,
-                      make_sdesc(vb + ks * 2048, KV_HALF, 1024), idesc_pv, ks > 0 ? 1u : 0u);
+              umma_ts(tmem + COL_O + 128 * pb, tmem + COL_S + 64 * pb + ks * 8, d_v + ((ks * 2048) >> 4), idesc_pv,
+                      ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars->o_full[pb]);
             umma_commit(&bars->s_free[pb]);
