@@ -48,8 +48,11 @@
  *    NULL = the legacy default stream). Arguments are validated on the host
  *    before anything is launched; an invalid call returns an error and
  *    launches nothing.
- *  - Kernel-side failures (a bounded wait that expired) are recorded in a status
- *    word at the start of the workspace; read it with sas_device_status().
+ *  - Kernel-side failures (a bounded wait that expired, an index out of range) are
+ *    recorded in a status word at the start of the workspace; read it with
+ *    sas_device_status(). Once the word holds an error, every later bounded wait
+ *    of the call gives up, so the outputs of that call are not defined; clear the
+ *    word (sas_device_status_clear) before reusing the workspace.
  *  - sm_scale multiplies q.k only; the log gate is added unscaled.
  *  - The fp32 data type runs on a CUDA-core kernel; bf16 runs on tcgen05
  *    tensor-core kernels (fwd/bwd: d = 128).
@@ -252,12 +255,13 @@ SAS_API int sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, i
  * padded). The bf16 kernels then build their per-block row lists from it (4 bytes
  * per selected block) instead of thresholding each row's gates again; the
  * attended set and the results are the same. An entry that is not an earlier
- * block of its row is skipped and reported as a device-side bounds error.
+ * block of its row is never used to index anything and is reported as a
+ * device-side bounds error (the call's outputs are then not defined).
  * O [B,Hq,T,d] of `dtype`; LSE [B,Hq,T] fp32. T % 64 == 0, NB == T / 64,
  * Hq % Hkv == 0, d in {64, 128} (fp32) or d == 128 (bf16).
  * Kbudget: the budget K given to the selection (the threshold keeps at most K-1
  * historical blocks per row; a threshold that keeps more is reported as a
- * device-side bounds error and its extra blocks are not attended). For bf16 the
+ * device-side bounds error, and the call's outputs are then not defined). For bf16 the
  * workspace holds per-block row lists and one partial output per (position,
  * attended block), about T * K * Hq/Hkv KiB per (b, g), processed in batches of
  * (b, g) of at most 8 GiB of partials; when one (b, g) alone needs more, or a
@@ -283,7 +287,8 @@ SAS_API int sas_fwd(const void* Q, const void* K, const void* V, int dtype, cons
  * (fully written: zero outside the selection). Kbudget: the budget K given to
  * sas_select_threshold (the threshold keeps at most K-1 historical blocks per row;
  * internal per-block row lists are sized by it; a threshold that keeps more is
- * reported as a device-side bounds error). ws: sas_bwd_workspace_size bytes
+ * reported as a device-side bounds error, and the outputs are then not defined).
+ * ws: sas_bwd_workspace_size bytes
  * (for bf16 it holds an fp32 dQ accumulator and the per-block row lists).
  */
 SAS_API int sas_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, int dtype,
@@ -319,8 +324,9 @@ SAS_API int sas_decode_fwd(const void* q, const void* Kc, const void* Vc, int dt
  * Kp/Vp [num_pages, Hkv, 64, d] bf16: one page holds one 64-token block of every
  * KV head (the head's 64 rows contiguous). page_table [B, max_pages] int32
  * DEVICE; entries of blocks 0..(seqlen[b]-1)/64 must lie in 0..num_pages-1 (an
- * entry outside is reported as a device-side bounds error and its block is
- * skipped); entries past a sequence's last block are never read. Pages may be
+ * entry outside is reported as a device-side bounds error and no copy is issued
+ * for its block; o is then not defined); entries past a sequence's last block are
+ * never read. Pages may be
  * shared between sequences. seqlen [B] int32 DEVICE, 1 <= L <= max_pages * 64.
  * s [B,Hkv,NBmax] fp32 with NBmax >= max_pages. Other arguments, the workspace
  * (sas_decode_workspace_size with Lmax = max_pages * 64) and errors as for

@@ -72,3 +72,29 @@ def test_lists_from_sel_give_the_same_attention(kind, w):
     assert max_abs(to_np(O1), ref["O"]) <= 2e-2
     for name, got in zip(("dQ", "dK", "dV", "dLogG"), g1):
         assert rel_l2(to_np(got), ref[name]) <= 1e-2, name
+
+
+def test_sel_entries_outside_their_row_are_reported():
+    """An index-list entry that is not an earlier block of its row (here the row's own block, and one past the
+    block count) is never used as an index: it is reported as a bounds error in the status word, and the call
+    completes (every wait of the call then gives up, so its outputs are not defined). After the word is
+    cleared, a call on the same workspace with a correct list is clean and equals the thresholding path."""
+    w = workloads.custom("sel_bad", "bf16", B=1, Hq=8, Hkv=2, d=128, T=1024, K=4)
+    inp = workloads.make_training_inputs(w, seed=31)
+    Q, K, V, s = (dev(inp[k]) for k in ("Q", "K", "V", "s"))
+    logG, tau, tidx, sel = binding.gate_and_select(s, w.K, want_sel=True)
+    bad = sel.clone()
+    bad[0, 0, 200, 0] = 200 // w.block      # the row's own block: not historical
+    bad[0, 1, 900, 1] = 1000                # past the block count
+    ws = binding.workspace(binding.sas_fwd_workspace_size(w.B, w.Hq, w.Hkv, w.T, w.d, w.K, 1))
+    O_ref, L_ref = binding.forward(Q, K, V, logG, tau, tidx, w.K, w.sm_scale)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(w.B, w.Hq, w.T, device="cuda")
+    binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws, sel=bad)
+    torch.cuda.synchronize()
+    assert binding.sas_device_status(ws) == 2          # bounds error
+    binding.sas_device_status_clear(ws)
+    binding.sas_fwd(Q, K, V, logG, tau, tidx, O, LSE, w.K, w.sm_scale, ws, sel=sel)
+    torch.cuda.synchronize()
+    assert binding.sas_device_status(ws) == 0
+    assert torch.equal(O, O_ref) and torch.equal(LSE, L_ref)
