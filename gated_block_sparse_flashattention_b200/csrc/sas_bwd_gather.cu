@@ -10,7 +10,7 @@
 // of its rows' blocks (most of the tile masked), each CTA owns one KV block j of
 // one (b, g) and visits exactly the rows that attend it: its own 64 positions
 // (causal) and the positions that selected j, gathered P at a time (x G heads
-// = up to 128 rows) with TMA row-gather loads. Per tile, on tcgen05:
+// = up to 128 rows) by cp.async copies of packed chunks. Per tile, on tcgen05:
 //   S = Q K_j^T, dP = dO V_j^T              (M = 128 rows, N = 64 keys)
 //   dV_j^T += dO^T P, dK_j^T += Q^T dS      (M = 128 features, N = 64 keys, K = rows)
 //   dQ_rows = dS K_j                        (M = 128 rows, N = 128 features, K = 64 keys)

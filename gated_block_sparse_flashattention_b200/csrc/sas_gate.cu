@@ -44,9 +44,8 @@ __device__ __forceinline__ void select_keys_regs(const uint32_t (&keys)[KREG], i
   const int lane = threadIdx.x & 31;
   uint32_t tkey = 0u, asc = 0u;
   int tidx = -1;
-  // The ascending list (a second warp sort) only when it is requested. Budgets
-  // up to 16 blocks bound the threshold by the lanes' largest keys, larger ones
-  // (up to 63) by their two largest.
+  // Budgets up to 16 blocks: the threshold from the lanes' largest keys, and the
+  // ascending list (when requested) by a second warp sort of the 32 candidates.
   if (H <= 16 && pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(hist), &tkey, &tidx, out ? &asc : nullptr)) {
     if (lane == 0) {
       *tau_out = key_float(tkey);
