@@ -5,7 +5,10 @@
 // §5.1 "Inference implementation" (per-KV-group selection, GQA, gathering only
 // the selected KV blocks).
 //
-// bf16 storage, three kernels:
+// bf16 storage, contiguous cache, rows of up to 512 blocks and at least three
+// (b, g) groups per four SMs: one kernel, decode_group_kernel, one CTA per
+// (b, g) that selects, streams the group's blocks and writes o.
+// Otherwise (paged caches, longer rows, fewer groups), three kernels:
 //   decode_select_kernel    one warp (one CTA) per (b, g): Top-(K-1) of the score
 //                           row; the attended list [c, selected blocks] goes to
 //                           the workspace (rows over 1024 blocks:
@@ -1351,6 +1354,331 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
   }
 }
 
+// ---------------------------------------------------------------------------- one CTA per (b, g), bf16
+// The decode step in one kernel, for problems with about as many groups as SMs:
+// CTA (b, g) selects the group's blocks itself, streams them through an NS-stage
+// TMA ring and writes the group's G rows of o. No partials, no merge, and the
+// copy of the current block (which needs no selection) starts before the
+// selection runs.
+//
+// Warp 4, the producer, loads the sequence length and the score row together,
+// starts the copies of q and of the current block into stage 0, selects the
+// other blocks into the attended list in shared memory (and sel_out), then fills
+// one stage per attended block as the stages come free; a stage holding block
+// -1 ends the list. Warps 0-3 compute each block as decode_fused_mma_kernel's
+// warps do: each owns 16 of the block's 64 keys, with its own online softmax
+// state in registers. After the last block the four states go to shared memory
+// (the ring's first 32 KB, free by then) and are combined in warp order, so the
+// result does not depend on timing.
+constexpr int kGrpThreads = 32 * (kDecWarps + 1);
+constexpr uint32_t kGrpWarpOut = 16u * D * 4u;   // one warp's [16 rows][D] fp32 output
+static_assert(kDecWarps * kGrpWarpOut <= kStageBytes, "the combined outputs fit in one ring stage");
+
+struct GroupLayout {
+  uint32_t q, zero, comb, att, scratch, bar, total;
+};
+__host__ __device__ inline GroupLayout group_layout(int NS, int K) {
+  GroupLayout l;
+  l.q = (uint32_t)NS * kStageBytes;      // q rows of the group: up to 16 x 256 bytes
+  l.zero = l.q + 16u * 256u;             // one zero row (MMA rows G..15)
+  l.comb = l.zero + 256u;                // [warps][16 rows] (max, sum)
+  l.att = l.comb + kDecWarps * 16 * 2 * 4;   // attended list: [current, selected...]
+  l.scratch = l.att + ((uint32_t)K * 4u + 15u) / 16u * 16u;   // 256 words for the selection
+  l.bar = l.scratch + 1024u;             // full/empty barriers, stage blocks, copies, group info
+  l.total = l.bar + 256u;
+  return l;
+}
+
+template <int NS, int KREG>
+__global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
+    decode_group_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
+                        const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int G = p.G, K = p.K;
+  const int bg = blockIdx.x, b = bg / p.Hkv, g = bg % p.Hkv;
+  const GroupLayout lay = group_layout(NS, K);
+  uint8_t* qs = smem + lay.q;
+  uint8_t* zrow = smem + lay.zero;
+  float* comb = reinterpret_cast<float*>(smem + lay.comb);
+  int32_t* att_s = reinterpret_cast<int32_t*>(smem + lay.att);
+  uint32_t* sel_scratch = reinterpret_cast<uint32_t*>(smem + lay.scratch);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar);
+  uint64_t* empty = full + NS;
+  int* stage_m = reinterpret_cast<int*>(empty + NS);   // block in each stage; -1 ends the list
+  int* issued = stage_m + NS;                          // last list position placed in each stage (-1: none)
+  int* info = issued + NS;                             // sequence length, current block, log-gate LSE (float)
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecWarps);
+      issued[s] = -1;
+    }
+    fence_barrier_init();
+  }
+  if (warp == 0) reinterpret_cast<uint2*>(zrow)[lane] = make_uint2(0u, 0u);
+  __syncthreads();
+
+  if (warp == kDecWarps) {
+    // ------------------------------------------------------------ producer and selection
+    const float* srow = p.s + (long long)bg * p.NBmax;
+    float sv[KREG];
+#pragma unroll
+    for (int i = 0; i < KREG; ++i) sv[i] = (lane + 32 * i < p.NBmax) ? __ldg(srow + lane + 32 * i) : 0.f;
+    const int L = p.seqlen[b];
+    const bool valid = L >= 1 && L <= p.Lmax;
+    const int c = valid ? (L - 1) / kBlock : 0;
+    if (lane == 0) {
+      info[0] = L;
+      info[1] = c;
+      if (!valid) {   // a sequence length outside the cache: nothing attended
+        set_status(p.status, SAS_DEV_ERR_BOUNDS);
+        stage_m[0] = -1;
+        mbar_arrive(&full[0]);
+        issued[0] = 0;
+      } else {
+        stage_m[0] = c;
+        mbar_expect_tx(&full[0], (uint32_t)G * 256u + kStageBytes);
+        tma_load_2d(qs, &tmq, &full[0], 0, b * p.Hq + g * G);
+        tma_load_3d(smem, &tmk, &full[0], 0, c * kBlock, bg);
+        tma_load_3d(smem + 8192, &tmk, &full[0], 64, c * kBlock, bg);
+        tma_load_3d(smem + kMmaTileBytes, &tmv, &full[0], 0, c * kBlock, bg);
+        tma_load_3d(smem + kMmaTileBytes + 8192, &tmv, &full[0], 64, c * kBlock, bg);
+        issued[0] = 0;
+      }
+    }
+    const int H = K - 1;
+    int32_t* so = p.sel_out ? p.sel_out + (long long)bg * H : nullptr;
+    int pos = 0;
+    if (valid) {
+      const int mode = (min(c, H) == 0) ? 0 : (c <= H ? 1 : 2);
+      pos = -1;
+      if (mode == 2 && H <= 32) {
+        uint32_t keys[KREG];
+#pragma unroll
+        for (int i = 0; i < KREG; ++i) keys[i] = (lane + 32 * i < c) ? float_key(sv[i]) : 0u;
+        uint32_t tk = 0u, asc = 0u, top = 0u;
+        int tidx = -1;
+        if (pivot_select_keys(keys, c, H, reinterpret_cast<uint2*>(sel_scratch), &tk, &tidx, so ? &asc : nullptr,
+                              so ? nullptr : &top)) {
+          if (lane < H) {
+            att_s[1 + lane] = (int32_t)(so ? asc : top);
+            if (so) so[lane] = (int32_t)asc;
+          }
+          pos = H;
+        }
+      }
+      if (pos < 0) pos = select_row(srow, c, H, mode, sel_scratch, att_s, so);
+      const float lse = p.apply_log_gate ? row_lse(srow, c) : 0.f;
+      if (lane == 0) reinterpret_cast<float*>(info)[2] = lse;
+    }
+    if (so)
+      for (int k = pos + lane; k < H; k += 32) so[k] = -1;
+    __syncwarp();   // the list (written by every lane) is visible to lane 0
+    bool ok = true;
+    // Position n of the list goes to stage n % NS; position 1 + pos is the end marker.
+    for (int n = 1; valid && ok && n <= 1 + pos; ++n) {
+      const int s = n % NS;
+      if (n >= NS) ok = warp_wait(&empty[s], (uint32_t)(n / NS - 1) & 1u, p.status);
+      if (!ok) break;
+      if (lane == 0) {
+        if (n <= pos) {
+          const int m = att_s[n];
+          stage_m[s] = m;
+          fence_proxy_async_smem();
+          mbar_expect_tx(&full[s], kStageBytes);
+          uint8_t* st = smem + s * kStageBytes;
+          tma_load_3d(st, &tmk, &full[s], 0, m * kBlock, bg);
+          tma_load_3d(st + 8192, &tmk, &full[s], 64, m * kBlock, bg);
+          tma_load_3d(st + kMmaTileBytes, &tmv, &full[s], 0, m * kBlock, bg);
+          tma_load_3d(st + kMmaTileBytes + 8192, &tmv, &full[s], 64, m * kBlock, bg);
+          issued[s] = n;
+        } else {
+          stage_m[s] = -1;
+          mbar_arrive(&full[s]);
+          issued[s] = n;
+        }
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ consumers (warps 0-3)
+    const int r8 = lane & 7, mi = lane >> 3;
+    const uint32_t k_row = (uint32_t)(16 * warp + (mi >> 1) * 8 + r8) * 128u;
+    const uint32_t v_row = (uint32_t)(16 * warp + (mi & 1) * 8 + r8) * 128u;
+    uint32_t k_x[4], v_x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      k_x[j] = (uint32_t)(((2 * j + (mi & 1)) ^ r8) << 4);
+      v_x[j] = (uint32_t)(((2 * j + (mi >> 1)) ^ r8) << 4);
+    }
+    const int qrow = r8 + (mi & 1) * 8;
+    float run_m0 = -INFINITY, run_m1 = -INFINITY, run_l0 = 0.f, run_l1 = 0.f;   // log2 domain
+    float oacc[16][4];
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd) oacc[nd][0] = oacc[nd][1] = oacc[nd][2] = oacc[nd][3] = 0.f;
+    uint32_t qa[8][4];
+    int L = 0, c = 0;
+    for (int n = 0;; ++n) {
+      const int s = n % NS;
+      if (!warp_wait(&full[s], (uint32_t)(n / NS) & 1u, p.status)) break;
+      const int m = stage_m[s];
+      if (m < 0) break;
+      if (n == 0) {   // the group's length and q rows arrived with stage 0
+        L = info[0];
+        c = info[1];
+        const uint32_t qa_addr = (qrow < G) ? smem_u32(qs + qrow * 256) + (mi >> 1) * 16u : smem_u32(zrow);
+        const uint32_t qstep = (qrow < G) ? 32u : 0u;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) ldsm_x4(qa_addr + ks * qstep, qa[ks]);
+      }
+      const int nk = (m == c) ? (L - m * kBlock) : kBlock;   // keys present in this block
+      const uint32_t st = smem_u32(smem + s * kStageBytes);
+      bool zeroed = false;
+      if (nk < 16 * warp + 16) {
+        // Rows past the end of the sequence may hold any bits; P is zero there, and
+        // zero V rows keep 0 * NaN out of the P V products.
+        uint8_t* vs = smem + s * kStageBytes + kMmaTileBytes;
+        const int row0 = max(nk, 16 * warp);
+        for (int i = lane; i < (16 * warp + 16 - row0) * 16; i += 32) {
+          const int row = row0 + i / 16, chunk = i % 16;
+          *reinterpret_cast<uint4*>(vs + kv_tile_offset(row, chunk)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+        zeroed = true;
+      }
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t r[4];
+        ldsm_x4(st + (ks >> 2) * 8192u + k_row + k_x[ks & 3], r);
+        mma16816(sacc[0], qa[ks], r[0], r[1]);
+        mma16816(sacc[1], qa[ks], r[2], r[3]);
+      }
+      // The list positions past 0 were filled after the log-gate LSE was stored.
+      const float bias =
+          (p.apply_log_gate && m != c) ? p.s[(long long)bg * p.NBmax + m] - reinterpret_cast<float*>(info)[2] : 0.f;
+      const float sl2 = p.sm_scale * kLog2e, bl2 = bias * kLog2e;
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[j][e] = fmaf(sacc[j][e], sl2, bl2);
+      if (nk < kBlock) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (16 * warp + 8 * j + 2 * tig + (e & 1) >= nk) sacc[j][e] = -INFINITY;
+      }
+      float mx0 = fmaxf(fmaxf(sacc[0][0], sacc[0][1]), fmaxf(sacc[1][0], sacc[1][1]));
+      float mx1 = fmaxf(fmaxf(sacc[0][2], sacc[0][3]), fmaxf(sacc[1][2], sacc[1][3]));
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (__any_sync(0xffffffffu, mx0 > run_m0 + 8.f || mx1 > run_m1 + 8.f)) {
+        const float nm0 = fmaxf(run_m0, mx0), nm1 = fmaxf(run_m1, mx1);
+        const float a0 = (run_m0 == -INFINITY) ? 0.f : ex2(run_m0 - nm0);
+        const float a1 = (run_m1 == -INFINITY) ? 0.f : ex2(run_m1 - nm1);
+        run_m0 = nm0;
+        run_m1 = nm1;
+        run_l0 *= a0;
+        run_l1 *= a1;
+#pragma unroll
+        for (int nd = 0; nd < 16; ++nd) {
+          oacc[nd][0] *= a0;
+          oacc[nd][1] *= a0;
+          oacc[nd][2] *= a1;
+          oacc[nd][3] *= a1;
+        }
+      }
+      const float sub0 = (run_m0 == -INFINITY) ? 0.f : run_m0, sub1 = (run_m1 == -INFINITY) ? 0.f : run_m1;
+      float pv[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        pv[j][0] = ex2(sacc[j][0] - sub0);
+        pv[j][1] = ex2(sacc[j][1] - sub0);
+        pv[j][2] = ex2(sacc[j][2] - sub1);
+        pv[j][3] = ex2(sacc[j][3] - sub1);
+      }
+      run_l0 += (pv[0][0] + pv[0][1]) + (pv[1][0] + pv[1][1]);
+      run_l1 += (pv[0][2] + pv[0][3]) + (pv[1][2] + pv[1][3]);
+      const uint32_t pa[4] = {pack_bf16(pv[0][0], pv[0][1]), pack_bf16(pv[0][2], pv[0][3]),
+                              pack_bf16(pv[1][0], pv[1][1]), pack_bf16(pv[1][2], pv[1][3])};
+      const uint32_t vst = st + kMmaTileBytes;
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {
+        uint32_t r[4];
+        ldsm_x4_t(vst + (np >> 2) * 8192u + v_row + v_x[np & 3], r);
+        mma16816(oacc[2 * np], pa, r[0], r[1]);
+        mma16816(oacc[2 * np + 1], pa, r[2], r[3]);
+      }
+      if (zeroed) fence_proxy_async_smem();   // the generic writes come before the stage's next copy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // ------------------------------------------------------------ combine the four warps, write o
+    float l0 = run_l0, l1 = run_l1;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    named_bar_sync(1, 32 * kDecWarps);   // every consumer is done with the ring
+    float* wout = reinterpret_cast<float*>(smem) + warp * (kGrpWarpOut / 4);
+    if (tig == 0) {
+      comb[(warp * 16 + gid) * 2] = run_m0;
+      comb[(warp * 16 + gid) * 2 + 1] = l0;
+      comb[(warp * 16 + gid + 8) * 2] = run_m1;
+      comb[(warp * 16 + gid + 8) * 2 + 1] = l1;
+    }
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd) {
+      *reinterpret_cast<float2*>(wout + gid * D + nd * 8 + 2 * tig) = make_float2(oacc[nd][0], oacc[nd][1]);
+      *reinterpret_cast<float2*>(wout + (gid + 8) * D + nd * 8 + 2 * tig) = make_float2(oacc[nd][2], oacc[nd][3]);
+    }
+    named_bar_sync(1, 32 * kDecWarps);
+    const float* wall = reinterpret_cast<const float*>(smem);
+    for (int i = tid; i < G * (D / 4); i += 32 * kDecWarps) {
+      const int h = i / (D / 4), d4 = i % (D / 4);
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, comb[(w * 16 + h) * 2]);
+      float den = 0.f;
+      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float mw = comb[(w * 16 + h) * 2];
+        if (mw != -INFINITY) {
+          const float a = ex2(mw - M);
+          den = fmaf(a, comb[(w * 16 + h) * 2 + 1], den);
+          const float4 v = *reinterpret_cast<const float4*>(wall + w * (kGrpWarpOut / 4) + h * D + d4 * 4);
+          num.x = fmaf(a, v.x, num.x);
+          num.y = fmaf(a, v.y, num.y);
+          num.z = fmaf(a, v.z, num.z);
+          num.w = fmaf(a, v.w, num.w);
+        }
+      }
+      const float sc = 1.f / den;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.o) +
+                                                              ((long long)b * p.Hq + g * G + h) * D + d4 * 4);
+      dst[0] = __floats2bfloat162_rn(num.x * sc, num.y * sc);
+      dst[1] = __floats2bfloat162_rn(num.z * sc, num.w * sc);
+    }
+  }
+  __syncthreads();
+  if (tid == kDecWarps * 32 && *reinterpret_cast<volatile int32_t*>(p.status) != 0) {
+    // A wait gave up, so copies may still be in flight: they finish before the CTA
+    // exits. Each stage's last fill (a copy or the end marker) is the phase waited
+    // for; every earlier phase of the stage completes before it.
+    for (int s = 0; s < NS; ++s)
+      if (issued[s] >= 0) mbar_wait_drain(&full[s], (uint32_t)(issued[s] / NS) & 1u);
+  }
+}
+
 size_t smem_bytes(int dtype, int G) {
   const size_t el = dtype == 1 ? 2 : 4;
   return 2 * kBlock * D * el + ((size_t)G * kBlock + 2 * G + 2) * 4 + 8 + 16 + 128;
@@ -1414,6 +1742,44 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
   prm.n_slots = pb.K;
   prm.sm_scale = pb.sm_scale;
   cudaError_t e;
+  if (pb.dtype == 1 && !pb.page_table && pb.NBmax <= 512) {
+    // Contiguous bf16 cache, rows of up to 512 blocks and at least three groups
+    // per four SMs: the whole step is decode_group_kernel, one CTA
+    // per (b, g) (six ring stages and one CTA per SM up to one group per SM,
+    // three stages and two CTAs per SM beyond).
+    int dev = 0, sms = 148, smem_max = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+      return e;
+    const int NS = (long long)n_bg <= sms ? 6 : 3;
+    const size_t shm = group_layout(NS, pb.K).total + 1024;
+    if (4LL * (long long)n_bg >= 3LL * sms && shm <= (size_t)smem_max) {
+      CUtensorMap tk, tv, tq;
+      if (!make_tmap_bf16_3d(&tk, pb.Kc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
+          !make_tmap_bf16_3d(&tv, pb.Vc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
+          !make_tmap_bf16_rows(&tq, pb.q, D, (uint64_t)pb.B * pb.Hq, (uint32_t)G))
+        return cudaErrorInvalidValue;
+      auto group = [&](auto kernel) -> cudaError_t {
+        cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+        if (r != cudaSuccess) return r;
+        r = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (r != cudaSuccess) return r;
+        kernel<<<(unsigned)n_bg, kGrpThreads, shm, st>>>(prm, tk, tv, tq);
+        count_launch();
+        return cudaGetLastError();
+      };
+      if (NS == 6) {
+        if (pb.NBmax <= 128) return group(decode_group_kernel<6, 4>);
+        if (pb.NBmax <= 256) return group(decode_group_kernel<6, 8>);
+        return group(decode_group_kernel<6, 16>);
+      }
+      if (pb.NBmax <= 128) return group(decode_group_kernel<3, 4>);
+      if (pb.NBmax <= 256) return group(decode_group_kernel<3, 8>);
+      return group(decode_group_kernel<3, 16>);
+    }
+  }
   // Selection first (it also clears the counters); the attention kernel follows.
   // Both prefer all of L1 as shared memory, so that attention CTAs can start on
   // an SM while a selection CTA still runs there (a carveout change would have to
