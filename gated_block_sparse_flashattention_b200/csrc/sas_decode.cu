@@ -1361,44 +1361,52 @@ __global__ void __launch_bounds__(32 * kDecWarps, 2)
 // copy of the current block (which needs no selection) starts before the
 // selection runs.
 //
-// Warp 4, the producer, loads the sequence length and the score row together,
-// starts the copies of q and of the current block into stage 0, selects the
-// other blocks into the attended list in shared memory (and sel_out), then fills
-// one stage per attended block as the stages come free; a stage holding block
-// -1 ends the list. Warps 0-3 compute each block as decode_fused_mma_kernel's
-// warps do: each owns 16 of the block's 64 keys, with its own online softmax
-// state in registers. After the last block the four states go to shared memory
-// (the ring's first 32 KB, free by then) and are combined in warp order, so the
+// The producer warp (the last one) loads the sequence length and the score row
+// together, starts the copies of q and of the current block, selects the other
+// blocks into the attended list in shared memory (and sel_out), then fills one
+// stage per attended block as the stages come free; a stage holding block -1
+// ends the list. The compute warps form NSET sets of four. Set j takes the list
+// positions n = j (mod NSET), from stages n % NS, so the sets work on different
+// blocks at once. In a set each warp owns 16 of a block's 64 keys, computed as
+// decode_fused_mma_kernel's warps do, with its own online softmax state in
+// registers. After the last block the warps' states go to shared memory (the
+// ring's first stages, free by then) and are combined in warp order, so the
 // result does not depend on timing.
-constexpr int kGrpThreads = 32 * (kDecWarps + 1);
 constexpr uint32_t kGrpWarpOut = 16u * D * 4u;   // one warp's [16 rows][D] fp32 output
-static_assert(kDecWarps * kGrpWarpOut <= kStageBytes, "the combined outputs fit in one ring stage");
+
+template <int NSET>
+__host__ __device__ constexpr int group_threads() {
+  return 32 * (kDecWarps * NSET + 1);
+}
 
 struct GroupLayout {
   uint32_t q, zero, comb, att, scratch, bar, total;
 };
-__host__ __device__ inline GroupLayout group_layout(int NS, int K) {
+__host__ __device__ inline GroupLayout group_layout(int NS, int NSET, int K) {
   GroupLayout l;
   l.q = (uint32_t)NS * kStageBytes;      // q rows of the group: up to 16 x 256 bytes
   l.zero = l.q + 16u * 256u;             // one zero row (MMA rows G..15)
-  l.comb = l.zero + 256u;                // [warps][16 rows] (max, sum)
-  l.att = l.comb + kDecWarps * 16 * 2 * 4;   // attended list: [current, selected...]
+  l.comb = l.zero + 256u;                // [compute warps][16 rows] (max, sum)
+  l.att = l.comb + (uint32_t)(kDecWarps * NSET) * 16u * 2u * 4u;   // attended list: [current, selected...]
   l.scratch = l.att + ((uint32_t)K * 4u + 15u) / 16u * 16u;   // 256 words for the selection
-  l.bar = l.scratch + 1024u;             // full/empty barriers, stage blocks, copies, group info
+  l.bar = l.scratch + 1024u;             // barriers, stage blocks, fills, group info
   l.total = l.bar + 256u;
   return l;
 }
 
-template <int NS, int KREG>
-__global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
+template <int NS, int NSET, int KREG>
+__global__ void __launch_bounds__(group_threads<NSET>(), NS <= 3 ? 2 : 1)
     decode_group_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq) {
+  constexpr int kCw = kDecWarps * NSET;   // compute warps; warp kCw produces
+  static_assert(NS % NSET == 0, "every stage belongs to one set");
+  static_assert(kCw * kGrpWarpOut <= NS * kStageBytes, "the warps' outputs fit in the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
   const int G = p.G, K = p.K;
   const int bg = blockIdx.x, b = bg / p.Hkv, g = bg % p.Hkv;
-  const GroupLayout lay = group_layout(NS, K);
+  const GroupLayout lay = group_layout(NS, NSET, K);
   uint8_t* qs = smem + lay.q;
   uint8_t* zrow = smem + lay.zero;
   float* comb = reinterpret_cast<float*>(smem + lay.comb);
@@ -1406,9 +1414,10 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
   uint32_t* sel_scratch = reinterpret_cast<uint32_t*>(smem + lay.scratch);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar);
   uint64_t* empty = full + NS;
-  int* stage_m = reinterpret_cast<int*>(empty + NS);   // block in each stage; -1 ends the list
+  uint64_t* qbar = empty + NS;                         // the q rows (one phase)
+  int* stage_m = reinterpret_cast<int*>(qbar + 1);     // block in each stage; -1 ends the list
   int* issued = stage_m + NS;                          // last list position placed in each stage (-1: none)
-  int* info = issued + NS;                             // sequence length, current block, log-gate LSE (float)
+  int* info = issued + NS;   // sequence length, current block, log-gate LSE (float), q copy issued
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -1416,12 +1425,14 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
       mbar_init(&empty[s], kDecWarps);
       issued[s] = -1;
     }
+    mbar_init(qbar, 1);
+    info[3] = 0;
     fence_barrier_init();
   }
   if (warp == 0) reinterpret_cast<uint2*>(zrow)[lane] = make_uint2(0u, 0u);
   __syncthreads();
 
-  if (warp == kDecWarps) {
+  if (warp == kCw) {
     // ------------------------------------------------------------ producer and selection
     const float* srow = p.s + (long long)bg * p.NBmax;
     float sv[KREG];
@@ -1435,13 +1446,12 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
       info[1] = c;
       if (!valid) {   // a sequence length outside the cache: nothing attended
         set_status(p.status, SAS_DEV_ERR_BOUNDS);
-        stage_m[0] = -1;
-        mbar_arrive(&full[0]);
-        issued[0] = 0;
       } else {
+        info[3] = 1;
+        mbar_expect_tx(qbar, (uint32_t)G * 256u);
+        tma_load_2d(qs, &tmq, qbar, 0, b * p.Hq + g * G);
         stage_m[0] = c;
-        mbar_expect_tx(&full[0], (uint32_t)G * 256u + kStageBytes);
-        tma_load_2d(qs, &tmq, &full[0], 0, b * p.Hq + g * G);
+        mbar_expect_tx(&full[0], kStageBytes);
         tma_load_3d(smem, &tmk, &full[0], 0, c * kBlock, bg);
         tma_load_3d(smem + 8192, &tmk, &full[0], 64, c * kBlock, bg);
         tma_load_3d(smem + kMmaTileBytes, &tmv, &full[0], 0, c * kBlock, bg);
@@ -1478,13 +1488,16 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
       for (int k = pos + lane; k < H; k += 32) so[k] = -1;
     __syncwarp();   // the list (written by every lane) is visible to lane 0
     bool ok = true;
-    // Position n of the list goes to stage n % NS; position 1 + pos is the end marker.
-    for (int n = 1; valid && ok && n <= 1 + pos; ++n) {
+    // Position n of the list goes to stage n % NS. Positions 0..P-1 hold blocks
+    // (position 0, the current block, is already on its way); the next NSET
+    // positions are end markers, one for each set.
+    const int P = valid ? 1 + pos : 0;
+    for (int n = valid ? 1 : 0; ok && n < P + NSET; ++n) {
       const int s = n % NS;
       if (n >= NS) ok = warp_wait(&empty[s], (uint32_t)(n / NS - 1) & 1u, p.status);
       if (!ok) break;
       if (lane == 0) {
-        if (n <= pos) {
+        if (n < P) {
           const int m = att_s[n];
           stage_m[s] = m;
           fence_proxy_async_smem();
@@ -1494,20 +1507,20 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
           tma_load_3d(st + 8192, &tmk, &full[s], 64, m * kBlock, bg);
           tma_load_3d(st + kMmaTileBytes, &tmv, &full[s], 0, m * kBlock, bg);
           tma_load_3d(st + kMmaTileBytes + 8192, &tmv, &full[s], 64, m * kBlock, bg);
-          issued[s] = n;
         } else {
           stage_m[s] = -1;
           mbar_arrive(&full[s]);
-          issued[s] = n;
         }
+        issued[s] = n;
       }
       __syncwarp();
     }
   } else {
-    // ------------------------------------------------------------ consumers (warps 0-3)
+    // ------------------------------------------------------------ compute warps
+    const int set = warp / kDecWarps, kw = warp % kDecWarps;   // kw: the warp's 16 keys of a block
     const int r8 = lane & 7, mi = lane >> 3;
-    const uint32_t k_row = (uint32_t)(16 * warp + (mi >> 1) * 8 + r8) * 128u;
-    const uint32_t v_row = (uint32_t)(16 * warp + (mi & 1) * 8 + r8) * 128u;
+    const uint32_t k_row = (uint32_t)(16 * kw + (mi >> 1) * 8 + r8) * 128u;
+    const uint32_t v_row = (uint32_t)(16 * kw + (mi & 1) * 8 + r8) * 128u;
     uint32_t k_x[4], v_x[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -1521,12 +1534,15 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
     for (int nd = 0; nd < 16; ++nd) oacc[nd][0] = oacc[nd][1] = oacc[nd][2] = oacc[nd][3] = 0.f;
     uint32_t qa[8][4];
     int L = 0, c = 0;
-    for (int n = 0;; ++n) {
+    bool have_q = false;
+    for (int n = set;; n += NSET) {
       const int s = n % NS;
       if (!warp_wait(&full[s], (uint32_t)(n / NS) & 1u, p.status)) break;
       const int m = stage_m[s];
       if (m < 0) break;
-      if (n == 0) {   // the group's length and q rows arrived with stage 0
+      if (!have_q) {   // the group's length was stored before any block's copy; q has its own barrier
+        if (!warp_wait(qbar, 0u, p.status)) break;
+        have_q = true;
         L = info[0];
         c = info[1];
         const uint32_t qa_addr = (qrow < G) ? smem_u32(qs + qrow * 256) + (mi >> 1) * 16u : smem_u32(zrow);
@@ -1537,12 +1553,12 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
       const int nk = (m == c) ? (L - m * kBlock) : kBlock;   // keys present in this block
       const uint32_t st = smem_u32(smem + s * kStageBytes);
       bool zeroed = false;
-      if (nk < 16 * warp + 16) {
+      if (nk < 16 * kw + 16) {
         // Rows past the end of the sequence may hold any bits; P is zero there, and
         // zero V rows keep 0 * NaN out of the P V products.
         uint8_t* vs = smem + s * kStageBytes + kMmaTileBytes;
-        const int row0 = max(nk, 16 * warp);
-        for (int i = lane; i < (16 * warp + 16 - row0) * 16; i += 32) {
+        const int row0 = max(nk, 16 * kw);
+        for (int i = lane; i < (16 * kw + 16 - row0) * 16; i += 32) {
           const int row = row0 + i / 16, chunk = i % 16;
           *reinterpret_cast<uint4*>(vs + kv_tile_offset(row, chunk)) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -1570,7 +1586,7 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
         for (int j = 0; j < 2; ++j)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (16 * warp + 8 * j + 2 * tig + (e & 1) >= nk) sacc[j][e] = -INFINITY;
+            if (16 * kw + 8 * j + 2 * tig + (e & 1) >= nk) sacc[j][e] = -INFINITY;
       }
       float mx0 = fmaxf(fmaxf(sacc[0][0], sacc[0][1]), fmaxf(sacc[1][0], sacc[1][1]));
       float mx1 = fmaxf(fmaxf(sacc[0][2], sacc[0][3]), fmaxf(sacc[1][2], sacc[1][3]));
@@ -1620,14 +1636,14 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    // ------------------------------------------------------------ combine the four warps, write o
+    // ------------------------------------------------------------ combine the compute warps, write o
     float l0 = run_l0, l1 = run_l1;
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
-    named_bar_sync(1, 32 * kDecWarps);   // every consumer is done with the ring
+    named_bar_sync(1, 32 * kCw);   // every compute warp is done with the ring
     float* wout = reinterpret_cast<float*>(smem) + warp * (kGrpWarpOut / 4);
     if (tig == 0) {
       comb[(warp * 16 + gid) * 2] = run_m0;
@@ -1640,17 +1656,17 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
       *reinterpret_cast<float2*>(wout + gid * D + nd * 8 + 2 * tig) = make_float2(oacc[nd][0], oacc[nd][1]);
       *reinterpret_cast<float2*>(wout + (gid + 8) * D + nd * 8 + 2 * tig) = make_float2(oacc[nd][2], oacc[nd][3]);
     }
-    named_bar_sync(1, 32 * kDecWarps);
+    named_bar_sync(1, 32 * kCw);
     const float* wall = reinterpret_cast<const float*>(smem);
-    for (int i = tid; i < G * (D / 4); i += 32 * kDecWarps) {
+    for (int i = tid; i < G * (D / 4); i += 32 * kCw) {
       const int h = i / (D / 4), d4 = i % (D / 4);
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, comb[(w * 16 + h) * 2]);
+      for (int w = 0; w < kCw; ++w) M = fmaxf(M, comb[(w * 16 + h) * 2]);
       float den = 0.f;
       float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
+      for (int w = 0; w < kCw; ++w) {
         const float mw = comb[(w * 16 + h) * 2];
         if (mw != -INFINITY) {
           const float a = ex2(mw - M);
@@ -1670,10 +1686,11 @@ __global__ void __launch_bounds__(kGrpThreads, NS <= 3 ? 2 : 1)
     }
   }
   __syncthreads();
-  if (tid == kDecWarps * 32 && *reinterpret_cast<volatile int32_t*>(p.status) != 0) {
+  if (tid == kCw * 32 && *reinterpret_cast<volatile int32_t*>(p.status) != 0) {
     // A wait gave up, so copies may still be in flight: they finish before the CTA
     // exits. Each stage's last fill (a copy or the end marker) is the phase waited
     // for; every earlier phase of the stage completes before it.
+    if (info[3]) mbar_wait_drain(qbar, 0u);
     for (int s = 0; s < NS; ++s)
       if (issued[s] >= 0) mbar_wait_drain(&full[s], (uint32_t)(issued[s] / NS) & 1u);
   }
@@ -1753,31 +1770,33 @@ cudaError_t launch_decode(const DecodeProblem& pb, void* ws, cudaStream_t st) {
     if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
       return e;
     const int NS = (long long)n_bg <= sms ? 6 : 3;
-    const size_t shm = group_layout(NS, pb.K).total + 1024;
+    const size_t shm = group_layout(NS, NS == 6 ? 2 : 1, pb.K).total + 1024;
     if (4LL * (long long)n_bg >= 3LL * sms && shm <= (size_t)smem_max) {
       CUtensorMap tk, tv, tq;
       if (!make_tmap_bf16_3d(&tk, pb.Kc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
           !make_tmap_bf16_3d(&tv, pb.Vc, D, (uint64_t)pb.Lmax, (uint64_t)n_bg, kBlock) ||
           !make_tmap_bf16_rows(&tq, pb.q, D, (uint64_t)pb.B * pb.Hq, (uint32_t)G))
         return cudaErrorInvalidValue;
-      auto group = [&](auto kernel) -> cudaError_t {
+      auto group = [&](auto kernel, int threads) -> cudaError_t {
         cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
         if (r != cudaSuccess) return r;
         r = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared);
         if (r != cudaSuccess) return r;
-        kernel<<<(unsigned)n_bg, kGrpThreads, shm, st>>>(prm, tk, tv, tq);
+        kernel<<<(unsigned)n_bg, threads, shm, st>>>(prm, tk, tv, tq);
         count_launch();
         return cudaGetLastError();
       };
-      if (NS == 6) {
-        if (pb.NBmax <= 128) return group(decode_group_kernel<6, 4>);
-        if (pb.NBmax <= 256) return group(decode_group_kernel<6, 8>);
-        return group(decode_group_kernel<6, 16>);
+      if (NS == 6) {   // one CTA per SM: two sets of compute warps
+        constexpr int t = group_threads<2>();
+        if (pb.NBmax <= 128) return group(decode_group_kernel<6, 2, 4>, t);
+        if (pb.NBmax <= 256) return group(decode_group_kernel<6, 2, 8>, t);
+        return group(decode_group_kernel<6, 2, 16>, t);
       }
-      if (pb.NBmax <= 128) return group(decode_group_kernel<3, 4>);
-      if (pb.NBmax <= 256) return group(decode_group_kernel<3, 8>);
-      return group(decode_group_kernel<3, 16>);
+      constexpr int t = group_threads<1>();   // two CTAs per SM: one set each
+      if (pb.NBmax <= 128) return group(decode_group_kernel<3, 1, 4>, t);
+      if (pb.NBmax <= 256) return group(decode_group_kernel<3, 1, 8>, t);
+      return group(decode_group_kernel<3, 1, 16>, t);
     }
   }
   // Selection first (it also clears the counters); the attention kernel follows.
